@@ -1,0 +1,320 @@
+"""Throughput of the top-1 MoE gate: routed tokens/s for one full step
+(route + forward + backward + aux loss + lambda update) and its fraction of the
+TF32/HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--math tf32|ffma]
+                    [--workload NAME] [--impl native|reference]
+
+One JSON line on rank 0. N > 1 runs under torchrun as N independent replicas
+(one per GPU, each with its own batch: the gate has no cross-GPU exchange),
+timed on the device as the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+if HERE not in sys.path:
+    sys.path.insert(0, HERE)
+
+from bwd_route_b200 import workloads as wl  # noqa: E402
+
+METRIC = "routed tokens/s (fwd+bwd+aux) at 1 B200; % of TF32/HBM roofline"
+UNIT = "tokens/s"
+# nominal dense TF32 / BF16 tensor throughput ratio (1.1 vs 2.25 PFLOP/s)
+TF32_OVER_BF16 = 1.1 / 2.25
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CPU_SAMPLE_TOKENS = 8192
+REF_STEP_TOKENS = 512
+
+
+def load_peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic(spec):
+    """Bytes and flops the method itself must move / compute for one step."""
+    T, E, H = spec.T, spec.E, spec.H
+    step_bytes = T * (4 * (5 * H + 3 * E) + 16) + 2 * E * H * H * 4
+    step_flops = 6 * H * H * T
+    per_kernel_bytes = {
+        # x read, routed written, perm read; W and bias
+        "fwd": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
+        # d_out read, d_x written, perm read; W^T
+        "d_x": T * (8 * H + 4) + E * H * H * 4,
+        # x and d_out read, perm read; dW and db written
+        "wgrad": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
+    }
+    return step_bytes, step_flops, per_kernel_bytes
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period: float = 0.02):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def cpu_oracle_tokens_per_s(inp, n_tokens: int):
+    """The CPU oracle, as it stands, on the first n_tokens tokens of the workload."""
+    import oracle
+    sample = wl.token_sample(inp, n_tokens)
+    t0 = time.perf_counter()
+    oracle.step(sample)
+    dt = time.perf_counter() - t0
+    return sample.spec.T / dt, dt, sample.spec.T
+
+
+def run_reference(args, spec):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = wl.generate(spec)
+    sample_tokens = min(REF_STEP_TOKENS, spec.T)
+    for _ in range(args.warmup):
+        cpu_oracle_tokens_per_s(inp, sample_tokens)
+    times = []
+    for _ in range(args.steps):
+        _, dt, n = cpu_oracle_tokens_per_s(inp, sample_tokens)
+        times.append(dt)
+    per_step = sum(times) / len(times)
+    value = sample_tokens / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "B": spec.B, "N_H": spec.N_H, "E": spec.E, "H": spec.H,
+                   "tokens": spec.T, "math": "fp64 oracle"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"first {sample_tokens} tokens of {spec.name} per step (route, forward, "
+                                   f"d_x, dW/db, aux) in plain single-threaded C, fp64 accumulation"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--math", choices=["tf32", "ffma"], default="tf32")
+    ap.add_argument("--workload", default=wl.THROUGHPUT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    spec = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, spec)
+        return
+    args.warmup = max(args.warmup, 3)
+
+    import torch
+    import torch.distributed as dist
+
+    from bwd_route_b200 import ops
+    from bwd_route_b200.gate import MoETop1Gate
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    math_mode = ops.MOE_MATH_TF32 if args.math == "tf32" else ops.MOE_MATH_FFMA
+    inp = wl.generate(spec)
+    T, E, H = spec.T, spec.E, spec.H
+    logits = torch.from_numpy(inp.gate_logits).to(dev)
+    x = torch.from_numpy(inp.x).to(dev)
+    d_out = torch.from_numpy(inp.d_out).to(dev)
+    W = torch.from_numpy(inp.W).to(dev)
+    bias = torch.from_numpy(inp.bias).to(dev)
+    gate = MoETop1Gate(W, bias, spec.B, spec.N_H, math_mode, inp.lambda_floor, inp.lambda_max_extra,
+                       inp.ent_target, inp.ent_ema)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        # the backward is issued as two calls (d_x; dW and db) so that each
+        # contraction kernel can be timed on its own
+        if ev:
+            ev[0].record(stream)
+        gate.route(logits)
+        if ev:
+            ev[1].record(stream)
+        gate.forward(x)
+        if ev:
+            ev[2].record(stream)
+        ops.moe_top1_bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, gate.d_x, None, None, 0,
+                         gate.ws)
+        if ev:
+            ev[3].record(stream)
+        ops.moe_top1_bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, None, gate.dW, gate.db, 0,
+                         gate.ws)
+        if ev:
+            ev[4].record(stream)
+        gate.aux(logits)
+        gate.update_lambda()
+        if ev:
+            ev[5].record(stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    flags = ops.moe_top1_device_flags(gate.ws)
+    if flags:
+        raise RuntimeError(f"device flags set during warm-up: {flags:#x}")
+
+    # timed region: K whole steps, events on the launching stream
+    per_call = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for k in range(args.steps):
+            step(per_call[k])
+        end.record(stream)
+        barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    names = ["route", "fwd", "d_x", "wgrad", "aux+lambda"]
+    call_ms = {n: sum(per_call[k][i].elapsed_time(per_call[k][i + 1]) for k in range(args.steps)) / args.steps
+               for i, n in enumerate(names)}
+    flags = ops.moe_top1_device_flags(gate.ws)
+
+    # end to end through the public API: inputs from pinned host memory, loss back to the host
+    h_logits = torch.from_numpy(inp.gate_logits).pin_memory()
+    h_x = torch.from_numpy(inp.x).pin_memory()
+    h_dout = torch.from_numpy(inp.d_out).pin_memory()
+    h_loss = torch.empty(2, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        logits.copy_(h_logits, non_blocking=True)
+        x.copy_(h_x, non_blocking=True)
+        d_out.copy_(h_dout, non_blocking=True)
+        gate.step(logits, x, d_out)
+        h_loss.copy_(gate.loss, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        step_bytes, step_flops, kbytes = algorithmic(spec)
+        hbm = float(peaks["hbm_gbs"])
+        tf32_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * TF32_OVER_BF16
+        t_roof = max(step_bytes / (hbm * 1e9), step_flops / (tf32_sus * 1e12))
+        value = world * T / (ms_per_step * 1e-3)
+        dominant = max(["fwd", "d_x", "wgrad"], key=lambda n: call_ms[n])
+        achieved = kbytes[dominant] / (call_ms[dominant] * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": spec.name, "B": spec.B, "N_H": spec.N_H, "E": E, "H": H, "tokens": T,
+                       "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (x, d_out, routed, d_x: 4 x %.2f GB), no flush" % (T * H * 4 / 1e9)},
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": None, "peak_source": f"{peak_kind} hbm_gbs"},
+            "step_roofline": {"bytes": step_bytes, "flops": step_flops, "t_roofline_ms": t_roof * 1e3,
+                              "frac": t_roof * 1e3 / ms_per_step,
+                              "peaks": {"hbm_gbs": hbm, "tf32_tflops": tf32_sus,
+                                        "source": f"{peak_kind}; tf32 = bf16_tflops_sustained x 1.1/2.25"}},
+            "per_call_ms": call_ms,
+            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
+                    "h2d_bytes_per_step": T * (E + 2 * H) * 4, "d2h_bytes_per_step": 8},
+            "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode),
+            "clocks": clocks.summary(),
+            "device_flags": flags,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, dt, n = cpu_oracle_tokens_per_s(inp, CPU_SAMPLE_TOKENS)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": f"first {n} tokens of {spec.name}: route, forward, d_x, dW/db and "
+                                              f"aux in plain single-threaded C (fp64 accumulation), {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

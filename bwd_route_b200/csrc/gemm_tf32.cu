@@ -1,0 +1,525 @@
+// gemm_tf32.cu -- tcgen05 (5th-generation tensor core) TF32 kernels of the
+// expert contractions, fed by TMA, accumulating in tensor memory (TMEM).
+//
+// foxhunt commit 11b96dac6a ("Top-1 Mixture-of-Experts gate per Switch
+// Transformer"), kernel list / PERFORMANCE: the forward applies the selected
+// expert's [H, H] linear (routed[t,o] = sum_i W[e*,o,i] x[t,i] + b[e*,o]); the
+// backward runs the chain rule through the selected expert only
+// (d_x[t,i] = sum_o W[e*,o,i] d_out[t,o]; dW[e,o,i] = sum_{t in e} d_out[t,o]
+// x[t,i]; db[e,o] = sum_{t in e} d_out[t,o]). The pages give one block per
+// token and one thread per output channel; here the tokens of an expert are
+// contiguous in the routing permutation, so each expert is a dense GEMM:
+//
+//   grouped_tf32_kernel : persistent, one CTA per SM. A tile is 128 sorted
+//     tokens x all H outputs. Warp 0 gathers the tile's token rows with TMA
+//     tile::gather4 (128-byte swizzle) and loads the expert's weight slab with a
+//     2D TMA box; warp 1 issues tcgen05.mma kind::tf32 (M=128, N=H, K=8) into
+//     one of two TMEM accumulators; warps 2-5 drain the other accumulator
+//     (tcgen05.ld), add the bias, and store the rows back to their original
+//     token positions with coalesced 128-byte stores.
+//
+//   wgrad_tf32_kernel : one CTA per range of the sorted token list (range c of
+//     expert e -> partial-sum slot c + e). Both operands are MN-major (tokens
+//     are the contraction index): the CTA gathers 32 tokens of d_out and x per
+//     stage and issues M=128 x N=H MMAs with the whole dW[e] (H x H fp32) held
+//     in TMEM. Warps 2-5 sum d_out over the same staged tokens for db, then
+//     drain the accumulator into the slot. A separate kernel adds the slots in
+//     a fixed pairwise order (no atomics: foxhunt commit b23f8f2efa,
+//     Discipline).
+//
+// The tensor core reads each fp32 operand as TF32 (its 10 leading mantissa
+// bits) and accumulates in fp32. Every pipeline wait is bounded (common.cuh).
+#include <cstdint>
+#include <cstdio>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-5: epilogue
+constexpr int kMaxStages = 8;
+
+struct __align__(8) Ctl {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort;
+    int off[33];
+    int tstart[33];
+};
+
+// ------------------------------------------------------------------ grouped GEMM
+template <int H>
+struct GCfg {
+    static constexpr int BM = 128;
+    static constexpr int KCH = H / 32;                // 32 fp32 = one 128-byte swizzle row
+    static constexpr int A_BYTES = BM * 128;          // 16 KiB
+    static constexpr int B_BYTES = H * 128;           // 16 / 32 KiB
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (H == 256) ? 4 : 6;
+    static constexpr int STG_BYTES = 4 * 32 * 128;    // epilogue staging: 4 warps x 32 rows x 128 B
+    static constexpr int TMEM_COLS = 2 * H;           // two accumulators
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + static_cast<int>(sizeof(Ctl));
+    static_assert(STAGES <= kMaxStages, "stages");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ int find_expert(const int* tstart, int E, int tile) {
+    int e = 0;
+    while (e + 1 < E && tstart[e + 1] <= tile) ++e;
+    return e;
+}
+
+template <int H>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_constant__ CUtensorMap tm_b,
+                    const float* __restrict__ bias, const int32_t* __restrict__ offsets,
+                    const int32_t* __restrict__ perm, int T, int E, int accumulate, float* __restrict__ out,
+                    uint32_t* __restrict__ dev_flags) {
+    using C = GCfg<H>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    float* stg = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], 4);
+        }
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_src);
+        tma_prefetch_desc(&tm_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ts = 0;
+        for (int e = 0; e < E; ++e) {
+            ctl->tstart[e] = ts;
+            ts += (ctl->off[e + 1] - ctl->off[e] + C::BM - 1) / C::BM;
+        }
+        ctl->tstart[E] = ts;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    const int ntiles = ctl->tstart[E];
+    volatile int* abort = &ctl->abort;
+
+    if (warp == 0) {
+        // ---------------- TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int e = find_expert(ctl->tstart, E, tile);
+            const int row0 = ctl->off[e] + (tile - ctl->tstart[e]) * C::BM;
+            const int nrows = min(C::BM, ctl->off[e + 1] - row0);
+            int tok[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = 4 * lane + j;
+                tok[j] = (r < nrows) ? perm[row0 + r] : T;  // row T is outside the tensor: zeros
+            }
+            bool ok = true;
+            for (int kc = 0; kc < C::KCH && ok; ++kc) {
+                if (lane == 0) ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                uint8_t* a = stages + stage * C::STAGE_BYTES;
+                if (lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
+                __syncwarp();
+                tma_gather4(a + lane * 512, &tm_src, kc * 32, tok[0], tok[1], tok[2], tok[3], &ctl->full[stage]);
+                if (lane == 0) tma_load_2d(a + C::A_BYTES, &tm_b, kc * 32, e * H, &ctl->full[stage]);
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (!ok) break;
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one thread)
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_tf32(128, H, 0, 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                if (!(ok = mbar_wait(&ctl->tempty[acc], acc_phase ^ 1, abort, dev_flags))) break;
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(acc * H);
+                for (int kc = 0; kc < C::KCH; ++kc) {
+                    if (!(ok = mbar_wait(&ctl->full[stage], phase, abort, dev_flags))) break;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(stages + stage * C::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_tf32(d, sw128_desc(a_addr + ks * 32, 16, 1024), sw128_desc(b_addr + ks * 32, 16, 1024),
+                                 idesc, (kc | ks) != 0 ? 1u : 0u);
+                    mma_commit(&ctl->empty[stage]);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue: TMEM -> registers -> smem transpose -> rows
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        float* my = stg + (warp - 2) * 32 * 32;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int e = find_expert(ctl->tstart, E, tile);
+            const int row0 = ctl->off[e] + (tile - ctl->tstart[e]) * C::BM;
+            const int nrows = min(C::BM, ctl->off[e + 1] - row0);
+            const int myrow = 32 * q + lane;
+            const int tok_mine = (myrow < nrows) ? perm[row0 + myrow] : -1;
+            if (!mbar_wait(&ctl->tfull[acc], acc_phase, abort, dev_flags)) break;
+            __syncwarp();
+            tc_fence_after();
+            const int j = lane & 7;
+#pragma unroll 1
+            for (int c = 0; c < H / 32; ++c) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * H + c * 32), v);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    *reinterpret_cast<float4*>(my + lane * 32 + ((jj ^ (lane & 7)) * 4)) =
+                        make_float4(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3]);
+                __syncwarp();
+                float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (bias) bv = __ldg(reinterpret_cast<const float4*>(bias + static_cast<int64_t>(e) * H + c * 32) + j);
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int R = it * 4 + (lane >> 3);
+                    float4 val = *reinterpret_cast<const float4*>(my + R * 32 + ((j ^ (R & 7)) * 4));
+                    const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
+                    if (tok >= 0) {
+                        val.x += bv.x;
+                        val.y += bv.y;
+                        val.z += bv.z;
+                        val.w += bv.w;
+                        float* dst = out + static_cast<int64_t>(tok) * H + c * 32 + j * 4;
+                        if (accumulate) {
+                            const float4 o = *reinterpret_cast<const float4*>(dst);
+                            val.x += o.x;
+                            val.y += o.y;
+                            val.z += o.z;
+                            val.w += o.w;
+                            *reinterpret_cast<float4*>(dst) = val;
+                        } else {
+                            st_global_cs_v4(dst, val);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ weight gradient
+template <int H>
+struct WCfg {
+    static constexpr int KT = 32;                    // tokens per stage (4 MMAs of K = 8)
+    static constexpr int G = H / 32;                 // 128-byte column groups
+    static constexpr int GROUP_BYTES = KT * 128;     // one group: KT rows x 128 B (4 KiB)
+    static constexpr int OP_BYTES = G * GROUP_BYTES; // one operand per stage
+    static constexpr int STAGE_BYTES = 2 * OP_BYTES; // d_out then x
+    static constexpr int STAGES = (H == 256) ? 3 : 6;
+    static constexpr int MH = H / 128;               // 128-row halves of dW
+    static constexpr int TMEM_COLS = MH * H;
+    static constexpr int STG_BYTES = 4 * 32 * 128;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + static_cast<int>(sizeof(Ctl));
+    static_assert(STAGES <= kMaxStages, "stages");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+    static_assert((2 * G) % 4 == 0, "gather split");
+};
+
+template <int H>
+__global__ void __launch_bounds__(kThreads, 1)
+wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x,
+                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int T, int E, int P,
+                  float* __restrict__ part, float* __restrict__ part_db, uint32_t* __restrict__ dev_flags) {
+    using C = WCfg<H>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    float* stg = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1 + 4);  // MMA commit + the four db warps
+        }
+        mbar_init(&ctl->tfull[0], 1);
+        mbar_init(&ctl->tempty[0], 4);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_g);
+        tma_prefetch_desc(&tm_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+    const int lo = static_cast<int>(split_lo(c, T, P)), hi = static_cast<int>(split_lo(c + 1, T, P));
+
+    if (warp == 0) {
+        // ---------------- TMA producer: 32 tokens of d_out and x per stage
+        const int jq = lane & 7;          // which 4-token quad this lane gathers
+        const int combo0 = lane >> 3;     // first (operand, group) combination
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int e = 0; e < E && ok; ++e) {
+            const int s = max(lo, ctl->off[e]), t = min(hi, ctl->off[e + 1]);
+            for (int p0 = s; p0 < t; p0 += C::KT) {
+                const int tok_lane = (p0 + lane < t) ? perm[p0 + lane] : T;  // row T reads zeros
+                int r[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) r[k] = __shfl_sync(0xffffffffu, tok_lane, 4 * jq + k);
+                if (lane == 0) ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                uint8_t* base = stages + stage * C::STAGE_BYTES;
+                if (lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
+                __syncwarp();
+#pragma unroll
+                for (int m = 0; m < (2 * C::G) / 4; ++m) {
+                    const int combo = combo0 + 4 * m;
+                    const int operand = combo / C::G, g = combo % C::G;
+                    tma_gather4(base + operand * C::OP_BYTES + g * C::GROUP_BYTES + jq * 512,
+                                operand == 0 ? &tm_g : &tm_x, g * 32, r[0], r[1], r[2], r[3], &ctl->full[stage]);
+                }
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_tf32(128, H, 1, 1);  // both operands MN-major
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int e = 0; e < E && ok; ++e) {
+                const int s = max(lo, ctl->off[e]), t = min(hi, ctl->off[e + 1]);
+                if (s >= t) continue;
+                if (!(ok = mbar_wait(&ctl->tempty[0], acc_phase ^ 1, abort, dev_flags))) break;
+                tc_fence_after();
+                bool first = true;
+                for (int p0 = s; p0 < t; p0 += C::KT) {
+                    if (!(ok = mbar_wait(&ctl->full[stage], phase, abort, dev_flags))) break;
+                    tc_fence_after();
+                    const uint32_t g_addr = smem_u32(stages + stage * C::STAGE_BYTES);
+                    const uint32_t x_addr = g_addr + C::OP_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+                        for (int mh = 0; mh < C::MH; ++mh) {
+                            const uint64_t adesc = sw128_desc(g_addr + mh * 4 * C::GROUP_BYTES + ks * 1024, C::GROUP_BYTES, 1024);
+                            const uint64_t bdesc = sw128_desc(x_addr + ks * 1024, C::GROUP_BYTES, 1024);
+                            mma_tf32(tmem + static_cast<uint32_t>(mh * H), adesc, bdesc, idesc,
+                                     (first && ks == 0) ? 0u : 1u);
+                        }
+                    }
+                    first = false;
+                    mma_commit(&ctl->empty[stage]);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->tfull[0]);
+                acc_phase ^= 1;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- db over the staged d_out rows, then drain dW to the slot
+        const int tid = threadIdx.x - 64;  // 0..127: owns d_out column o = tid (and tid + 128)
+        const int q = warp & 3;
+        float* my = stg + (warp - 2) * 32 * 32;
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int e = 0; e < E && ok; ++e) {
+            const int s = max(lo, ctl->off[e]), t = min(hi, ctl->off[e + 1]);
+            if (s >= t) continue;
+            float db0 = 0.0f, db1 = 0.0f;
+            for (int p0 = s; p0 < t; p0 += C::KT) {
+                if (!(ok = mbar_wait(&ctl->full[stage], phase, abort, dev_flags))) break;
+                const uint8_t* gt = stages + stage * C::STAGE_BYTES;
+#pragma unroll
+                for (int h = 0; h < C::MH; ++h) {
+                    const int o = tid + 128 * h;
+                    const int g = o >> 5, jo = o & 31;
+                    const uint8_t* colbase = gt + g * C::GROUP_BYTES + (jo & 3) * 4;
+                    float acc = 0.0f;
+#pragma unroll 8
+                    for (int rr = 0; rr < C::KT; ++rr)
+                        acc += *reinterpret_cast<const float*>(colbase + rr * 128 + (((jo >> 2) ^ (rr & 7)) << 4));
+                    if (h == 0) db0 += acc; else db1 += acc;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->empty[stage]);
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (!ok) break;
+            if (!(ok = mbar_wait(&ctl->tfull[0], acc_phase, abort, dev_flags))) break;
+            __syncwarp();
+            tc_fence_after();
+            const int64_t slot = static_cast<int64_t>(c) + e;
+            const int j = lane & 7;
+#pragma unroll 1
+            for (int mh = 0; mh < C::MH; ++mh) {
+#pragma unroll 1
+                for (int cc = 0; cc < H / 32; ++cc) {
+                    float v[32];
+                    tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(mh * H + cc * 32), v);
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        *reinterpret_cast<float4*>(my + lane * 32 + ((jj ^ (lane & 7)) * 4)) =
+                            make_float4(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int it = 0; it < 8; ++it) {
+                        const int R = it * 4 + (lane >> 3);
+                        const float4 val = *reinterpret_cast<const float4*>(my + R * 32 + ((j ^ (R & 7)) * 4));
+                        const int o = mh * 128 + 32 * q + R;
+                        *reinterpret_cast<float4*>(part + (slot * H + o) * H + cc * 32 + j * 4) = val;
+                    }
+                    __syncwarp();
+                }
+            }
+            part_db[slot * H + tid] = db0;
+            if (C::MH == 2) part_db[slot * H + tid + 128] = db1;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[0]);
+            acc_phase ^= 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float* bias, const int32_t* offsets,
+                                const int32_t* perm, int64_t T, int E, int H, int accumulate, float* out,
+                                uint32_t* dev_flags, int num_sms, cudaStream_t s) {
+    CUtensorMap tm_a, tm_b;
+    if (!make_map_2d(&tm_a, src, static_cast<uint64_t>(T), H, 32, 1)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&tm_b, Bsrc, static_cast<uint64_t>(E) * H, H, 32, H)) return cudaErrorInvalidValue;
+    const int64_t tiles = (T + 127) / 128 + E;
+    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    cudaError_t err;
+    if (H == 256) {
+        err = set_smem(grouped_tf32_kernel<256>, GCfg<256>::SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        grouped_tf32_kernel<256><<<grid, kThreads, GCfg<256>::SMEM_BYTES, s>>>(
+            tm_a, tm_b, bias, offsets, perm, static_cast<int>(T), E, accumulate, out, dev_flags);
+    } else {
+        err = set_smem(grouped_tf32_kernel<128>, GCfg<128>::SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        grouped_tf32_kernel<128><<<grid, kThreads, GCfg<128>::SMEM_BYTES, s>>>(
+            tm_a, tm_b, bias, offsets, perm, static_cast<int>(T), E, accumulate, out, dev_flags);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
+                              int64_t T, int E, int H, float* part, float* part_db, uint32_t* dev_flags,
+                              cudaStream_t s) {
+    CUtensorMap tm_g, tm_x;
+    if (!make_map_2d(&tm_g, d_out, static_cast<uint64_t>(T), H, 32, 1)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&tm_x, x, static_cast<uint64_t>(T), H, 32, 1)) return cudaErrorInvalidValue;
+    const int P = wgrad_splits(T);
+    cudaError_t err;
+    if (H == 256) {
+        err = set_smem(wgrad_tf32_kernel<256>, WCfg<256>::SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        wgrad_tf32_kernel<256><<<P, kThreads, WCfg<256>::SMEM_BYTES, s>>>(tm_g, tm_x, offsets, perm,
+                                                                         static_cast<int>(T), E, P, part, part_db,
+                                                                         dev_flags);
+    } else {
+        err = set_smem(wgrad_tf32_kernel<128>, WCfg<128>::SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        wgrad_tf32_kernel<128><<<P, kThreads, WCfg<128>::SMEM_BYTES, s>>>(tm_g, tm_x, offsets, perm,
+                                                                         static_cast<int>(T), E, P, part, part_db,
+                                                                         dev_flags);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

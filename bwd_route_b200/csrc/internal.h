@@ -1,0 +1,121 @@
+// internal.h -- host-side declarations shared by the kernel files and the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+// Tokens handled by one block of the routing and aux kernels.
+constexpr int kRouteTokPerBlk = 1024;
+constexpr int kAuxTokPerBlk = 1024;
+
+// Weight-gradient contraction: the expert-sorted token list is cut into
+// `wgrad_splits(T)` equal ranges (further cut at expert boundaries); range c
+// of expert e produces partial sum slot c + e. The split count depends on T
+// only, so the reduction tree -- and hence every bit of dW and db -- is fixed
+// for a given routing.
+constexpr int kWgradMaxSplits = 148;
+constexpr int kWgradMinTokPerSplit = 256;
+inline int wgrad_splits(int64_t T) {
+    int64_t p = (T + kWgradMinTokPerSplit - 1) / kWgradMinTokPerSplit;
+    if (p < 1) p = 1;
+    if (p > kWgradMaxSplits) p = kWgradMaxSplits;
+    return static_cast<int>(p);
+}
+// First sorted position of split c (floor(c * T / P)); ranges are [lo(c), lo(c+1)).
+__host__ __device__ inline int64_t split_lo(int c, int64_t T, int P) { return (static_cast<int64_t>(c) * T) / P; }
+
+struct WsLayout {
+    size_t flags = 0;        // uint32 flag word (256 B reserved)
+    size_t route_counts = 0; // int32 [nblk_route][E]
+    size_t route_base = 0;   // int32 [nblk_route][E]
+    size_t aux_psum = 0;     // float [nblk_aux][E]
+    size_t w_t = 0;          // float [E][H][H]  transposed expert weights (TF32 d_x)
+    size_t wg_part = 0;      // float [P + E][H][H] dW partial sums
+    size_t wg_part_db = 0;   // float [P + E][H]    db partial sums
+    size_t route_end = 0;    // bytes the routing / aux calls need
+    size_t total = 0;        // bytes every call needs
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int64_t T, int E, int H) {
+    WsLayout L;
+    const int64_t nr = T > 0 ? (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk : 1;
+    const int64_t na = T > 0 ? (T + kAuxTokPerBlk - 1) / kAuxTokPerBlk : 1;
+    const int P = wgrad_splits(T);
+    size_t off = 0;
+    L.flags = off;
+    off += 256;
+    L.route_counts = off;
+    off = align_up(off + sizeof(int32_t) * nr * E, 256);
+    L.route_base = off;
+    off = align_up(off + sizeof(int32_t) * nr * E, 256);
+    L.aux_psum = off;
+    off = align_up(off + sizeof(float) * na * E, 256);
+    L.route_end = off;
+    if (H > 0) {
+        L.w_t = off;
+        off = align_up(off + sizeof(float) * static_cast<size_t>(E) * H * H, 256);
+        L.wg_part = off;
+        off = align_up(off + sizeof(float) * static_cast<size_t>(P + E) * H * H, 256);
+        L.wg_part_db = off;
+        off = align_up(off + sizeof(float) * static_cast<size_t>(P + E) * H, 256);
+    }
+    L.total = off;
+    return L;
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns the cudaError_t of its launch(es).
+cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_idx, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, int32_t* blk_counts, int32_t* blk_base,
+                         cudaStream_t s);
+
+cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, int E, const float* lambda_eff,
+                       float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,
+                       cudaStream_t s);
+
+cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float lambda_max_extra, float ent_target,
+                              float* lambda_eff, cudaStream_t s);
+
+// out[perm[r], n] = sum_k src[perm[r], k] * B_e[n, k] (+ bias[e, n]) for the
+// sorted rows r of expert e. b_kmajor = 1: B_e[n, k] = Wsrc[e][n][k] (forward);
+// b_kmajor = 0: B_e[n, k] = Wsrc[e][k][n] (input gradient).
+cudaError_t launch_grouped_ffma(const float* src, const float* Wsrc, const float* bias, const int32_t* offsets,
+                                const int32_t* perm, int64_t T, int E, int H, int b_kmajor, int accumulate,
+                                float* out, cudaStream_t s);
+
+// Same contraction on tcgen05 (TF32 in, FP32 accumulate). Bsrc is [E][H][H]
+// with Bsrc[e][n][k] = B_e[n, k] (K-major).
+cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float* bias, const int32_t* offsets,
+                                const int32_t* perm, int64_t T, int E, int H, int accumulate, float* out,
+                                uint32_t* dev_flags, int num_sms, cudaStream_t s);
+
+cudaError_t launch_transpose_w(const float* W, int E, int H, float* Wt, cudaStream_t s);
+
+// Per-range partial sums of dW / db into the slot buffers (see wgrad_splits).
+cudaError_t launch_wgrad_ffma(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
+                              int64_t T, int E, int H, float* part, float* part_db, cudaStream_t s);
+cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
+                              int64_t T, int E, int H, float* part, float* part_db, uint32_t* dev_flags,
+                              cudaStream_t s);
+// Fixed-order pairwise sum of the slots of each expert into dW / db (either may be null).
+cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const int32_t* offsets, int64_t T,
+                                int E, int H, float* dW, float* db, int acc_dw, int acc_db, cudaStream_t s);
+
+// Driver entry point for tensor-map encoding (resolved at run time, so the
+// library does not link libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+// 2D fp32 tensor [rows][cols] with a 128-byte-swizzled box of box_cols x box_rows.
+bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                 uint32_t box_rows);
+
+}  // namespace moe

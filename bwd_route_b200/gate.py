@@ -1,0 +1,78 @@
+"""One full pass of the top-1 MoE gate through the C ABI.
+
+MoETop1Gate owns the device buffers (allocated with torch: plumbing only) and
+runs, in stream order, the five library calls of a training step:
+
+    moe_top1_route -> moe_top1_fwd -> moe_top1_bwd -> moe_aux_loss_fwd_bwd
+    -> moe_lambda_eff_update
+
+The step mirrors the training loop of foxhunt commit 9170d24fe3 ("Single
+source of truth for the attention path", PerceptionTrainer integration):
+forward through the MoE dispatch, backward through it, then the load-balance
+loss, whose weight lambda_eff is read from device memory and updated by the
+controller of foxhunt commit 2d0e6b6bdc at the end of the step.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import ops
+
+
+class MoETop1Gate:
+    # kernels launched per step() with T > 0: route 3, fwd 1, bwd (TF32: transpose +
+    # d_x + wgrad + reduce = 4; FFMA: d_x + wgrad + reduce = 3), aux 2, lambda 1
+    @staticmethod
+    def launches_per_step(math: int) -> int:
+        return 3 + 1 + (4 if math == ops.MOE_MATH_TF32 else 3) + 2 + 1
+
+    def __init__(self, W: torch.Tensor, bias: torch.Tensor, B: int, N_H: int, math: int = ops.MOE_MATH_TF32,
+                 lambda_floor: float = 0.01, lambda_max_extra: float = 0.09, ent_target: float = 1.0,
+                 ent_ema: float = 0.0, stats: bool = True):
+        assert W.is_cuda and W.dtype == torch.float32 and W.dim() == 3
+        self.E, self.H = W.shape[0], W.shape[1]
+        self.B, self.N_H, self.T = B, N_H, B * N_H
+        self.math = math
+        self.W, self.bias = W, bias
+        dev = W.device
+        f32 = torch.float32
+        T, E, H = self.T, self.E, self.H
+        self.lambda_floor, self.lambda_max_extra, self.ent_target = lambda_floor, lambda_max_extra, ent_target
+        self.routing = ops.Routing.empty(T, E, dev)
+        self.routed = torch.empty(T, H, dtype=f32, device=dev)
+        self.d_x = torch.empty(T, H, dtype=f32, device=dev)
+        self.dW = torch.empty(E, H, H, dtype=f32, device=dev)
+        self.db = torch.empty(E, H, dtype=f32, device=dev)
+        self.d_logits = torch.empty(T, E, dtype=f32, device=dev)
+        self.loss = torch.zeros(2, dtype=f32, device=dev)
+        self.mean_p = torch.zeros(E, dtype=f32, device=dev)
+        self.stats = torch.zeros(3 * E + 4, dtype=f32, device=dev) if stats else None
+        self.lambda_eff = torch.full((1,), lambda_floor, dtype=f32, device=dev)
+        self.ent_ema = torch.full((1,), ent_ema, dtype=f32, device=dev)
+        self.ws = ops.new_workspace(T, E, H, dev)
+
+    def route(self, gate_logits, stream=None):
+        ops.moe_top1_route(gate_logits, self.B, self.N_H, self.E, self.routing, self.ws, stream)
+
+    def forward(self, x, stream=None):
+        ops.moe_top1_fwd(x, self.W, self.bias, self.routing, self.B, self.N_H, self.E, self.H, self.math,
+                         self.routed, self.ws, stream)
+
+    def backward(self, x, d_out, stream=None):
+        ops.moe_top1_bwd(x, self.W, d_out, self.routing, self.B, self.N_H, self.E, self.H, self.math, self.d_x,
+                         self.dW, self.db, 0, self.ws, stream)
+
+    def aux(self, gate_logits, stream=None):
+        ops.moe_aux_loss_fwd_bwd(gate_logits, self.routing.counts, self.B, self.N_H, self.E, self.lambda_eff,
+                                 self.d_logits, self.loss, self.mean_p, self.stats, self.ws, stream)
+
+    def update_lambda(self, stream=None):
+        ops.moe_lambda_eff_update(self.ent_ema, self.lambda_floor, self.lambda_max_extra, self.ent_target,
+                                  self.lambda_eff, stream)
+
+    def step(self, gate_logits, x, d_out, stream=None):
+        self.route(gate_logits, stream)
+        self.forward(x, stream)
+        self.backward(x, d_out, stream)
+        self.aux(gate_logits, stream)
+        self.update_lambda(stream)

@@ -1,0 +1,196 @@
+/*
+ * moe_top1.h -- C ABI of the B200 (sm_100a) top-1 mixture-of-experts gate.
+ *
+ * The gate routes each of T = B * N_H context tokens to the expert whose gate
+ * logit is largest and applies that expert's [H, H] linear with bias; its
+ * backward sends gradients through the selected expert only; a load-balance
+ * auxiliary loss, scaled by an adaptive lambda, gives the gate its gradient.
+ *
+ * Sources (page title, section):
+ *   [P1] foxhunt commit 11b96dac6a, "Top-1 Mixture-of-Experts gate per Switch
+ *        Transformer": kernel list, ARCHITECTURE, PERFORMANCE.
+ *   [P2] foxhunt commit 2d0e6b6bdc, "Replace static moe_lambda=0.01 with a
+ *        GPU-driven controller": formula, Wiring.
+ *   [P3] foxhunt commit b23f8f2efa, "Local L40S profile": reduce_axis0 and
+ *        Discipline (block tree-reduce, no atomicAdd).
+ *   [P5] foxhunt commit 9170d24fe3, "Single source of truth for the attention
+ *        path": MHA additions (d_ctx must not alias other gradients),
+ *        PerceptionTrainer integration (capture-safe zero_grads at step start).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  All tensors are dense, row-major, fp32 unless stated. Token t of
+ *   sample b and horizon h is row t = b * N_H + h. gate_logits [T, E];
+ *   x, d_out, routed, d_x [T, H]; W [E, H, H] with W[e][o][i] (row o = output
+ *   channel, column i = input channel, so y = W x); bias, db [E, H];
+ *   dW [E, H, H] like W.
+ * Pointers.  Every tensor pointer is a DEVICE pointer owned by the caller; the
+ *   library never allocates, frees or copies to the host, and never
+ *   synchronises (except moe_top1_device_flags). Float tensors must be 16-byte
+ *   aligned. `stream` is a cudaStream_t (NULL = legacy default stream); all work
+ *   is enqueued on it in order, so the calls can be captured in a CUDA graph.
+ * Workspace.  `workspace` is caller-owned device memory of at least
+ *   moe_top1_workspace_bytes(T, E, H) bytes, 256-byte aligned, initialised once
+ *   with moe_top1_workspace_init. Calls that share a workspace must be ordered
+ *   on one stream.
+ * Shapes.  1 <= E <= 32; 0 <= T < 2^31 - 256; H a multiple of 32 with
+ *   32 <= H <= 256 for MOE_MATH_FFMA, H = 128 or 256 for MOE_MATH_TF32.
+ * Errors.  Arguments are validated on the host before anything is launched; a
+ *   bad argument returns a status and enqueues nothing. A launch error returns
+ *   MOE_ERR_CUDA. A kernel that gives up on a bounded wait records a bit in the
+ *   workspace flag word (read with moe_top1_device_flags) instead of hanging.
+ * Determinism.  For the same inputs, math mode and device every output is
+ *   bitwise identical from run to run: reductions use fixed-order trees and no
+ *   floating-point atomics ([P3] Discipline).
+ */
+#ifndef MOE_TOP1_H
+#define MOE_TOP1_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_TOP1_ABI_VERSION 1
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,       /* null pointer where one is required, negative size, bad scalar */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2, /* E, H or T outside the supported range */
+    MOE_ERR_MISALIGNED = 3,        /* a float tensor or the workspace is not aligned */
+    MOE_ERR_ALIAS = 4,             /* an output overlaps another output or an input */
+    MOE_ERR_WORKSPACE = 5,         /* workspace missing or smaller than required */
+    MOE_ERR_CUDA = 6,              /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE_CHECK = 7       /* (moe_top1_device_flags) a kernel recorded a failure */
+} moe_status_t;
+
+typedef enum {
+    MOE_MATH_TF32 = 0, /* tcgen05 tensor cores, TF32 inputs, FP32 accumulation */
+    MOE_MATH_FFMA = 1  /* FP32 fused multiply-add on the CUDA cores */
+} moe_math_t;
+
+/* Bits of the device flag word. */
+#define MOE_FLAG_WAIT_TIMEOUT 0x1u  /* a pipeline wait ran past its bound */
+
+/* Routing result: caller-owned device buffers. */
+typedef struct {
+    int32_t* expert_idx; /* [T]     selected expert of each token */
+    int32_t* counts;     /* [E]     tokens routed to each expert */
+    int32_t* offsets;    /* [E + 1] exclusive prefix sum of counts; offsets[E] = T */
+    int32_t* perm;       /* [T]     tokens grouped by expert, ascending t inside a group */
+} moe_routing_t;
+
+/* Bytes of workspace that every entry point below needs for T tokens, E experts,
+ * H channels (the maximum over all entry points and math modes). */
+size_t moe_top1_workspace_bytes(int64_t T, int32_t E, int32_t H);
+
+/* Clears the workspace flag word (enqueued on `stream`). */
+moe_status_t moe_top1_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Routing. [P1] kernel list ("select top-1 expert from gate_logits") and
+ * PERFORMANCE ("Top-1 chosen by thread 0 per block"): the expert of token t is
+ * the argmax over e of gate_logits[t, e]; on a tie the lowest index wins (the
+ * result of a scan from e = 0 that moves only on a strictly greater value, so a
+ * NaN at e = 0 selects expert 0 and a NaN elsewhere is never selected).
+ * Also writes counts, offsets and the stable permutation perm (the r-th token
+ * of expert e, in ascending t, is perm[offsets[e] + r]). Integer results are
+ * exact. Needs the workspace.
+ */
+moe_status_t moe_top1_route(const float* gate_logits, int64_t B, int64_t N_H, int32_t E,
+                            const moe_routing_t* out, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * Forward. [P1] kernel list ("apply its [H, H] linear to fused_ctx") and
+ * PERFORMANCE (one output channel = a dot product over the H inputs):
+ *   routed[t, o] = sum_i W[e*, o, i] * x[t, i] + bias[e*, o],  e* = expert_idx[t].
+ * `routing` is the result of moe_top1_route on the same tokens (device
+ * pointers; only offsets and perm are read). routed is overwritten and must
+ * not overlap x, W or bias. MOE_MATH_TF32 rounds x and W to TF32 inside the
+ * tensor core and accumulates in FP32; MOE_MATH_FFMA multiplies in FP32.
+ */
+moe_status_t moe_top1_fwd(const float* x, const float* W, const float* bias,
+                          const moe_routing_t* routing, int64_t B, int64_t N_H, int32_t E,
+                          int32_t H, moe_math_t math, float* routed, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Accumulate flags of moe_top1_bwd: a set bit adds the result to the output
+ * buffer instead of overwriting it ([P1] kernel list calls d_fused_ctx an
+ * accumulator; [P5] zeroes the gradients at step start). */
+#define MOE_ACC_DX 0x1u
+#define MOE_ACC_DW 0x2u
+#define MOE_ACC_DB 0x4u
+
+/*
+ * Backward (straight-through). [P1] kernel list ("chain-rule grads through the
+ * SELECTED expert's W and bias ... Inactive experts get zero contribution") and
+ * ARCHITECTURE ("gate logit grad is zero from the expert path"):
+ *   d_x[t, i]   = sum_o W[e*, o, i] * d_out[t, o]
+ *   dW[e, o, i] = sum_{t : e*(t) = e} d_out[t, o] * x[t, i]
+ *   db[e, o]    = sum_{t : e*(t) = e} d_out[t, o]
+ * An expert with no tokens gets exactly 0 in dW and db. No gradient is written
+ * for the gate logits (only the aux loss below produces one). Any of d_x, dW,
+ * db may be NULL to skip it. Outputs are overwritten unless the matching
+ * MOE_ACC_* bit is set. The sums over tokens are per-expert contractions
+ * reduced in a fixed-order tree (replacing [P3]'s per-token scratch and
+ * reduce_axis0). Outputs must not overlap each other or any input ([P5]).
+ */
+moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out,
+                          const moe_routing_t* routing, int64_t B, int64_t N_H, int32_t E,
+                          int32_t H, moe_math_t math, float* d_x, float* dW, float* db,
+                          uint32_t accumulate_flags, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * Load-balance auxiliary loss and its logit gradient. [P1] kernel list
+ * ("softmax of gate_logits + load-balancing auxiliary loss (frac . prob_mean x
+ * N_EXPERTS)"), ARCHITECTURE (frac comes from the non-differentiable top-1
+ * choice, so only prob_mean carries gradient) and [P2] Wiring (the loss kernel
+ * reads lambda from device memory):
+ *   p[t, e]   = softmax_e(gate_logits[t, :])  (shifted by the row max)
+ *   frac[e]   = counts[e] / T,   mean_p[e] = (1/T) sum_t p[t, e]
+ *   aux_raw   = E * (sum_e counts[e] * mean_p[e]) / T
+ *   d_logits[t, j] = lambda * (E / T) * p[t, j] * (frac[j] - sum_e frac[e] p[t, e])
+ * with lambda = *lambda_eff (device scalar). Writes loss_out[0] = aux_raw,
+ * loss_out[1] = lambda * aux_raw, mean_p [E], d_logits [T, E] (overwritten;
+ * may be NULL) and, if stats is not NULL, stats [3E + 4] = frac[E], mean_p[E],
+ * counts[E] (as float), aux_raw, lambda, H(frac), H(mean_p) where
+ * H(q) = -sum q ln q (0 ln 0 = 0). T = 0 gives zeros everywhere. counts must be
+ * the routing of the same tokens. Needs the workspace.
+ */
+moe_status_t moe_aux_loss_fwd_bwd(const float* gate_logits, const int32_t* counts, int64_t B,
+                                  int64_t N_H, int32_t E, const float* lambda_eff,
+                                  float* d_logits, float* loss_out, float* mean_p, float* stats,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Adaptive load-balance weight. [P2] opening paragraph:
+ *   lambda_eff = lambda_floor + lambda_max_extra * max(0, ent_target - ent_ema) / ent_target
+ * ent_ema and lambda_eff are device scalars (lambda_eff may equal ent_ema's
+ * buffer only if the caller no longer needs ent_ema); a NaN ent_ema gives the
+ * floor. ent_target must be finite and > 0 ([P2] uses 0.7 * ln E); the
+ * floor and the extra must be finite and >= 0.
+ */
+moe_status_t moe_lambda_eff_update(const float* ent_ema, float lambda_floor,
+                                   float lambda_max_extra, float ent_target, float* lambda_eff,
+                                   void* stream);
+
+/* Synchronises `stream`, returns the workspace flag word in *flags_out and
+ * clears it. MOE_ERR_DEVICE_CHECK if any bit was set. (Debug / tests.) */
+moe_status_t moe_top1_device_flags(void* workspace, size_t workspace_bytes, void* stream,
+                                   uint32_t* flags_out);
+
+/* Human-readable name of a status. Never NULL. */
+const char* moe_status_string(moe_status_t status);
+
+/* MOE_TOP1_ABI_VERSION of the built library. */
+int32_t moe_top1_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_TOP1_H */

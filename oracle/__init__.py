@@ -47,6 +47,7 @@ def _load():
         lib.oracle_fwd.argtypes = [P, P, P, P, i64, i32, i32, i32, P]
         lib.oracle_bwd_dx.argtypes = [P, P, P, i64, i32, i32, i32, P]
         lib.oracle_bwd_dw.argtypes = [P, P, P, i64, i32, i32, i32, P, P, P, P]
+        lib.oracle_bwd_db.argtypes = [P, P, i64, i32, i32, P, P]
         lib.oracle_bwd_dw_entries.argtypes = [P, P, P, i64, i32, i32, i64, P, P, P, P, P]
         lib.oracle_aux.argtypes = [P, P, i64, i32, ctypes.c_float, P, P, P, P, P]
         lib.oracle_lambda_eff.restype = ctypes.c_double
@@ -112,6 +113,16 @@ def bwd_dw(x, d_out, expert_idx, E: int, tf32_mode: int = TF32_NONE):
     _load().oracle_bwd_dw(_p(x), _p(d_out), _p(idx), T, E, H, tf32_mode,
                           _p(dW), _p(db), _p(sW), _p(sb))
     return dW, db, sW, sb
+
+
+def bwd_db(d_out, expert_idx, E: int):
+    """-> (db [E,H], db_scale [E,H]) float64."""
+    d_out, idx = _f32(d_out), _i32(expert_idx)
+    T, H = d_out.shape
+    db = np.empty((E, H), np.float64)
+    sb = np.empty((E, H), np.float64)
+    _load().oracle_bwd_db(_p(d_out), _p(idx), T, E, H, _p(db), _p(sb))
+    return db, sb
 
 
 def bwd_dw_entries(x, d_out, expert_idx, e_list, o_list, i_list, tf32_mode: int = TF32_NONE):

@@ -174,6 +174,23 @@ void oracle_bwd_dw(const float* x, const float* d_out, const int32_t* expert_idx
         for (int64_t k = 0; k < (int64_t)E * H; ++k) db_scale[k] = sqrt(db_scale[k]);
 }
 
+/* db alone (the second sum above), for full-size workloads.                  */
+void oracle_bwd_db(const float* d_out, const int32_t* expert_idx, int64_t T, int32_t E, int32_t H,
+                   double* db, double* db_scale)
+{
+    memset(db, 0, sizeof(double) * (size_t)(E * H));
+    memset(db_scale, 0, sizeof(double) * (size_t)(E * H));
+    for (int64_t t = 0; t < T; ++t) {
+        const int32_t e = expert_idx[t];
+        for (int32_t o = 0; o < H; ++o) {
+            const double g = (double)d_out[t * H + o];
+            db[(int64_t)e * H + o] += g;
+            db_scale[(int64_t)e * H + o] += g * g;
+        }
+    }
+    for (int64_t k = 0; k < (int64_t)E * H; ++k) db_scale[k] = sqrt(db_scale[k]);
+}
+
 /* The same sums for a list of n single entries (e, o, i) -- for full-size     */
 /* workloads, where the whole dW is too slow on one core.                      */
 void oracle_bwd_dw_entries(const float* x, const float* d_out, const int32_t* expert_idx,

@@ -1,0 +1,276 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Integers (routing) must match bit for bit; floating point within the
+tolerances of gpu_harness.TOL, element by element. Every output buffer is
+surrounded by guard bands that must come back untouched, and the device flag
+word must stay clear.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bwd_route_b200 import ops
+from bwd_route_b200 import workloads as wl
+from gpu_harness import TOL, assert_close, run_gpu, tf32_mode
+
+pytestmark = pytest.mark.gpu
+
+MATHS = [ops.MOE_MATH_FFMA, ops.MOE_MATH_TF32]
+MATH_ID = {ops.MOE_MATH_FFMA: "ffma", ops.MOE_MATH_TF32: "tf32"}
+
+# Workloads the oracle finishes in seconds (full comparison).
+SMALL = ["tiny_b8_e4_h128", "tiny_uniform_b8_e4_h128", "tiny_identity_b8_e4_h128", "small_b1024_e4_h128",
+         "skewed_b4096_e8_h128", "ties_b16384_e4_h128", "collapsed_b16384_e4_h128"]
+
+# Ragged and degenerate shapes: token counts that are not tile multiples, one
+# token, one expert, odd expert counts, the maximum expert count, H = 256.
+EDGE = [
+    wl.make_spec("one_token_e4_h128", 1, 1, 4, 128, 11),
+    wl.make_spec("ragged_b1025_e4_h128", 1025, 5, 4, 128, 12),
+    wl.make_spec("single_expert_b300_e1_h128", 300, 1, 1, 128, 13),
+    wl.make_spec("odd_experts_b999_e5_h128", 999, 3, 5, 128, 14),
+    wl.make_spec("max_experts_b2000_e32_h128", 2000, 3, 32, 128, 15),
+    wl.make_spec("h256_b1500_e8_h256", 1500, 3, 8, 256, 16),
+    wl.make_spec("h256_skewed_b777_e3_h256", 777, 1, 3, 256, 17, skew_expert=1, skew_value=3.0),
+]
+
+
+def lam_of(inp):
+    return float(np.float32(oracle.lambda_eff(inp.ent_ema, inp.lambda_floor, inp.lambda_max_extra,
+                                              inp.ent_target)))
+
+
+def check_all(inp, math, full=True):
+    lam = lam_of(inp)
+    g = run_gpu(inp, math, lam)
+    assert g["flags"] == 0
+    assert g["guards_ok"], "a kernel wrote outside its output"
+    idx, counts, offsets, perm = oracle.route(inp.gate_logits)
+    np.testing.assert_array_equal(g["expert_idx"], idx)
+    np.testing.assert_array_equal(g["counts"], counts)
+    np.testing.assert_array_equal(g["offsets"], offsets)
+    np.testing.assert_array_equal(g["perm"], perm)
+    atol, rtol = TOL[math]
+    mode = tf32_mode(math)
+    assert_close("routed", g["routed"], oracle.fwd(inp.x, inp.W, inp.bias, idx, mode), atol, rtol)
+    assert_close("d_x", g["d_x"], oracle.bwd_dx(inp.W, inp.d_out, idx, mode), atol, rtol)
+    dW, db, sW, sb = oracle.bwd_dw(inp.x, inp.d_out, idx, inp.spec.E, mode)
+    assert_close("dW", g["dW"], dW, atol, rtol, scale=sW)
+    assert_close("db", g["db"], db, atol, rtol, scale=sb)
+    for e in range(inp.spec.E):
+        if counts[e] == 0:  # inactive experts: exactly zero
+            assert np.all(g["dW"][e] == 0.0) and np.all(g["db"][e] == 0.0)
+    check_aux(inp, g, counts, lam)
+    return g
+
+
+def check_aux(inp, g, counts, lam):
+    T, E = inp.spec.T, inp.spec.E
+    o = oracle.aux(inp.gate_logits, counts, lam)
+    assert abs(g["loss"][0] - o["aux_raw"]) <= 1e-5 * abs(o["aux_raw"]) + 1e-7
+    assert abs(g["loss"][1] - o["loss"]) <= 1e-5 * abs(o["loss"]) + 1e-9
+    assert_close("mean_p", g["mean_p"], o["mean_p"], 1e-7, 1e-5)
+    # d_logits is O(lambda E / T): compare it in units of lambda E / T
+    unit = lam * E / T
+    assert_close("d_logits/(lambda E/T)", g["d_logits"].astype(np.float64) / unit, o["d_logits_unscaled"],
+                 1e-5, 1e-5)
+    st = g["stats"]
+    np.testing.assert_allclose(st[:E], counts / T, rtol=1e-6)
+    np.testing.assert_array_equal(st[E:2 * E], g["mean_p"])
+    np.testing.assert_array_equal(st[2 * E:3 * E], counts.astype(np.float32))
+    assert st[3 * E] == g["loss"][0] and st[3 * E + 1] == np.float32(lam)
+    f = counts / T
+    hf = -sum(v * math.log(v) for v in f if v > 0)
+    hm = -sum(v * math.log(v) for v in o["mean_p"] if v > 0)
+    assert abs(st[3 * E + 2] - hf) <= 1e-5 * max(1.0, hf) and abs(st[3 * E + 3] - hm) <= 1e-5 * max(1.0, hm)
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+@pytest.mark.parametrize("name", SMALL)
+def test_full_parity(name, math_mode):
+    check_all(wl.generate(wl.WORKLOADS[name]), math_mode)
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+@pytest.mark.parametrize("spec", EDGE, ids=lambda s: s.name)
+def test_edge_parity(spec, math_mode):
+    check_all(wl.generate(spec), math_mode)
+
+
+def test_identity_experts_bit_exact():
+    inp = wl.generate(wl.WORKLOADS["tiny_identity_b8_e4_h128"])
+    g = run_gpu(inp, ops.MOE_MATH_FFMA, 0.01, parts=("route", "fwd"))
+    np.testing.assert_array_equal(g["routed"], inp.x)
+    g = run_gpu(inp, ops.MOE_MATH_TF32, 0.01, parts=("route", "fwd"))
+    rnd = np.vectorize(lambda v: oracle.tf32_round(v, tf32_mode(ops.MOE_MATH_TF32)), otypes=[np.float32])
+    np.testing.assert_array_equal(g["routed"], rnd(inp.x))
+
+
+def test_tf32_operand_rounding_rule():
+    """Black-box probe of how tcgen05 kind::tf32 reads an fp32 operand: with an
+    identity expert the output is the rounded input itself, so inputs whose low
+    13 mantissa bits sit just below, at and above half a TF32 ulp tell the rules
+    apart. The parity tests use the rule that matches (gpu_harness.TF32_RULE)."""
+    base = np.float32(1.0) + np.float32(2.0 ** -10) * np.arange(8, dtype=np.float32)
+    low = np.array([0x0FFF, 0x1000, 0x1001, 0x1FFF, 0x0001, 0x0800], dtype=np.uint32)
+    vals = []
+    for b in base:
+        for sgn in (1, -1):
+            for lb in low:
+                u = np.array([b * sgn], np.float32).view(np.uint32)[0] | lb
+                vals.append(np.array([u], np.uint32).view(np.float32)[0])
+    H, E = 128, 1
+    T = (len(vals) + H - 1) // H
+    x = np.zeros((T, H), np.float32)
+    x.flat[:len(vals)] = vals
+    spec = wl.make_spec("tf32_probe", T, 1, E, H, 1)
+    inp = wl.Inputs(spec, np.zeros((T, E), np.float32), x, np.zeros((T, H), np.float32),
+                    np.eye(H, dtype=np.float32)[None].copy(), np.zeros((E, H), np.float32))
+    g = run_gpu(inp, ops.MOE_MATH_TF32, 0.01, parts=("route", "fwd"))
+    got = g["routed"]
+    matches = {}
+    for mode in (oracle.TF32_RZ, oracle.TF32_RNA, oracle.TF32_RNE):
+        want = np.vectorize(lambda v: oracle.tf32_round(v, mode), otypes=[np.float32])(x)
+        matches[mode] = bool(np.array_equal(got, want))
+    print("tf32 rounding rule matches (RZ, RNA, RNE):", matches)
+    assert sum(matches.values()) == 1, matches
+    assert matches[tf32_mode(ops.MOE_MATH_TF32)], matches
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_deterministic_bitwise(math_mode):
+    inp = wl.generate(wl.WORKLOADS["skewed_b4096_e8_h128"])
+    a = run_gpu(inp, math_mode, 0.02)
+    b = run_gpu(inp, math_mode, 0.02)
+    for k in ["expert_idx", "perm", "routed", "d_x", "dW", "db", "d_logits", "loss", "mean_p", "stats"]:
+        assert a[k].tobytes() == b[k].tobytes(), k
+
+
+def test_uniform_logits_aux_is_exactly_one():
+    inp = wl.generate(wl.WORKLOADS["tiny_uniform_b8_e4_h128"])
+    g = run_gpu(inp, ops.MOE_MATH_FFMA, 0.03, parts=("route", "aux"))
+    assert g["loss"][0] == 1.0
+    assert np.all(g["mean_p"] == 0.25)
+    T = inp.spec.T
+    frac = g["counts"] / T
+    expect = np.float32(0.03) * (frac[None, :] - 0.25) / T * np.ones((T, 1))
+    np.testing.assert_allclose(g["d_logits"], expect, rtol=1e-6, atol=1e-12)
+    # rows of the softmax gradient sum to zero
+    assert np.all(np.abs(g["d_logits"].sum(axis=1)) <= 1e-6 * np.abs(g["d_logits"]).sum(axis=1) + 1e-12)
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_accumulate_flags(math_mode):
+    inp = wl.generate(wl.make_spec("acc_b600_e4_h128", 600, 2, 4, 128, 21))
+    rng = np.random.default_rng(0)
+    T, E, H = inp.spec.T, inp.spec.E, inp.spec.H
+    pre = {"d_x": rng.standard_normal((T, H)).astype(np.float32),
+           "dW": rng.standard_normal((E, H, H)).astype(np.float32),
+           "db": rng.standard_normal((E, H)).astype(np.float32)}
+    plain = run_gpu(inp, math_mode, 0.01, parts=("route", "bwd"))
+    acc = run_gpu(inp, math_mode, 0.01, parts=("route", "bwd"), preset=pre,
+                  acc_flags=ops.MOE_ACC_DX | ops.MOE_ACC_DW | ops.MOE_ACC_DB)
+    for k in ("d_x", "dW", "db"):
+        np.testing.assert_array_equal(acc[k], (pre[k] + plain[k]).astype(np.float32), err_msg=k)
+
+
+def test_empty_batch():
+    spec = wl.make_spec("empty", 0, 5, 4, 128, 1)
+    inp = wl.generate(spec)
+    pre = {"dW": np.ones((4, 128, 128), np.float32), "db": np.ones((4, 128), np.float32),
+           "counts": np.full(4, 7, np.int32), "offsets": np.full(5, 7, np.int32)}
+    for m in MATHS:
+        g = run_gpu(inp, m, 0.01, preset=pre)
+        assert g["flags"] == 0 and g["guards_ok"]
+        assert np.all(g["counts"] == 0) and np.all(g["offsets"] == 0)
+        assert np.all(g["dW"] == 0) and np.all(g["db"] == 0)
+        assert np.all(g["loss"] == 0) and np.all(g["mean_p"] == 0)
+
+
+def test_route_special_values():
+    nan, inf = np.nan, np.inf
+    rows = [[nan, 1, 2, 0], [1, nan, 2, 0], [3, nan, 2, 0], [-0.0, 0.0, -1, 0], [-inf, -inf, -inf, -inf],
+            [-inf, -5, -inf, -6], [inf, inf, 1, 0], [1, 1, 1, 1], [0, 0, 0, nan], [nan, nan, nan, nan]]
+    lg = np.array(rows * 7, np.float32)
+    T = lg.shape[0]
+    spec = wl.make_spec("special", T, 1, 4, 128, 1)
+    inp = wl.Inputs(spec, lg, np.zeros((T, 128), np.float32), np.zeros((T, 128), np.float32),
+                    np.zeros((4, 128, 128), np.float32), np.zeros((4, 128), np.float32))
+    g = run_gpu(inp, ops.MOE_MATH_FFMA, 0.01, parts=("route",))
+    idx, counts, offsets, perm = oracle.route(lg)
+    np.testing.assert_array_equal(g["expert_idx"], idx)
+    np.testing.assert_array_equal(g["perm"], perm)
+    np.testing.assert_array_equal(g["counts"], counts)
+
+
+@pytest.mark.parametrize("E", [1, 2, 3, 7, 8, 9, 16, 17, 31, 32])
+def test_route_expert_counts(E):
+    T = 4099
+    rng = np.random.default_rng(E)
+    lg = rng.integers(0, 3, size=(T, E)).astype(np.float32)  # many ties
+    spec = wl.make_spec(f"route_e{E}", T, 1, E, 128, 1)
+    inp = wl.Inputs(spec, lg, np.zeros((0, 128), np.float32), np.zeros((0, 128), np.float32),
+                    np.zeros((E, 128, 128), np.float32), np.zeros((E, 128), np.float32))
+    g = run_gpu(inp, ops.MOE_MATH_FFMA, 0.01, parts=("route",))
+    idx, counts, offsets, perm = oracle.route(lg)
+    np.testing.assert_array_equal(g["expert_idx"], idx)
+    np.testing.assert_array_equal(g["counts"], counts)
+    np.testing.assert_array_equal(g["offsets"], offsets)
+    np.testing.assert_array_equal(g["perm"], perm)
+
+
+def test_lambda_eff_kernel():
+    K = 8
+    target = 0.7 * math.log(K)
+    cases = [1.381, 0.746, target + 0.1, target, target / 2, 0.0, math.log(K), float("nan")]
+    for ent in cases:
+        e = torch.tensor([ent], dtype=torch.float32, device="cuda")
+        lam = torch.zeros(1, dtype=torch.float32, device="cuda")
+        ops.moe_lambda_eff_update(e, 0.01, 0.09, target, lam)
+        ref = oracle.lambda_eff(float(np.float32(ent)), 0.01, 0.09, float(np.float32(target))) \
+            if not math.isnan(ent) else 0.01
+        assert abs(lam.item() - ref) <= 1e-6, (ent, lam.item(), ref)
+    e = torch.tensor([1.381], dtype=torch.float32, device="cuda")
+    lam = torch.zeros(1, dtype=torch.float32, device="cuda")
+    ops.moe_lambda_eff_update(e, 0.01, 0.09, target, lam)
+    assert abs(lam.item() - 0.0146) <= 5e-5  # the value printed on the controller page
+
+
+@pytest.fixture(scope="module")
+def large():
+    return wl.generate(wl.WORKLOADS[wl.THROUGHPUT_WORKLOAD])
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_large_workload_sampled(large, math_mode):
+    """1,048,576 tokens, H = 256, in the launch configuration the benchmark times:
+    routing and aux in full, the per-token outputs on sampled tokens, dW on
+    sampled entries and db in full."""
+    inp = large
+    lam = lam_of(inp)
+    g = run_gpu(inp, math_mode, lam)
+    assert g["flags"] == 0 and g["guards_ok"]
+    idx, counts, offsets, perm = oracle.route(inp.gate_logits)
+    np.testing.assert_array_equal(g["expert_idx"], idx)
+    np.testing.assert_array_equal(g["counts"], counts)
+    np.testing.assert_array_equal(g["offsets"], offsets)
+    np.testing.assert_array_equal(g["perm"], perm)
+    atol, rtol = TOL[math_mode]
+    mode = tf32_mode(math_mode)
+    rng = np.random.default_rng(99)
+    rows = np.sort(rng.choice(inp.spec.T, 512, replace=False))
+    rows = np.concatenate([rows, [0, inp.spec.T - 1], perm[offsets[1:-1]]])  # ends and expert boundaries
+    assert_close("routed", g["routed"][rows], oracle.fwd(inp.x[rows], inp.W, inp.bias, idx[rows], mode), atol, rtol)
+    assert_close("d_x", g["d_x"][rows], oracle.bwd_dx(inp.W, inp.d_out[rows], idx[rows], mode), atol, rtol)
+    n = 96
+    e_l = rng.integers(0, inp.spec.E, n)
+    o_l = rng.integers(0, inp.spec.H, n)
+    i_l = rng.integers(0, inp.spec.H, n)
+    vals, scales = oracle.bwd_dw_entries(inp.x, inp.d_out, idx, e_l, o_l, i_l, mode)
+    assert_close("dW", g["dW"][e_l, o_l, i_l], vals, atol, rtol, scale=scales)
+    db, sb = oracle.bwd_db(inp.d_out, idx, inp.spec.E)
+    assert_close("db", g["db"], db, atol, rtol, scale=sb)
+    check_aux(inp, g, counts, lam)

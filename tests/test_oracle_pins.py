@@ -278,6 +278,16 @@ def test_dw_entries_match_full_and_scale_is_rss():
     assert sW[e, o, ii] >= abs(dW[e, o, ii]) - 1e-12
 
 
+def test_db_alone_matches_column_sums():
+    inp = wl.generate(wl.WORKLOADS["skewed_b4096_e8_h128"])
+    idx, *_ = oracle.route(inp.gate_logits)
+    db, sb = oracle.bwd_db(inp.d_out, idx, 8)
+    for e in range(8):
+        sel = inp.d_out[idx == e].astype(np.float64)
+        np.testing.assert_allclose(db[e], sel.sum(axis=0), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(sb[e], np.sqrt((sel ** 2).sum(axis=0)), rtol=1e-12, atol=1e-12)
+
+
 def test_tf32_mode_rounds_gemm_inputs_only():
     inp = tiny()
     idx, *_ = oracle.route(inp.gate_logits)
