@@ -160,11 +160,10 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Shared-memory matrix descriptor (sm_100 "version 1"), 128-byte swizzle.
-//   K-major operand : rows of 128 B along K, 8-row groups 1024 B apart (SBO);
-//                     LBO is unused (encoded 1).
-//   MN-major operand: 128 B runs along M/N; consecutive 128-B runs along M/N
-//                     are LBO bytes apart; 8-row groups along K are SBO apart.
+// Shared-memory matrix descriptors (sm_100 "version 1").
+// K-major operand, 128-byte swizzle (16-byte granules, 8-row / 1024-byte
+// pattern): rows of 128 B along K, 8-row groups SBO bytes apart; LBO unused
+// (encoded 1).
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_bytes,
                                                uint32_t sbo_bytes) {
     uint64_t d = 0;
@@ -173,6 +172,21 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
     d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= 1ull << 46;  // descriptor version for sm_100
     d |= 2ull << 61;  // SWIZZLE_128B
+    return d;
+}
+
+// MN-major 32-bit (TF32) operand: the tensor core accepts only the 128-byte
+// swizzle with 32-byte granules (granule index XOR row mod 4, 512-byte
+// pattern; the TMA mode CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B writes it). 128-B
+// runs along M/N are LBO bytes apart; 4-row groups along K are SBO bytes apart.
+__device__ __forceinline__ uint64_t sw128_32b_mn_desc(uint32_t smem_addr, uint32_t lbo_bytes,
+                                                      uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;  // descriptor version for sm_100
+    d |= 1ull << 61;  // SWIZZLE_128B_BASE32B
     return d;
 }
 

@@ -20,7 +20,8 @@
 //
 //   wgrad_tf32_kernel : one CTA per range of the sorted token list (range c of
 //     expert e -> partial-sum slot c + e). Both operands are MN-major (tokens
-//     are the contraction index): the CTA gathers 32 tokens of d_out and x per
+//     are the contraction index; for TF32 the tensor core then needs the
+//     128-byte swizzle with 32-byte granules): the CTA gathers 32 tokens of d_out and x per
 //     stage and issues M=128 x N=H MMAs with the whole dW[e] (H x H fp32) held
 //     in TMEM. Warps 2-5 sum d_out over the same staged tokens for db, then
 //     drain the accumulator into the slot. A separate kernel adds the slots in
@@ -372,8 +373,9 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
                     for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
                         for (int mh = 0; mh < C::MH; ++mh) {
-                            const uint64_t adesc = sw128_desc(g_addr + mh * 4 * C::GROUP_BYTES + ks * 1024, C::GROUP_BYTES, 1024);
-                            const uint64_t bdesc = sw128_desc(x_addr + ks * 1024, C::GROUP_BYTES, 1024);
+                            const uint64_t adesc =
+                                sw128_32b_mn_desc(g_addr + mh * 4 * C::GROUP_BYTES + ks * 1024, C::GROUP_BYTES, 512);
+                            const uint64_t bdesc = sw128_32b_mn_desc(x_addr + ks * 1024, C::GROUP_BYTES, 512);
                             mma_tf32(tmem + static_cast<uint32_t>(mh * H), adesc, bdesc, idesc,
                                      (first && ks == 0) ? 0u : 1u);
                         }
@@ -411,11 +413,12 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
                 for (int h = 0; h < C::MH; ++h) {
                     const int o = tid + 128 * h;
                     const int g = o >> 5, jo = o & 31;
-                    const uint8_t* colbase = gt + g * C::GROUP_BYTES + (jo & 3) * 4;
+                    // 32-byte granule (jo / 8) of row rr sits at granule (jo / 8) ^ (rr % 4)
+                    const uint8_t* colbase = gt + g * C::GROUP_BYTES + (jo & 7) * 4;
                     float acc = 0.0f;
 #pragma unroll 8
                     for (int rr = 0; rr < C::KT; ++rr)
-                        acc += *reinterpret_cast<const float*>(colbase + rr * 128 + (((jo >> 2) ^ (rr & 7)) << 4));
+                        acc += *reinterpret_cast<const float*>(colbase + rr * 128 + (((jo >> 3) ^ (rr & 3)) << 5));
                     if (h == 0) db0 += acc; else db1 += acc;
                 }
                 __syncwarp();
@@ -502,8 +505,8 @@ cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t*
                               int64_t T, int E, int H, float* part, float* part_db, uint32_t* dev_flags,
                               cudaStream_t s) {
     CUtensorMap tm_g, tm_x;
-    if (!make_map_2d(&tm_g, d_out, static_cast<uint64_t>(T), H, 32, 1)) return cudaErrorInvalidValue;
-    if (!make_map_2d(&tm_x, x, static_cast<uint64_t>(T), H, 32, 1)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&tm_g, d_out, static_cast<uint64_t>(T), H, 32, 1, true)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&tm_x, x, static_cast<uint64_t>(T), H, 32, 1, true)) return cudaErrorInvalidValue;
     const int P = wgrad_splits(T);
     cudaError_t err;
     if (H == 256) {

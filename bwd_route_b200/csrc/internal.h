@@ -114,8 +114,9 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn get_encode_tiled();
 
-// 2D fp32 tensor [rows][cols] with a 128-byte-swizzled box of box_cols x box_rows.
+// 2D fp32 tensor [rows][cols] with a 128-byte-swizzled box of box_cols x box_rows
+// (16-byte granules, or 32-byte granules when atom32 is set).
 bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                 uint32_t box_rows);
+                 uint32_t box_rows, bool atom32 = false);
 
 }  // namespace moe

@@ -64,6 +64,9 @@ WORKLOADS = {
                                  skew_expert=4, skew_value=2.0),
     # 1,048,576 tokens, H = 256: the throughput workload.
     "large_b65536_e8_h256": Spec("large_b65536_e8_h256", 65536, 16, 8, 256, 1004),
+    # 262,144 tokens, H = 256: the throughput workload's shape at a quarter of the
+    # tokens (activations still larger than L2), for profiler captures.
+    "mid_b16384_e8_h256": Spec("mid_b16384_e8_h256", 16384, 16, 8, 256, 1006),
     # 81,920 tokens with logits in {0, 1}: frequent argmax ties.
     "ties_b16384_e4_h128": Spec("ties_b16384_e4_h128", 16384, 5, 4, 128, 1005, logits="binary"),
     # the same with +10 on expert 0: every token collapses onto expert 0.
