@@ -12,6 +12,7 @@
 namespace moe {
 
 cudaError_t aux_set_smem_limits();
+cudaError_t route_set_smem_limits();
 
 namespace {
 
@@ -38,6 +39,7 @@ cudaError_t device_info(DeviceInfo** out) {
     }
     if (!d.aux_ready) {
         e = aux_set_smem_limits();
+        if (e == cudaSuccess) e = route_set_smem_limits();
         if (e != cudaSuccess) return e;
         d.aux_ready = true;
     }
@@ -194,6 +196,8 @@ moe_status_t moe_top1_route(const float* gate_logits, int64_t B, int64_t N_H, in
     if (!workspace) return MOE_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
     if (workspace_bytes < L.route_end) return MOE_ERR_WORKSPACE;
+    DeviceInfo* dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     return cuda_status(launch_route(gate_logits, T, E, out->expert_idx, out->counts, out->offsets, out->perm,
                                     reinterpret_cast<int32_t*>(ws + L.route_counts),

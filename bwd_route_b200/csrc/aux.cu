@@ -105,29 +105,24 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
     }
 }
 
-// One block: mean_p from the per-block sums (double, fixed order), aux, loss, stats.
-__global__ void __launch_bounds__(256) aux_finalize_kernel(const float* __restrict__ blk_psum, int64_t nblk,
-                                                          const int32_t* __restrict__ counts, int64_t T, int E,
-                                                          const float* __restrict__ lambda_eff,
-                                                          float* __restrict__ loss_out, float* __restrict__ mean_p,
-                                                          float* __restrict__ stats) {
-    __shared__ double s_w[8];
+// One block: mean_p from the per-block sums (double, fixed order: warp e sums
+// expert e with lane-strided partials and an xor butterfly), then aux, loss and
+// stats.
+__global__ void __launch_bounds__(1024) aux_finalize_kernel(const float* __restrict__ blk_psum, int64_t nblk,
+                                                           const int32_t* __restrict__ counts, int64_t T, int E,
+                                                           const float* __restrict__ lambda_eff,
+                                                           float* __restrict__ loss_out, float* __restrict__ mean_p,
+                                                           float* __restrict__ stats) {
     __shared__ float s_mean[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int e = 0; e < E; ++e) {
+    if (warp < E) {
         double acc = 0.0;
-        for (int64_t b = threadIdx.x; b < nblk; b += blockDim.x) acc += static_cast<double>(blk_psum[b * E + e]);
+        for (int64_t b = lane; b < nblk; b += 32) acc += static_cast<double>(blk_psum[b * E + warp]);
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) s_w[warp] = acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double tot = 0.0;
-            for (int w = 0; w < 8; ++w) tot += s_w[w];
-            s_mean[e] = T > 0 ? static_cast<float>(tot / static_cast<double>(T)) : 0.0f;
-        }
-        __syncthreads();
+        if (lane == 0) s_mean[warp] = T > 0 ? static_cast<float>(acc / static_cast<double>(T)) : 0.0f;
     }
+    __syncthreads();
     if (threadIdx.x == 0) {
         const float lam = *lambda_eff;
         double acc = 0.0, hf = 0.0, hm = 0.0;
@@ -181,7 +176,7 @@ cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, in
         const cudaError_t err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
-    aux_finalize_kernel<<<1, 256, 0, s>>>(blk_psum, nblk, counts, T, E, lambda_eff, loss_out, mean_p, stats);
+    aux_finalize_kernel<<<1, 1024, 0, s>>>(blk_psum, nblk, counts, T, E, lambda_eff, loss_out, mean_p, stats);
     return cudaGetLastError();
 }
 

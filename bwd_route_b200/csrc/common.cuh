@@ -99,6 +99,23 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// ---------------------------------------------------------------- cp.async (LSU) gathers
+// 16-byte global -> shared copy through L2; src_bytes = 0 writes 16 zero bytes
+// and reads nothing.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// The mbarrier receives one arrival once every cp.async issued so far by this
+// thread has landed (the arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Orders shared-memory data observed by this thread (written through the
+// generic proxy, e.g. by cp.async) before its later tensor-core reads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 // Allocation is done by one whole warp; the TMEM address lands in *dst_smem.
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

@@ -248,6 +248,8 @@ struct PairwiseSum {
     }
 };
 
+constexpr int kBatch = 8;
+
 // grid.x: float4 groups of dW[e] (plus one trailing block for db), grid.y = E.
 __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ part,
                                                           const float* __restrict__ part_db,
@@ -280,8 +282,18 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
         const int64_t j = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;  // float4 index
         if (j >= HH / 4) return;
         PairwiseSum ps;
-        for (int c = c_lo; c <= c_hi; ++c)
-            ps.add(__ldg(reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c) + e) * HH) + j));
+        const float4* src = reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c_lo) + e) * HH) + j;
+        const int64_t stride4 = HH / 4;
+        for (int c0 = c_lo; c0 <= c_hi; c0 += kBatch) {
+            // issue a batch of independent loads, then add them in slot order
+            float4 v[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (c0 + u <= c_hi) v[u] = __ldg(src + static_cast<int64_t>(c0 - c_lo + u) * stride4);
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (c0 + u <= c_hi) ps.add(v[u]);
+        }
         float4 r = ps.result();
         float4* dst = reinterpret_cast<float4*>(dW + e * HH) + j;
         if (acc_dw) {

@@ -1,5 +1,5 @@
 // gemm_tf32.cu -- tcgen05 (5th-generation tensor core) TF32 kernels of the
-// expert contractions, fed by TMA, accumulating in tensor memory (TMEM).
+// expert contractions, accumulating in tensor memory (TMEM).
 //
 // foxhunt commit 11b96dac6a ("Top-1 Mixture-of-Experts gate per Switch
 // Transformer"), kernel list / PERFORMANCE: the forward applies the selected
@@ -8,30 +8,36 @@
 // (d_x[t,i] = sum_o W[e*,o,i] d_out[t,o]; dW[e,o,i] = sum_{t in e} d_out[t,o]
 // x[t,i]; db[e,o] = sum_{t in e} d_out[t,o]). The pages give one block per
 // token and one thread per output channel; here the tokens of an expert are
-// contiguous in the routing permutation, so each expert is a dense GEMM:
+// contiguous in the routing permutation, so each expert is a dense GEMM whose
+// token rows are gathered on the fly.
 //
-//   grouped_tf32_kernel : persistent, one CTA per SM. A tile is 128 sorted
-//     tokens x all H outputs. Warp 0 gathers the tile's token rows with TMA
-//     tile::gather4 (128-byte swizzle) and loads the expert's weight slab with a
-//     2D TMA box; warp 1 issues tcgen05.mma kind::tf32 (M=128, N=H, K=8) into
-//     one of two TMEM accumulators; warps 2-5 drain the other accumulator
-//     (tcgen05.ld), add the bias, and store the rows back to their original
-//     token positions with coalesced 128-byte stores.
+// Row gathers use cp.async (16 bytes per lane, eight lanes per 128-byte row
+// segment) into the swizzled shared-memory layout the MMA reads: measured on
+// the B200 with one CTA per SM and 96 KiB in flight, this path streams rows at
+// ~6.1 TB/s, where TMA tile::gather4 (512 bytes per operation) reaches
+// ~2.0 TB/s. The dense expert-weight operand is loaded by TMA.
+//
+//   grouped_tf32_kernel : persistent, one CTA per SM; a tile is 128 sorted
+//     tokens x all H outputs. Warps 4-7 gather the tile's rows (K-major,
+//     128-byte swizzle), one thread also loads the expert's weight slab by TMA;
+//     warp 8 issues tcgen05.mma kind::tf32 (M=128, N=H, K=8) into one of two
+//     TMEM accumulators; warps 0-3 drain the other accumulator (tcgen05.ld),
+//     add the bias and store the rows to their original token positions with
+//     coalesced 128-byte stores.
 //
 //   wgrad_tf32_kernel : one CTA per range of the sorted token list (range c of
-//     expert e -> partial-sum slot c + e). Both operands are MN-major (tokens
-//     are the contraction index; for TF32 the tensor core then needs the
-//     128-byte swizzle with 32-byte granules): the CTA gathers 32 tokens of d_out and x per
-//     stage and issues M=128 x N=H MMAs with the whole dW[e] (H x H fp32) held
-//     in TMEM. Warps 2-5 sum d_out over the same staged tokens for db, then
-//     drain the accumulator into the slot. A separate kernel adds the slots in
-//     a fixed pairwise order (no atomics: foxhunt commit b23f8f2efa,
-//     Discipline).
+//     expert e -> partial-sum slot c + e). Tokens are the contraction index, so
+//     both operands are MN-major, which for TF32 needs the 128-byte swizzle with
+//     32-byte granules. Warps 4-7 gather 32 tokens of d_out and x per stage;
+//     warp 8 issues M=128 x N=H MMAs with the whole dW[e] (H x H fp32) in TMEM;
+//     warps 0-3 sum d_out over the staged tokens for db, then drain dW into the
+//     slot. A separate kernel adds the slots in a fixed pairwise order (no
+//     atomics: foxhunt commit b23f8f2efa, Discipline).
 //
 // The tensor core reads each fp32 operand as TF32 (its 10 leading mantissa
-// bits) and accumulates in fp32. Every pipeline wait is bounded (common.cuh).
+// bits, the low 13 bits dropped) and accumulates in fp32. Every pipeline wait
+// is bounded (common.cuh).
 #include <cstdint>
-#include <cstdio>
 
 #include "common.cuh"
 #include "internal.h"
@@ -39,7 +45,10 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-5: epilogue
+// warps 0-3: epilogue (TMEM lane quadrant = warp), 4-7: producers, 8: MMA + TMEM owner
+constexpr int kThreads = 288;
+constexpr int kProducer0 = 128;
+constexpr int kMmaWarp = 8;
 constexpr int kMaxStages = 8;
 
 struct __align__(8) Ctl {
@@ -77,9 +86,9 @@ __device__ __forceinline__ int find_expert(const int* tstart, int E, int tile) {
 
 template <int H>
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_constant__ CUtensorMap tm_b,
+grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUtensorMap tm_b,
                     const float* __restrict__ bias, const int32_t* __restrict__ offsets,
-                    const int32_t* __restrict__ perm, int T, int E, int accumulate, float* __restrict__ out,
+                    const int32_t* __restrict__ perm, int E, int accumulate, float* __restrict__ out,
                     uint32_t* __restrict__ dev_flags) {
     using C = GCfg<H>;
     extern __shared__ uint8_t smem_raw[];
@@ -91,8 +100,8 @@ grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_con
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&ctl->full[s], 1);
-            mbar_init(&ctl->empty[s], 1);
+            mbar_init(&ctl->full[s], 128 + 1);  // 128 gather threads + the weight-slab thread
+            mbar_init(&ctl->empty[s], 1);       // tcgen05.commit
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
@@ -102,11 +111,8 @@ grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_con
         fence_mbar_init();
     }
     if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_src);
-        tma_prefetch_desc(&tm_b);
-    }
-    if (warp == 1) {
+    if (threadIdx.x == kProducer0) tma_prefetch_desc(&tm_b);
+    if (warp == kMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -126,38 +132,53 @@ grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_con
     const int ntiles = ctl->tstart[E];
     volatile int* abort = &ctl->abort;
 
-    if (warp == 0) {
-        // ---------------- TMA producer
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    if (warp >= 4 && warp < 8) {
+        // ---------------- producers: cp.async row gather (+ TMA weight slab)
+        const int ptid = threadIdx.x - kProducer0;  // 0..127
+        const int prow = ptid >> 3, pg = ptid & 7;  // row within a 16-row block, 16-byte granule
+        int tok[8], nxt[8];
+        auto load_tokens = [&](int tile, int (&t)[8]) {
             const int e = find_expert(ctl->tstart, E, tile);
             const int row0 = ctl->off[e] + (tile - ctl->tstart[e]) * C::BM;
             const int nrows = min(C::BM, ctl->off[e + 1] - row0);
-            int tok[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = 4 * lane + j;
-                tok[j] = (r < nrows) ? perm[row0 + r] : T;  // row T is outside the tensor: zeros
+            for (int it = 0; it < 8; ++it) {
+                const int r = it * 16 + prow;
+                t[it] = (r < nrows) ? perm[row0 + r] : -1;
             }
-            bool ok = true;
-            for (int kc = 0; kc < C::KCH && ok; ++kc) {
-                if (lane == 0) ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
+        };
+        if (static_cast<int>(blockIdx.x) < ntiles) load_tokens(blockIdx.x, tok);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            const int e = find_expert(ctl->tstart, E, tile);
+            if (tile + static_cast<int>(gridDim.x) < ntiles) load_tokens(tile + gridDim.x, nxt);
+            for (int kc = 0; kc < C::KCH; ++kc) {
+                if (!(ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags))) break;
                 uint8_t* a = stages + stage * C::STAGE_BYTES;
-                if (lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
-                __syncwarp();
-                tma_gather4(a + lane * 512, &tm_src, kc * 32, tok[0], tok[1], tok[2], tok[3], &ctl->full[stage]);
-                if (lane == 0) tma_load_2d(a + C::A_BYTES, &tm_b, kc * 32, e * H, &ctl->full[stage]);
+                if (ptid == 0) {
+                    mbar_arrive_expect_tx(&ctl->full[stage], C::B_BYTES);
+                    tma_load_2d(a + C::A_BYTES, &tm_b, kc * 32, e * H, &ctl->full[stage]);
+                }
+                const uint32_t a_u32 = smem_u32(a);
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int r = it * 16 + prow;
+                    const int t = tok[it];
+                    const float* gsrc = src + static_cast<int64_t>(t < 0 ? 0 : t) * H + kc * 32 + pg * 4;
+                    cp_async_16(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), gsrc, t < 0 ? 0u : 16u);
+                }
+                cp_async_arrive_noinc(&ctl->full[stage]);
                 if (++stage == C::STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
-            if (!ok) break;
+#pragma unroll
+            for (int it = 0; it < 8; ++it) tok[it] = nxt[it];
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_tf32(128, H, 0, 0);
@@ -172,6 +193,7 @@ grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_con
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * H);
                 for (int kc = 0; kc < C::KCH; ++kc) {
                     if (!(ok = mbar_wait(&ctl->full[stage], phase, abort, dev_flags))) break;
+                    fence_proxy_async_smem();
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(stages + stage * C::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + C::A_BYTES;
@@ -192,10 +214,10 @@ grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_con
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp < 4) {
         // ---------------- epilogue: TMEM -> registers -> smem transpose -> rows
-        const int q = warp & 3;  // TMEM lane quadrant this warp may access
-        float* my = stg + (warp - 2) * 32 * 32;
+        const int q = warp;  // TMEM lane quadrant
+        float* my = stg + warp * 32 * 32;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -253,7 +275,7 @@ grouped_tf32_kernel(const __grid_constant__ CUtensorMap tm_src, const __grid_con
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -264,6 +286,7 @@ template <int H>
 struct WCfg {
     static constexpr int KT = 32;                    // tokens per stage (4 MMAs of K = 8)
     static constexpr int G = H / 32;                 // 128-byte column groups
+    static constexpr int LOG_G = (G == 8) ? 3 : 2;
     static constexpr int GROUP_BYTES = KT * 128;     // one group: KT rows x 128 B (4 KiB)
     static constexpr int OP_BYTES = G * GROUP_BYTES; // one operand per stage
     static constexpr int STAGE_BYTES = 2 * OP_BYTES; // d_out then x
@@ -271,15 +294,16 @@ struct WCfg {
     static constexpr int MH = H / 128;               // 128-row halves of dW
     static constexpr int TMEM_COLS = MH * H;
     static constexpr int STG_BYTES = 4 * 32 * 128;
+    static constexpr int PER_THREAD = KT * G * 8 / 128;  // 16-byte granules per operand per producer thread
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + static_cast<int>(sizeof(Ctl));
+    static_assert(G == 4 || G == 8, "H");
     static_assert(STAGES <= kMaxStages, "stages");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-    static_assert((2 * G) % 4 == 0, "gather split");
 };
 
 template <int H>
 __global__ void __launch_bounds__(kThreads, 1)
-wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x,
+wgrad_tf32_kernel(const float* __restrict__ g_src, const float* __restrict__ x_src,
                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int T, int E, int P,
                   float* __restrict__ part, float* __restrict__ part_db, uint32_t* __restrict__ dev_flags) {
     using C = WCfg<H>;
@@ -293,8 +317,8 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&ctl->full[s], 1);
-            mbar_init(&ctl->empty[s], 1 + 4);  // MMA commit + the four db warps
+            mbar_init(&ctl->full[s], 128);     // 128 gather threads
+            mbar_init(&ctl->empty[s], 1 + 4);  // tcgen05.commit + the four db warps
         }
         mbar_init(&ctl->tfull[0], 1);
         mbar_init(&ctl->tempty[0], 4);
@@ -302,11 +326,7 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
         fence_mbar_init();
     }
     if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_g);
-        tma_prefetch_desc(&tm_x);
-    }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -317,40 +337,41 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
     volatile int* abort = &ctl->abort;
     const int lo = static_cast<int>(split_lo(c, T, P)), hi = static_cast<int>(split_lo(c + 1, T, P));
 
-    if (warp == 0) {
-        // ---------------- TMA producer: 32 tokens of d_out and x per stage
-        const int jq = lane & 7;          // which 4-token quad this lane gathers
-        const int combo0 = lane >> 3;     // first (operand, group) combination
+    if (warp >= 4 && warp < 8) {
+        // ---------------- producers: 32 tokens of d_out and x per stage, MN-major,
+        // 128-byte swizzle with 32-byte granules (granule index ^ row % 4)
+        const int ptid = threadIdx.x - kProducer0;  // 0..127
+        const int q16 = ptid & 7;                   // 16-byte granule within a 128-byte group row
+        const int g = (ptid >> 3) & (C::G - 1);     // column group
+        const int rsub = ptid >> (3 + C::LOG_G);    // row offset inside one pass
+        constexpr int ROWS_PER_PASS = 128 / (8 * C::G);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int e = 0; e < E && ok; ++e) {
             const int s = max(lo, ctl->off[e]), t = min(hi, ctl->off[e + 1]);
             for (int p0 = s; p0 < t; p0 += C::KT) {
-                const int tok_lane = (p0 + lane < t) ? perm[p0 + lane] : T;  // row T reads zeros
-                int r[4];
+                const int tok_lane = (p0 + lane < t) ? perm[p0 + lane] : -1;
+                if (!(ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags))) break;
+                const uint32_t base = smem_u32(stages + stage * C::STAGE_BYTES);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) r[k] = __shfl_sync(0xffffffffu, tok_lane, 4 * jq + k);
-                if (lane == 0) ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                uint8_t* base = stages + stage * C::STAGE_BYTES;
-                if (lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
-                __syncwarp();
-#pragma unroll
-                for (int m = 0; m < (2 * C::G) / 4; ++m) {
-                    const int combo = combo0 + 4 * m;
-                    const int operand = combo / C::G, g = combo % C::G;
-                    tma_gather4(base + operand * C::OP_BYTES + g * C::GROUP_BYTES + jq * 512,
-                                operand == 0 ? &tm_g : &tm_x, g * 32, r[0], r[1], r[2], r[3], &ctl->full[stage]);
+                for (int it = 0; it < C::PER_THREAD; ++it) {
+                    const int r = it * ROWS_PER_PASS + rsub;
+                    const int tk = __shfl_sync(0xffffffffu, tok_lane, r);
+                    const uint32_t off = g * C::GROUP_BYTES + r * 128 + ((((q16 >> 1) ^ (r & 3)) << 5) | ((q16 & 1) << 4));
+                    const int64_t row = static_cast<int64_t>(tk < 0 ? 0 : tk) * H + g * 32 + q16 * 4;
+                    const uint32_t nb = tk < 0 ? 0u : 16u;
+                    cp_async_16(base + off, g_src + row, nb);
+                    cp_async_16(base + C::OP_BYTES + off, x_src + row, nb);
                 }
+                cp_async_arrive_noinc(&ctl->full[stage]);
                 if (++stage == C::STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_tf32(128, H, 1, 1);  // both operands MN-major
@@ -366,6 +387,7 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
                 bool first = true;
                 for (int p0 = s; p0 < t; p0 += C::KT) {
                     if (!(ok = mbar_wait(&ctl->full[stage], phase, abort, dev_flags))) break;
+                    fence_proxy_async_smem();
                     tc_fence_after();
                     const uint32_t g_addr = smem_u32(stages + stage * C::STAGE_BYTES);
                     const uint32_t x_addr = g_addr + C::OP_BYTES;
@@ -393,11 +415,11 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp < 4) {
         // ---------------- db over the staged d_out rows, then drain dW to the slot
-        const int tid = threadIdx.x - 64;  // 0..127: owns d_out column o = tid (and tid + 128)
-        const int q = warp & 3;
-        float* my = stg + (warp - 2) * 32 * 32;
+        const int tid = threadIdx.x;  // 0..127: owns d_out column o = tid (and tid + 128)
+        const int q = warp;
+        float* my = stg + warp * 32 * 32;
         int stage = 0;
         uint32_t phase = 0;
         uint32_t acc_phase = 0;
@@ -465,7 +487,7 @@ wgrad_tf32_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constan
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -481,8 +503,7 @@ cudaError_t set_smem(K kernel, int bytes) {
 cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float* bias, const int32_t* offsets,
                                 const int32_t* perm, int64_t T, int E, int H, int accumulate, float* out,
                                 uint32_t* dev_flags, int num_sms, cudaStream_t s) {
-    CUtensorMap tm_a, tm_b;
-    if (!make_map_2d(&tm_a, src, static_cast<uint64_t>(T), H, 32, 1)) return cudaErrorInvalidValue;
+    CUtensorMap tm_b;
     if (!make_map_2d(&tm_b, Bsrc, static_cast<uint64_t>(E) * H, H, 32, H)) return cudaErrorInvalidValue;
     const int64_t tiles = (T + 127) / 128 + E;
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
@@ -490,13 +511,13 @@ cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float
     if (H == 256) {
         err = set_smem(grouped_tf32_kernel<256>, GCfg<256>::SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        grouped_tf32_kernel<256><<<grid, kThreads, GCfg<256>::SMEM_BYTES, s>>>(
-            tm_a, tm_b, bias, offsets, perm, static_cast<int>(T), E, accumulate, out, dev_flags);
+        grouped_tf32_kernel<256><<<grid, kThreads, GCfg<256>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
+                                                                               accumulate, out, dev_flags);
     } else {
         err = set_smem(grouped_tf32_kernel<128>, GCfg<128>::SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        grouped_tf32_kernel<128><<<grid, kThreads, GCfg<128>::SMEM_BYTES, s>>>(
-            tm_a, tm_b, bias, offsets, perm, static_cast<int>(T), E, accumulate, out, dev_flags);
+        grouped_tf32_kernel<128><<<grid, kThreads, GCfg<128>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
+                                                                               accumulate, out, dev_flags);
     }
     return cudaGetLastError();
 }
@@ -504,21 +525,18 @@ cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float
 cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
                               int64_t T, int E, int H, float* part, float* part_db, uint32_t* dev_flags,
                               cudaStream_t s) {
-    CUtensorMap tm_g, tm_x;
-    if (!make_map_2d(&tm_g, d_out, static_cast<uint64_t>(T), H, 32, 1, true)) return cudaErrorInvalidValue;
-    if (!make_map_2d(&tm_x, x, static_cast<uint64_t>(T), H, 32, 1, true)) return cudaErrorInvalidValue;
     const int P = wgrad_splits(T);
     cudaError_t err;
     if (H == 256) {
         err = set_smem(wgrad_tf32_kernel<256>, WCfg<256>::SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        wgrad_tf32_kernel<256><<<P, kThreads, WCfg<256>::SMEM_BYTES, s>>>(tm_g, tm_x, offsets, perm,
+        wgrad_tf32_kernel<256><<<P, kThreads, WCfg<256>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
                                                                          static_cast<int>(T), E, P, part, part_db,
                                                                          dev_flags);
     } else {
         err = set_smem(wgrad_tf32_kernel<128>, WCfg<128>::SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        wgrad_tf32_kernel<128><<<P, kThreads, WCfg<128>::SMEM_BYTES, s>>>(tm_g, tm_x, offsets, perm,
+        wgrad_tf32_kernel<128><<<P, kThreads, WCfg<128>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
                                                                          static_cast<int>(T), E, P, part, part_db,
                                                                          dev_flags);
     }

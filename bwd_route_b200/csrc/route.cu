@@ -10,10 +10,12 @@
 // index, and a NaN at e = 0 pins the result to 0.
 //
 // Three launches, all integer-exact and deterministic:
-//   1. route_count   : argmax of 1024 tokens per block, per-block expert counts
-//                      (warp ballots, no atomics).
-//   2. route_scan    : one block: counts, offsets and every block's base
-//                      position inside each expert's segment.
+//   1. route_count   : the block's 1024 x E logits are staged in shared memory
+//                      with 128-bit loads; lane groups reduce (value, index)
+//                      pairs with warp shuffles; per-block expert counts come
+//                      from warp ballots (no atomics).
+//   2. route_scan    : one block, one warp per expert: counts, offsets and every
+//                      block's base position inside each expert's segment.
 //   3. route_scatter : per-token rank inside its block (warp ballots in token
 //                      order), perm[base + rank] = t.
 #include <cstdint>
@@ -41,17 +43,28 @@ template <int LPT>  // lanes per token: a power of two >= E
 __global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __restrict__ logits, int64_t T, int E,
                                                               int32_t* __restrict__ expert_idx,
                                                               int32_t* __restrict__ blk_counts) {
+    extern __shared__ float4 s_lg4[];  // the block's logits, kRouteTokPerBlk * E floats
+    const float* s_lg = reinterpret_cast<const float*>(s_lg4);
     __shared__ int s_idx[kRouteTokPerBlk];
     __shared__ int s_wcnt[kWarps][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokPerBlk;
+    const int ntok = static_cast<int>((T - t0 < kRouteTokPerBlk) ? (T - t0) : kRouteTokPerBlk);
+    {
+        // coalesced 128-bit staging; the block's first float is 16-byte aligned (1024 * E * 4 bytes per block)
+        const int nflt = ntok * E, n4 = nflt / 4;
+        const float4* g4 = reinterpret_cast<const float4*>(logits + t0 * E);
+        for (int i = threadIdx.x; i < n4; i += kThreads) s_lg4[i] = __ldg(g4 + i);
+        float* s_w = reinterpret_cast<float*>(s_lg4);
+        for (int i = n4 * 4 + threadIdx.x; i < nflt; i += kThreads) s_w[i] = __ldg(logits + t0 * E + i);
+    }
+    __syncthreads();
     constexpr int TPW = 32 / LPT;  // tokens per warp per step
     const int sub = lane % LPT;
     for (int base = warp * TPW; base < kRouteTokPerBlk; base += kWarps * TPW) {
         const int tl = base + lane / LPT;
-        const int64_t t = t0 + tl;
-        const bool in = (t < T) && (sub < E);
-        const float raw = in ? __ldg(logits + t * E + sub) : 0.0f;
+        const bool in = (tl < ntok) && (sub < E);
+        const float raw = in ? s_lg[tl * E + sub] : 0.0f;
         float v = raw;
         int e = sub;
         bool ok = in && !isnan(raw);
@@ -63,14 +76,12 @@ __global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __re
             const bool ook = __shfl_xor_sync(0xffffffffu, ok, off);
             combine(v, e, ok, ov, oe, ook);
         }
-        const int k = nan0 ? 0 : e;
-        if (sub == 0) {
-            s_idx[tl] = (t < T) ? k : -1;
-            if (t < T) expert_idx[t] = k;
-        }
+        if (sub == 0) s_idx[tl] = (tl < ntok) ? (nan0 ? 0 : e) : -1;
     }
     __syncthreads();
-    // per-warp counts over the warp's 128 consecutive tokens; lane e keeps expert e
+    // write expert_idx coalesced; per-warp counts over the warp's 128 consecutive
+    // tokens; lane e keeps expert e
+    for (int i = threadIdx.x; i < ntok; i += kThreads) expert_idx[t0 + i] = s_idx[i];
     int cnt = 0;
 #pragma unroll
     for (int it = 0; it < kTokPerWarp / 32; ++it) {
@@ -89,72 +100,56 @@ __global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __re
     }
 }
 
-// Exclusive scan of blk_counts[.][e] over blocks for every expert, plus counts
-// and offsets. One block of 1024 threads walks the blocks in chunks of 1024.
+// One block, warp e scans the per-block counts of expert e: blk_base[b][e] =
+// offsets[e] + sum_{b' < b} blk_counts[b'][e]; also counts and offsets.
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ blk_counts, int64_t nblk,
                                                          int E, int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ blk_base) {
-    __shared__ int s_warp[32];
-    __shared__ int s_tot[33];
+    __shared__ int s_tot[32];
+    __shared__ int s_off[33];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // totals per expert
-    for (int e = 0; e < E; ++e) {
-        int acc = 0;
-        for (int64_t b = threadIdx.x; b < nblk; b += blockDim.x) acc += blk_counts[b * E + e];
+    constexpr int kBatch = 8;  // chunks of 32 blocks loaded before they are scanned
+    if (warp < E) {
+        const int e = warp;
+        int carry = 0;
+        for (int64_t c0 = 0; c0 < nblk; c0 += 32 * kBatch) {
+            int v[kBatch];
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) s_warp[warp] = acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int tot = 0;
-            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_warp[w];
-            s_tot[e] = tot;
+            for (int j = 0; j < kBatch; ++j) {
+                const int64_t b = c0 + j * 32 + lane;
+                v[j] = (b < nblk) ? blk_counts[b * E + e] : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                int incl = v[j];
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += u;
+                }
+                const int64_t b = c0 + j * 32 + lane;
+                if (b < nblk) blk_base[b * E + e] = carry + incl - v[j];
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
         }
-        __syncthreads();
+        if (lane == 0) s_tot[e] = carry;
     }
+    __syncthreads();
     if (threadIdx.x == 0) {
         int run = 0;
         for (int e = 0; e < E; ++e) {
             counts[e] = s_tot[e];
             offsets[e] = run;
-            s_warp[e] = run;  // reuse as the running base of expert e
+            s_off[e] = run;
             run += s_tot[e];
         }
         offsets[E] = run;
-        for (int e = 0; e < E; ++e) s_tot[e] = s_warp[e];
     }
     __syncthreads();
-    for (int e = 0; e < E; ++e) {
-        int carry = s_tot[e];
-        for (int64_t c0 = 0; c0 < nblk; c0 += blockDim.x) {
-            const int64_t b = c0 + threadIdx.x;
-            const int v = (b < nblk) ? blk_counts[b * E + e] : 0;
-            int incl = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += u;
-            }
-            if (lane == 31) s_warp[warp] = incl;
-            __syncthreads();
-            if (warp == 0) {
-                const int nw = blockDim.x >> 5;
-                int w = (lane < nw) ? s_warp[lane] : 0;
-                int wi = w;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int u = __shfl_up_sync(0xffffffffu, wi, off);
-                    if (lane >= off) wi += u;
-                }
-                if (lane < nw) s_warp[lane] = wi - w;  // exclusive warp prefix
-                if (lane == nw - 1) s_tot[32] = wi;    // chunk total
-            }
-            __syncthreads();
-            if (b < nblk) blk_base[b * E + e] = carry + s_warp[warp] + incl - v;
-            carry += s_tot[32];
-            __syncthreads();
-        }
+    if (warp < E) {
+        const int add = s_off[warp];
+        for (int64_t b = lane; b < nblk; b += 32) blk_base[b * E + warp] += add;
     }
 }
 
@@ -204,17 +199,26 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
                          int32_t* offsets, int32_t* perm, int32_t* blk_counts, int32_t* blk_base,
                          cudaStream_t s) {
     const int64_t nblk = (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk;
+    const size_t smem = sizeof(float) * kRouteTokPerBlk * E;
     if (E <= 4)
-        route_count_kernel<4><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<4><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     else if (E <= 8)
-        route_count_kernel<8><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<8><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     else if (E <= 16)
-        route_count_kernel<16><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<16><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     else
-        route_count_kernel<32><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<32><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     route_scan_kernel<<<1, 1024, 0, s>>>(blk_counts, nblk, E, counts, offsets, blk_base);
     route_scatter_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(expert_idx, T, E, blk_base, perm);
     return cudaGetLastError();
+}
+
+cudaError_t route_set_smem_limits() {
+    cudaError_t e = cudaFuncSetAttribute(route_count_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(float) * kRouteTokPerBlk * 16));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(route_count_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(float) * kRouteTokPerBlk * 32));
 }
 
 }  // namespace moe
