@@ -23,25 +23,25 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTokPerThread = kAuxTokPerBlk / kThreads;  // 4
+constexpr int kThreads = kAuxTokPerBlk;  // one token per thread
+constexpr int kWarps = kThreads / 32;
 
 template <int EMAX>
-__global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(kThreads, 1) aux_kernel(const float* __restrict__ logits,
                                                       const int32_t* __restrict__ counts, int64_t T, int E,
                                                       const float* __restrict__ lambda_eff,
                                                       float* __restrict__ d_logits, float* __restrict__ blk_psum) {
     extern __shared__ float4 s_tile4[];  // kAuxTokPerBlk * E floats (logits, then gradients)
     float* s_tile = reinterpret_cast<float*>(s_tile4);
     __shared__ float s_frac[32];
-    __shared__ float s_part[kThreads / 32][EMAX];
+    __shared__ float s_part[kWarps][EMAX];
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kAuxTokPerBlk;
     const int64_t ntok = (T - t0 < kAuxTokPerBlk) ? (T - t0) : kAuxTokPerBlk;
     const int64_t nflt = ntok * E;
     const float* src = logits + t0 * E;
     // coalesced 128-bit staging (the block's first float is 16-byte aligned: 1024 * E * 4 bytes per block)
     const int64_t n4 = nflt / 4;
-    for (int64_t i = threadIdx.x; i < n4; i += kThreads) s_tile4[i] = __ldg(reinterpret_cast<const float4*>(src) + i);
+    stage_f4<2>(s_tile4, reinterpret_cast<const float4*>(src), static_cast<int>(n4), threadIdx.x, kThreads);
     for (int64_t i = n4 * 4 + threadIdx.x; i < nflt; i += kThreads) s_tile[i] = __ldg(src + i);
     if (threadIdx.x < E) s_frac[threadIdx.x] = static_cast<float>(counts[threadIdx.x]) / static_cast<float>(T);
     __syncthreads();
@@ -50,9 +50,8 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
     float psum[EMAX];
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) psum[e] = 0.0f;
-    for (int j = 0; j < kTokPerThread; ++j) {
-        const int tl = j * kThreads + threadIdx.x;
-        if (tl >= ntok) break;
+    const int tl = threadIdx.x;  // this thread's token in the block
+    if (tl < ntok) {
         float* row = s_tile + static_cast<int64_t>(tl) * E;
         float p[EMAX];
         float m = row[0];
@@ -78,7 +77,7 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
 #pragma unroll
         for (int e = 0; e < EMAX; ++e) {
             if (e < E) {
-                psum[e] += p[e];
+                psum[e] = p[e];
                 row[e] = scale * (p[e] * (s_frac[e] - g));
             }
         }
@@ -95,7 +94,7 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
     __syncthreads();
     if (threadIdx.x < E) {
         float acc = s_part[0][threadIdx.x];
-        for (int w = 1; w < kThreads / 32; ++w) acc += s_part[w][threadIdx.x];
+        for (int w = 1; w < kWarps; ++w) acc += s_part[w][threadIdx.x];
         blk_psum[static_cast<int64_t>(blockIdx.x) * E + threadIdx.x] = acc;
     }
     if (d_logits) {
@@ -114,13 +113,31 @@ __global__ void __launch_bounds__(1024) aux_finalize_kernel(const float* __restr
                                                            float* __restrict__ loss_out, float* __restrict__ mean_p,
                                                            float* __restrict__ stats) {
     __shared__ float s_mean[32];
+    __shared__ double s_hf[32], s_hm[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp < E) {
         double acc = 0.0;
-        for (int64_t b = lane; b < nblk; b += 32) acc += static_cast<double>(blk_psum[b * E + warp]);
+        for (int64_t b0 = 0; b0 < nblk; b0 += 8 * 32) {
+            float v[8];  // eight independent loads, then added in block order
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t b = b0 + u * 32 + lane;
+                v[u] = (b < nblk) ? blk_psum[b * E + warp] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (b0 + u * 32 + lane < nblk) acc += static_cast<double>(v[u]);
+        }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) s_mean[warp] = T > 0 ? static_cast<float>(acc / static_cast<double>(T)) : 0.0f;
+        if (lane == 0) {
+            const float m = T > 0 ? static_cast<float>(acc / static_cast<double>(T)) : 0.0f;
+            s_mean[warp] = m;
+            // entropy terms of expert `warp` (0 ln 0 = 0)
+            const double f = T > 0 ? static_cast<double>(counts[warp]) / static_cast<double>(T) : 0.0;
+            s_hf[warp] = f > 0.0 ? f * log(f) : 0.0;
+            s_hm[warp] = m > 0.0f ? static_cast<double>(m) * log(static_cast<double>(m)) : 0.0;
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -128,9 +145,8 @@ __global__ void __launch_bounds__(1024) aux_finalize_kernel(const float* __restr
         double acc = 0.0, hf = 0.0, hm = 0.0;
         for (int e = 0; e < E; ++e) {
             acc += static_cast<double>(counts[e]) * static_cast<double>(s_mean[e]);
-            const double f = T > 0 ? static_cast<double>(counts[e]) / static_cast<double>(T) : 0.0;
-            if (f > 0.0) hf -= f * log(f);
-            if (s_mean[e] > 0.0f) hm -= static_cast<double>(s_mean[e]) * log(static_cast<double>(s_mean[e]));
+            hf -= s_hf[e];
+            hm -= s_hm[e];
         }
         const float aux_raw = T > 0 ? static_cast<float>(static_cast<double>(E) * acc / static_cast<double>(T)) : 0.0f;
         loss_out[0] = aux_raw;

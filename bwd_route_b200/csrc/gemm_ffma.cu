@@ -248,7 +248,25 @@ struct PairwiseSum {
     }
 };
 
-constexpr int kBatch = 8;
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+// Sum of n slots (slot k at src[k * stride]) in a fixed tree: slots are taken in
+// groups of eight added as ((s0+s1)+(s2+s3))+((s4+s5)+(s6+s7)) (missing slots of
+// the last group count as 0), and the group sums are added pairwise. The eight
+// loads of a group are independent, so they are in flight together.
+__device__ __forceinline__ float4 sum_slots(const float4* __restrict__ src, int64_t stride, int n) {
+    PairwiseSum ps;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = 0; k0 < n; k0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = (k0 + u < n) ? __ldg(src + static_cast<int64_t>(k0 + u) * stride) : z;
+        ps.add(add4(add4(add4(v[0], v[1]), add4(v[2], v[3])), add4(add4(v[4], v[5]), add4(v[6], v[7]))));
+    }
+    return ps.result();
+}
 
 // grid.x: float4 groups of dW[e] (plus one trailing block for db), grid.y = E.
 __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ part,
@@ -258,20 +276,21 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
                                                           float* __restrict__ db, int acc_dw, int acc_db) {
     __shared__ int s_c[2];
     const int e = blockIdx.y;
+    // the ranges c that overlap expert e's tokens [a, b) are contiguous: thread c
+    // tests range c (P <= blockDim.x) and the first / last overlapping one record it
+    const int64_t a = offsets[e], b = offsets[e + 1];
     if (threadIdx.x == 0) {
-        const int64_t a = offsets[e], b = offsets[e + 1];
-        int c_lo = 0, c_hi = -1;
-        if (a < b) {
-            c_lo = P;
-            for (int c = 0; c < P; ++c) {
-                if (split_lo(c, T, P) < b && split_lo(c + 1, T, P) > a) {
-                    if (c < c_lo) c_lo = c;
-                    c_hi = c;
-                }
-            }
+        s_c[0] = 0;
+        s_c[1] = -1;
+    }
+    __syncthreads();
+    if (a < b && static_cast<int>(threadIdx.x) < P) {
+        const int c = threadIdx.x;
+        const int64_t lo = split_lo(c, T, P), hi = split_lo(c + 1, T, P);
+        if (lo < b && hi > a) {
+            if (lo <= a) s_c[0] = c;      // the range that holds token a
+            if (hi >= b) s_c[1] = c;      // the range that holds token b - 1
         }
-        s_c[0] = c_lo;
-        s_c[1] = c_hi;
     }
     __syncthreads();
     const int c_lo = s_c[0], c_hi = s_c[1];
@@ -281,20 +300,8 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
         if (!dW) return;
         const int64_t j = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;  // float4 index
         if (j >= HH / 4) return;
-        PairwiseSum ps;
-        const float4* src = reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c_lo) + e) * HH) + j;
-        const int64_t stride4 = HH / 4;
-        for (int c0 = c_lo; c0 <= c_hi; c0 += kBatch) {
-            // issue a batch of independent loads, then add them in slot order
-            float4 v[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-                if (c0 + u <= c_hi) v[u] = __ldg(src + static_cast<int64_t>(c0 - c_lo + u) * stride4);
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-                if (c0 + u <= c_hi) ps.add(v[u]);
-        }
-        float4 r = ps.result();
+        float4 r = sum_slots(reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c_lo) + e) * HH) + j,
+                             HH / 4, c_hi - c_lo + 1);
         float4* dst = reinterpret_cast<float4*>(dW + e * HH) + j;
         if (acc_dw) {
             const float4 o = *dst;
@@ -305,10 +312,8 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
         if (!db) return;
         const int j = threadIdx.x;  // float4 index into db[e]
         if (j >= H / 4) return;
-        PairwiseSum ps;
-        for (int c = c_lo; c <= c_hi; ++c)
-            ps.add(__ldg(reinterpret_cast<const float4*>(part_db + (static_cast<int64_t>(c) + e) * H) + j));
-        float4 r = ps.result();
+        float4 r = sum_slots(reinterpret_cast<const float4*>(part_db + (static_cast<int64_t>(c_lo) + e) * H) + j,
+                             H / 4, c_hi - c_lo + 1);
         float4* dst = reinterpret_cast<float4*>(db + static_cast<int64_t>(e) * H) + j;
         if (acc_db) {
             const float4 o = *dst;

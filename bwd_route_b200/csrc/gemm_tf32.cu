@@ -19,8 +19,8 @@
 //
 //   grouped_tf32_kernel : persistent, one CTA per SM; a tile is 128 sorted
 //     tokens x all H outputs. Warps 4-7 gather the tile's rows (K-major,
-//     128-byte swizzle), one thread also loads the expert's weight slab by TMA;
-//     warp 8 issues tcgen05.mma kind::tf32 (M=128, N=H, K=8) into one of two
+//     128-byte swizzle) into a 6-deep ring; warp 9 streams the expert's weight
+//     slab by TMA into a 3-deep ring (it comes from L2); warp 8 issues tcgen05.mma kind::tf32 (M=128, N=H, K=8) into one of two
 //     TMEM accumulators; warps 0-3 drain the other accumulator (tcgen05.ld),
 //     add the bias and store the rows to their original token positions with
 //     coalesced 128-byte stores.
@@ -45,10 +45,19 @@
 namespace moe {
 namespace {
 
-// warps 0-3: epilogue (TMEM lane quadrant = warp), 4-7: producers, 8: MMA + TMEM owner
+// Weight gradient: warps 0-3 db + epilogue (TMEM lane quadrant = warp), 4-7
+// row-gather producers, 8 MMA issuer + TMEM owner.
 constexpr int kThreads = 288;
 constexpr int kProducer0 = 128;
 constexpr int kMmaWarp = 8;
+// Grouped GEMM: warps 0-7 epilogue (warp w drains TMEM lane quadrant w % 4,
+// column half w / 4), 8-11 row-gather producers, 12 MMA issuer + TMEM owner,
+// 13 weight-slab TMA loader.
+constexpr int kThreadsGrouped = 448;
+constexpr int kGEpiWarps = 8;
+constexpr int kGProducer0 = 256;
+constexpr int kGMmaWarp = 12;
+constexpr int kGBLoadWarp = 13;
 constexpr int kMaxStages = 8;
 
 struct __align__(8) Ctl {
@@ -63,18 +72,37 @@ struct __align__(8) Ctl {
 };
 
 // ------------------------------------------------------------------ grouped GEMM
+// Two shared-memory rings: the gathered token rows (A, from HBM, long latency:
+// deep ring) and the expert's weight slab (B, from L2: shallow ring). Each
+// k-chunk is 32 fp32 = one 128-byte swizzle row of K.
+// Barriers of the grouped GEMM: one full/empty pair per stage of each ring,
+// and the full/empty pair of each TMEM accumulator.
+struct __align__(8) GCtl {
+    uint64_t afull[kMaxStages];
+    uint64_t aempty[kMaxStages];
+    uint64_t bfull[kMaxStages];
+    uint64_t bempty[kMaxStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort;
+    int off[33];
+    int tstart[33];
+};
+
 template <int H>
 struct GCfg {
     static constexpr int BM = 128;
-    static constexpr int KCH = H / 32;                // 32 fp32 = one 128-byte swizzle row
+    static constexpr int KCH = H / 32;
     static constexpr int A_BYTES = BM * 128;          // 16 KiB
     static constexpr int B_BYTES = H * 128;           // 16 / 32 KiB
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (H == 256) ? 4 : 6;
-    static constexpr int STG_BYTES = 4 * 32 * 128;    // epilogue staging: 4 warps x 32 rows x 128 B
-    static constexpr int TMEM_COLS = 2 * H;           // two accumulators
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + static_cast<int>(sizeof(Ctl));
-    static_assert(STAGES <= kMaxStages, "stages");
+    static constexpr int A_STAGES = (H == 256) ? 6 : 8;
+    static constexpr int B_STAGES = (H == 256) ? 3 : 4;
+    static constexpr int RING_BYTES = A_STAGES * A_BYTES + B_STAGES * B_BYTES;
+    static constexpr int STG_BYTES = kGEpiWarps * 32 * 128;  // epilogue staging: 32 rows x 128 B per warp
+    static constexpr int TMEM_COLS = 2 * H;                  // two accumulators
+    static constexpr int SMEM_BYTES = 1024 + RING_BYTES + STG_BYTES + static_cast<int>(sizeof(GCtl));
+    static_assert(A_STAGES <= kMaxStages && B_STAGES <= kMaxStages, "stages");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -85,7 +113,7 @@ __device__ __forceinline__ int find_expert(const int* tstart, int E, int tile) {
 }
 
 template <int H>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsGrouped, 1)
 grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUtensorMap tm_b,
                     const float* __restrict__ bias, const int32_t* __restrict__ offsets,
                     const int32_t* __restrict__ perm, int E, int accumulate, float* __restrict__ out,
@@ -93,26 +121,31 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
     using C = GCfg<H>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* stages = smem;
-    float* stg = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
-    Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES);
+    uint8_t* aring = smem;
+    uint8_t* bring = smem + C::A_STAGES * C::A_BYTES;
+    float* stg = reinterpret_cast<float*>(smem + C::RING_BYTES);
+    GCtl* ctl = reinterpret_cast<GCtl*>(smem + C::RING_BYTES + C::STG_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&ctl->full[s], 128 + 1);  // 128 gather threads + the weight-slab thread
-            mbar_init(&ctl->empty[s], 1);       // tcgen05.commit
+        for (int s = 0; s < C::A_STAGES; ++s) {
+            mbar_init(&ctl->afull[s], 128);  // 128 gather threads
+            mbar_init(&ctl->aempty[s], 1);   // tcgen05.commit
+        }
+        for (int s = 0; s < C::B_STAGES; ++s) {
+            mbar_init(&ctl->bfull[s], 1);    // arrive.expect_tx + TMA bytes
+            mbar_init(&ctl->bempty[s], 1);   // tcgen05.commit
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], 4);
+            mbar_init(&ctl->tempty[b], kGEpiWarps);
         }
         ctl->abort = 0;
         fence_mbar_init();
     }
     if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
-    if (threadIdx.x == kProducer0) tma_prefetch_desc(&tm_b);
-    if (warp == kMmaWarp) {
+    if (warp == kGBLoadWarp && lane == 0) tma_prefetch_desc(&tm_b);
+    if (warp == kGMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -132,9 +165,9 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
     const int ntiles = ctl->tstart[E];
     volatile int* abort = &ctl->abort;
 
-    if (warp >= 4 && warp < 8) {
-        // ---------------- producers: cp.async row gather (+ TMA weight slab)
-        const int ptid = threadIdx.x - kProducer0;  // 0..127
+    if (warp >= kGProducer0 / 32 && warp < kGProducer0 / 32 + 4) {
+        // ---------------- producers: cp.async row gather
+        const int ptid = threadIdx.x - kGProducer0;  // 0..127
         const int prow = ptid >> 3, pg = ptid & 7;  // row within a 16-row block, 16-byte granule
         int tok[8], nxt[8];
         auto load_tokens = [&](int tile, int (&t)[8]) {
@@ -148,20 +181,14 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
             }
         };
         if (static_cast<int>(blockIdx.x) < ntiles) load_tokens(blockIdx.x, tok);
-        int stage = 0;
-        uint32_t phase = 0;
+        int sa = 0;
+        uint32_t pa = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-            const int e = find_expert(ctl->tstart, E, tile);
             if (tile + static_cast<int>(gridDim.x) < ntiles) load_tokens(tile + gridDim.x, nxt);
             for (int kc = 0; kc < C::KCH; ++kc) {
-                if (!(ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags))) break;
-                uint8_t* a = stages + stage * C::STAGE_BYTES;
-                if (ptid == 0) {
-                    mbar_arrive_expect_tx(&ctl->full[stage], C::B_BYTES);
-                    tma_load_2d(a + C::A_BYTES, &tm_b, kc * 32, e * H, &ctl->full[stage]);
-                }
-                const uint32_t a_u32 = smem_u32(a);
+                if (!(ok = mbar_wait(&ctl->aempty[sa], pa ^ 1, abort, dev_flags))) break;
+                const uint32_t a_u32 = smem_u32(aring + sa * C::A_BYTES);
 #pragma unroll
                 for (int it = 0; it < 8; ++it) {
                     const int r = it * 16 + prow;
@@ -169,21 +196,41 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                     const float* gsrc = src + static_cast<int64_t>(t < 0 ? 0 : t) * H + kc * 32 + pg * 4;
                     cp_async_16(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), gsrc, t < 0 ? 0u : 16u);
                 }
-                cp_async_arrive_noinc(&ctl->full[stage]);
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1;
+                cp_async_arrive_noinc(&ctl->afull[sa]);
+                if (++sa == C::A_STAGES) {
+                    sa = 0;
+                    pa ^= 1;
                 }
             }
 #pragma unroll
             for (int it = 0; it < 8; ++it) tok[it] = nxt[it];
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kGBLoadWarp) {
+        // ---------------- weight-slab loader: TMA, at most B_STAGES chunks ahead of the MMA
+        if (lane == 0) {
+            int sb = 0;
+            uint32_t pb = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int e = find_expert(ctl->tstart, E, tile);
+                for (int kc = 0; kc < C::KCH; ++kc) {
+                    if (!(ok = mbar_wait(&ctl->bempty[sb], pb ^ 1, abort, dev_flags))) break;
+                    mbar_arrive_expect_tx(&ctl->bfull[sb], C::B_BYTES);
+                    tma_load_2d(bring + sb * C::B_BYTES, &tm_b, kc * 32, e * H, &ctl->bfull[sb]);
+                    if (++sb == C::B_STAGES) {
+                        sb = 0;
+                        pb ^= 1;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kGMmaWarp) {
         // ---------------- MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_tf32(128, H, 0, 0);
-            int stage = 0;
-            uint32_t phase = 0;
+            int sa = 0, sb = 0;
+            uint32_t pa = 0, pb = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
@@ -192,19 +239,25 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * H);
                 for (int kc = 0; kc < C::KCH; ++kc) {
-                    if (!(ok = mbar_wait(&ctl->full[stage], phase, abort, dev_flags))) break;
+                    if (!(ok = mbar_wait(&ctl->afull[sa], pa, abort, dev_flags))) break;
+                    if (!(ok = mbar_wait(&ctl->bfull[sb], pb, abort, dev_flags))) break;
                     fence_proxy_async_smem();
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(stages + stage * C::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + C::A_BYTES;
+                    const uint32_t a_addr = smem_u32(aring + sa * C::A_BYTES);
+                    const uint32_t b_addr = smem_u32(bring + sb * C::B_BYTES);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_tf32(d, sw128_desc(a_addr + ks * 32, 16, 1024), sw128_desc(b_addr + ks * 32, 16, 1024),
                                  idesc, (kc | ks) != 0 ? 1u : 0u);
-                    mma_commit(&ctl->empty[stage]);
-                    if (++stage == C::STAGES) {
-                        stage = 0;
-                        phase ^= 1;
+                    mma_commit(&ctl->aempty[sa]);
+                    mma_commit(&ctl->bempty[sb]);
+                    if (++sa == C::A_STAGES) {
+                        sa = 0;
+                        pa ^= 1;
+                    }
+                    if (++sb == C::B_STAGES) {
+                        sb = 0;
+                        pb ^= 1;
                     }
                 }
                 if (!ok) break;
@@ -214,10 +267,14 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
             }
         }
         __syncwarp();
-    } else if (warp < 4) {
-        // ---------------- epilogue: TMEM -> registers -> smem transpose -> rows
-        const int q = warp;  // TMEM lane quadrant
+    } else if (warp < kGEpiWarps) {
+        // ---------------- epilogue: TMEM -> registers -> smem transpose -> rows.
+        // Warp w owns TMEM lanes 32 (w % 4) .. +31 (tile rows) and the column half w / 4.
+        constexpr int HALF = H / 2;
+        const int q = warp & 3;
+        const int c0 = (warp >> 2) * HALF;
         float* my = stg + warp * 32 * 32;
+        const int j = lane & 7;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -226,45 +283,54 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
             const int nrows = min(C::BM, ctl->off[e + 1] - row0);
             const int myrow = 32 * q + lane;
             const int tok_mine = (myrow < nrows) ? perm[row0 + myrow] : -1;
+            // the bias this lane adds in each 32-column chunk, loaded before the wait
+            float4 bv[HALF / 32];
+#pragma unroll
+            for (int c = 0; c < HALF / 32; ++c)
+                bv[c] = bias ? __ldg(reinterpret_cast<const float4*>(bias + static_cast<int64_t>(e) * H + c0 + c * 32) + j)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, abort, dev_flags)) break;
             __syncwarp();
             tc_fence_after();
-            const int j = lane & 7;
-#pragma unroll 1
-            for (int c = 0; c < H / 32; ++c) {
-                float v[32];
-                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * H + c * 32), v);
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj)
-                    *reinterpret_cast<float4*>(my + lane * 32 + ((jj ^ (lane & 7)) * 4)) =
-                        make_float4(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3]);
-                __syncwarp();
-                float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (bias) bv = __ldg(reinterpret_cast<const float4*>(bias + static_cast<int64_t>(e) * H + c * 32) + j);
+            for (int cc = 0; cc < HALF / 64; ++cc) {
+                float v[64];
+                tmem_ld_32x32b_x64(tmem + (static_cast<uint32_t>(32 * q) << 16) +
+                                       static_cast<uint32_t>(acc * H + c0 + cc * 64), v);
 #pragma unroll
-                for (int it = 0; it < 8; ++it) {
-                    const int R = it * 4 + (lane >> 3);
-                    float4 val = *reinterpret_cast<const float4*>(my + R * 32 + ((j ^ (R & 7)) * 4));
-                    const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
-                    if (tok >= 0) {
-                        val.x += bv.x;
-                        val.y += bv.y;
-                        val.z += bv.z;
-                        val.w += bv.w;
-                        float* dst = out + static_cast<int64_t>(tok) * H + c * 32 + j * 4;
-                        if (accumulate) {
-                            const float4 o = *reinterpret_cast<const float4*>(dst);
-                            val.x += o.x;
-                            val.y += o.y;
-                            val.z += o.z;
-                            val.w += o.w;
-                            *reinterpret_cast<float4*>(dst) = val;
-                        } else {
-                            st_global_cs_v4(dst, val);
+                for (int h = 0; h < 2; ++h) {
+                    const int c = cc * 2 + h;  // 32-column chunk within the half
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        *reinterpret_cast<float4*>(my + lane * 32 + ((jj ^ (lane & 7)) * 4)) =
+                            make_float4(v[32 * h + 4 * jj], v[32 * h + 4 * jj + 1], v[32 * h + 4 * jj + 2],
+                                        v[32 * h + 4 * jj + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int it = 0; it < 8; ++it) {
+                        const int R = it * 4 + (lane >> 3);
+                        float4 val = *reinterpret_cast<const float4*>(my + R * 32 + ((j ^ (R & 7)) * 4));
+                        const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
+                        if (tok >= 0) {
+                            val.x += bv[c].x;
+                            val.y += bv[c].y;
+                            val.z += bv[c].z;
+                            val.w += bv[c].w;
+                            float* dst = out + static_cast<int64_t>(tok) * H + c0 + c * 32 + j * 4;
+                            if (accumulate) {
+                                const float4 o = *reinterpret_cast<const float4*>(dst);
+                                val.x += o.x;
+                                val.y += o.y;
+                                val.z += o.z;
+                                val.w += o.w;
+                                *reinterpret_cast<float4*>(dst) = val;
+                            } else {
+                                st_global_cs_v4(dst, val);
+                            }
                         }
                     }
+                    __syncwarp();
                 }
-                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
@@ -275,7 +341,7 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == kGMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -511,12 +577,12 @@ cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float
     if (H == 256) {
         err = set_smem(grouped_tf32_kernel<256>, GCfg<256>::SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        grouped_tf32_kernel<256><<<grid, kThreads, GCfg<256>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
+        grouped_tf32_kernel<256><<<grid, kThreadsGrouped, GCfg<256>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
                                                                                accumulate, out, dev_flags);
     } else {
         err = set_smem(grouped_tf32_kernel<128>, GCfg<128>::SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        grouped_tf32_kernel<128><<<grid, kThreads, GCfg<128>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
+        grouped_tf32_kernel<128><<<grid, kThreadsGrouped, GCfg<128>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
                                                                                accumulate, out, dev_flags);
     }
     return cudaGetLastError();

@@ -26,9 +26,11 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;                 // route_scatter
 constexpr int kWarps = kThreads / 32;
 constexpr int kTokPerWarp = kRouteTokPerBlk / kWarps;  // 128
+constexpr int kCountThreads = 1024;           // route_count: one block of 32 warps per 1024 tokens
+constexpr int kCountWarps = kCountThreads / 32;
 
 __device__ __forceinline__ void combine(float& v, int& e, bool& ok, float ov, int oe, bool ook) {
     const bool take = ook && (!ok || ov > v || (ov == v && oe < e));
@@ -40,28 +42,27 @@ __device__ __forceinline__ void combine(float& v, int& e, bool& ok, float ov, in
 }
 
 template <int LPT>  // lanes per token: a power of two >= E
-__global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __restrict__ logits, int64_t T, int E,
+__global__ void __launch_bounds__(kCountThreads, 1) route_count_kernel(const float* __restrict__ logits, int64_t T, int E,
                                                               int32_t* __restrict__ expert_idx,
                                                               int32_t* __restrict__ blk_counts) {
     extern __shared__ float4 s_lg4[];  // the block's logits, kRouteTokPerBlk * E floats
     const float* s_lg = reinterpret_cast<const float*>(s_lg4);
     __shared__ int s_idx[kRouteTokPerBlk];
-    __shared__ int s_wcnt[kWarps][32];
+    __shared__ int s_wcnt[kCountWarps][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokPerBlk;
     const int ntok = static_cast<int>((T - t0 < kRouteTokPerBlk) ? (T - t0) : kRouteTokPerBlk);
     {
         // coalesced 128-bit staging; the block's first float is 16-byte aligned (1024 * E * 4 bytes per block)
         const int nflt = ntok * E, n4 = nflt / 4;
-        const float4* g4 = reinterpret_cast<const float4*>(logits + t0 * E);
-        for (int i = threadIdx.x; i < n4; i += kThreads) s_lg4[i] = __ldg(g4 + i);
+        stage_f4<2>(s_lg4, reinterpret_cast<const float4*>(logits + t0 * E), n4, threadIdx.x, kCountThreads);
         float* s_w = reinterpret_cast<float*>(s_lg4);
-        for (int i = n4 * 4 + threadIdx.x; i < nflt; i += kThreads) s_w[i] = __ldg(logits + t0 * E + i);
+        for (int i = n4 * 4 + threadIdx.x; i < nflt; i += kCountThreads) s_w[i] = __ldg(logits + t0 * E + i);
     }
     __syncthreads();
     constexpr int TPW = 32 / LPT;  // tokens per warp per step
     const int sub = lane % LPT;
-    for (int base = warp * TPW; base < kRouteTokPerBlk; base += kWarps * TPW) {
+    for (int base = warp * TPW; base < kRouteTokPerBlk; base += kCountWarps * TPW) {
         const int tl = base + lane / LPT;
         const bool in = (tl < ntok) && (sub < E);
         const float raw = in ? s_lg[tl * E + sub] : 0.0f;
@@ -79,29 +80,28 @@ __global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __re
         if (sub == 0) s_idx[tl] = (tl < ntok) ? (nan0 ? 0 : e) : -1;
     }
     __syncthreads();
-    // write expert_idx coalesced; per-warp counts over the warp's 128 consecutive
+    // write expert_idx coalesced; per-warp counts over the warp's 32 consecutive
     // tokens; lane e keeps expert e
-    for (int i = threadIdx.x; i < ntok; i += kThreads) expert_idx[t0 + i] = s_idx[i];
+    const int k = s_idx[threadIdx.x];
+    if (threadIdx.x < ntok) expert_idx[t0 + threadIdx.x] = k;
     int cnt = 0;
-#pragma unroll
-    for (int it = 0; it < kTokPerWarp / 32; ++it) {
-        const int k = s_idx[warp * kTokPerWarp + it * 32 + lane];
-        for (int e = 0; e < E; ++e) {
-            const int c = __popc(__ballot_sync(0xffffffffu, k == e));
-            if (lane == e) cnt += c;
-        }
+    for (int e = 0; e < E; ++e) {
+        const int c = __popc(__ballot_sync(0xffffffffu, k == e));
+        if (lane == e) cnt = c;
     }
     s_wcnt[warp][lane] = cnt;
     __syncthreads();
     if (threadIdx.x < E) {
         int total = 0;
-        for (int w = 0; w < kWarps; ++w) total += s_wcnt[w][threadIdx.x];
+        for (int w = 0; w < kCountWarps; ++w) total += s_wcnt[w][threadIdx.x];
         blk_counts[static_cast<int64_t>(blockIdx.x) * E + threadIdx.x] = total;
     }
 }
 
 // One block, warp e scans the per-block counts of expert e: blk_base[b][e] =
-// offsets[e] + sum_{b' < b} blk_counts[b'][e]; also counts and offsets.
+// offsets[e] + sum_{b' < b} blk_counts[b'][e]; also counts and offsets. Two
+// passes over the counts (totals, then the scan with the expert's offset), each
+// with batches of independent loads.
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ blk_counts, int64_t nblk,
                                                          int E, int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
@@ -109,10 +109,38 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
     __shared__ int s_tot[32];
     __shared__ int s_off[33];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kBatch = 8;  // chunks of 32 blocks loaded before they are scanned
+    constexpr int kBatch = 8;  // chunks of 32 blocks loaded before they are used
+    if (warp < E) {
+        int tot = 0;
+        for (int64_t c0 = 0; c0 < nblk; c0 += 32 * kBatch) {
+            int v[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int64_t b = c0 + j * 32 + lane;
+                v[j] = (b < nblk) ? blk_counts[b * E + warp] : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) tot += v[j];
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
+        if (lane == 0) s_tot[warp] = tot;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            counts[e] = s_tot[e];
+            offsets[e] = run;
+            s_off[e] = run;
+            run += s_tot[e];
+        }
+        offsets[E] = run;
+    }
+    __syncthreads();
     if (warp < E) {
         const int e = warp;
-        int carry = 0;
+        int carry = s_off[e];
         for (int64_t c0 = 0; c0 < nblk; c0 += 32 * kBatch) {
             int v[kBatch];
 #pragma unroll
@@ -133,23 +161,6 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
                 carry += __shfl_sync(0xffffffffu, incl, 31);
             }
         }
-        if (lane == 0) s_tot[e] = carry;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            counts[e] = s_tot[e];
-            offsets[e] = run;
-            s_off[e] = run;
-            run += s_tot[e];
-        }
-        offsets[E] = run;
-    }
-    __syncthreads();
-    if (warp < E) {
-        const int add = s_off[warp];
-        for (int64_t b = lane; b < nblk; b += 32) blk_base[b * E + warp] += add;
     }
 }
 
@@ -201,13 +212,13 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
     const int64_t nblk = (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk;
     const size_t smem = sizeof(float) * kRouteTokPerBlk * E;
     if (E <= 4)
-        route_count_kernel<4><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<4><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     else if (E <= 8)
-        route_count_kernel<8><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<8><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     else if (E <= 16)
-        route_count_kernel<16><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<16><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     else
-        route_count_kernel<32><<<(unsigned)nblk, kThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<32><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
     route_scan_kernel<<<1, 1024, 0, s>>>(blk_counts, nblk, E, counts, offsets, blk_base);
     route_scatter_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(expert_idx, T, E, blk_base, perm);
     return cudaGetLastError();
