@@ -28,8 +28,9 @@ _STATUS = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED_SHAPE", "MOE_ER
 EXPORTED = [
     "moe_top1_workspace_bytes", "moe_top1_workspace_init", "moe_top1_route", "moe_top1_fwd",
     "moe_top1_bwd", "moe_aux_loss_fwd_bwd", "moe_lambda_eff_update", "moe_top1_device_flags",
-    "moe_status_string", "moe_top1_abi_version",
+    "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc",
 ]
+MOE_NOALLOC_MAX_TOKENS = 2097152
 
 
 class MoeError(RuntimeError):
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.argtypes = [I32]
         L.moe_top1_abi_version.restype = I32
         L.moe_top1_abi_version.argtypes = []
+        L.moe_top1_route_noalloc.restype = I32
+        L.moe_top1_route_noalloc.argtypes = [P, I64, I64, I32, ctypes.POINTER(RoutingC), P]
         _lib = L
     return _lib
 
@@ -147,6 +150,16 @@ def moe_top1_route(gate_logits: torch.Tensor, B: int, N_H: int, E: int, routing:
     rc = routing.c()
     _check("moe_top1_route", lib().moe_top1_route(_ptr(gate_logits, torch.float32), B, N_H, E, ctypes.byref(rc),
                                                   _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_top1_route_noalloc(gate_logits: torch.Tensor, B: int, N_H: int, E: int, routing: Routing, stream=None):
+    """Routing without a workspace, for callers that cannot allocate device memory:
+    the routing scratch lives in a fixed 512 KiB device array inside the library
+    (at most MOE_NOALLOC_MAX_TOKENS tokens). Calls that may overlap on the GPU
+    share that array and must be ordered by the caller."""
+    rc = routing.c()
+    _check("moe_top1_route_noalloc", lib().moe_top1_route_noalloc(_ptr(gate_logits, torch.float32), B, N_H, E,
+                                                                  ctypes.byref(rc), _stream(stream)))
 
 
 def moe_top1_fwd(x, W, bias, routing: Routing, B: int, N_H: int, E: int, H: int, math: int, routed,

@@ -104,6 +104,30 @@ moe_status_t moe_top1_route(const float* gate_logits, int64_t B, int64_t N_H, in
                             void* stream);
 
 /*
+ * Routing without a workspace. The pages have no counterpart: this entry point
+ * exists for callers that cannot allocate device memory -- a plug-in whose host
+ * framework hands it only input and output tensors and owns every byte of
+ * device memory, or a runtime that plans all of its device memory up front and
+ * allows no allocation while it runs. Same arguments (minus the workspace),
+ * outputs and exact results as moe_top1_route; the per-block scratch of the
+ * routing kernels lives in a fixed device array inside the library instead:
+ * 512 KiB on every GPU that loads the library, held until the process exits.
+ * Limits: T = B * N_H <= MOE_NOALLOC_MAX_TOKENS and E <= 32; a larger call
+ * returns MOE_ERR_UNSUPPORTED_SHAPE and launches nothing.
+ * The first call on a device looks up the array's device address and sets
+ * kernel attributes, with that device current; make that first call before
+ * any stream capture.
+ * All calls share the one array: calls that can run on the GPU at the same time
+ * (other streams, other host threads) race on it, so the caller must order them.
+ * The array keeps the last call's contents; the kernels overwrite every entry
+ * they read, so nothing needs clearing between calls. Allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library call).
+ */
+#define MOE_NOALLOC_MAX_TOKENS 2097152
+moe_status_t moe_top1_route_noalloc(const float* gate_logits, int64_t B, int64_t N_H, int32_t E,
+                                    const moe_routing_t* out, void* stream);
+
+/*
  * Forward. [P1] kernel list ("apply its [H, H] linear to fused_ctx") and
  * PERFORMANCE (one output channel = a dot product over the H inputs):
  *   routed[t, o] = sum_i W[e*, o, i] * x[t, i] + bias[e*, o],  e* = expert_idx[t].
