@@ -2,9 +2,9 @@
 // adaptive lambda controller.
 //
 // foxhunt commit 11b96dac6a ("Top-1 Mixture-of-Experts gate per Switch
-// Transformer"), kernel list and ARCHITECTURE: softmax of the gate logits and
-// aux = frac . prob_mean x N_EXPERTS, where frac comes from the
-// non-differentiable top-1 choice (straight-through: only prob_mean carries
+// Transformer"), kernel list and ARCHITECTURE: a softmax of the gate logits and
+// the balance loss aux = E * sum_e frac_e * mean_p_e, where frac comes from the
+// non-differentiable top-1 choice (straight-through: only mean_p carries
 // gradient). foxhunt commit 2d0e6b6bdc ("Replace static moe_lambda=0.01 with a
 // GPU-driven controller"): lambda_eff = floor + max_extra * max(0, target -
 // ent_ema) / target, read by the loss kernel from device memory. foxhunt commit

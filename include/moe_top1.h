@@ -90,9 +90,9 @@ size_t moe_top1_workspace_bytes(int64_t T, int32_t E, int32_t H);
 moe_status_t moe_top1_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Routing. [P1] kernel list ("select top-1 expert from gate_logits") and
- * PERFORMANCE ("Top-1 chosen by thread 0 per block"): the expert of token t is
- * the argmax over e of gate_logits[t, e]; on a tie the lowest index wins (the
+ * Routing. [P1] kernel list (the forward picks one expert per token from the
+ * gate logits) and PERFORMANCE (one thread per block makes that choice): the
+ * expert of token t is the argmax over e of gate_logits[t, e]; on a tie the lowest index wins (the
  * result of a scan from e = 0 that moves only on a strictly greater value, so a
  * NaN at e = 0 selects expert 0 and a NaN elsewhere is never selected).
  * Also writes counts, offsets and the stable permutation perm (the r-th token
@@ -128,8 +128,9 @@ moe_status_t moe_top1_route_noalloc(const float* gate_logits, int64_t B, int64_t
                                     const moe_routing_t* out, void* stream);
 
 /*
- * Forward. [P1] kernel list ("apply its [H, H] linear to fused_ctx") and
- * PERFORMANCE (one output channel = a dot product over the H inputs):
+ * Forward. [P1] kernel list (the chosen expert's [H, H] linear is applied to
+ * the token's context vector) and PERFORMANCE (one output channel = a dot
+ * product over the H inputs):
  *   routed[t, o] = sum_i W[e*, o, i] * x[t, i] + bias[e*, o],  e* = expert_idx[t].
  * `routing` is the result of moe_top1_route on the same tokens (device
  * pointers; only offsets and perm are read). routed is overwritten and must
@@ -149,9 +150,10 @@ moe_status_t moe_top1_fwd(const float* x, const float* W, const float* bias,
 #define MOE_ACC_DB 0x4u
 
 /*
- * Backward (straight-through). [P1] kernel list ("chain-rule grads through the
- * SELECTED expert's W and bias ... Inactive experts get zero contribution") and
- * ARCHITECTURE ("gate logit grad is zero from the expert path"):
+ * Backward (straight-through). [P1] kernel list (gradients flow only through
+ * the selected expert's weights and bias; the other experts receive nothing)
+ * and ARCHITECTURE (the top-1 choice is not differentiable, so the expert path
+ * gives the gate logits no gradient):
  *   d_x[t, i]   = sum_o W[e*, o, i] * d_out[t, o]
  *   dW[e, o, i] = sum_{t : e*(t) = e} d_out[t, o] * x[t, i]
  *   db[e, o]    = sum_{t : e*(t) = e} d_out[t, o]
@@ -169,11 +171,12 @@ moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out,
                           void* stream);
 
 /*
- * Load-balance auxiliary loss and its logit gradient. [P1] kernel list
- * ("softmax of gate_logits + load-balancing auxiliary loss (frac . prob_mean x
- * N_EXPERTS)"), ARCHITECTURE (frac comes from the non-differentiable top-1
- * choice, so only prob_mean carries gradient) and [P2] Wiring (the loss kernel
- * reads lambda from device memory):
+ * Load-balance auxiliary loss and its logit gradient. [P1] kernel list (a
+ * softmax of the gate logits feeds a balance loss built from the usage
+ * fraction, the mean probability and the expert count), ARCHITECTURE (the
+ * usage fraction comes from the non-differentiable top-1 choice, so only the
+ * mean probability carries gradient) and [P2] Wiring (the loss kernel reads
+ * lambda from device memory):
  *   p[t, e]   = softmax_e(gate_logits[t, :])  (shifted by the row max)
  *   frac[e]   = counts[e] / T,   mean_p[e] = (1/T) sum_t p[t, e]
  *   aux_raw   = E * (sum_e counts[e] * mean_p[e]) / T

@@ -134,8 +134,8 @@ void oracle_bwd_dx(const float* W, const float* d_out, const int32_t* expert_idx
 }
 
 /* ------------------------------------------------------------------------- */
-/* Backward, weight and bias gradients. [P1] kernel list: "inactive experts   */
-/* get zero contribution"; only the selected expert receives                  */
+/* Backward, weight and bias gradients. [P1] kernel list: only the selected  */
+/* expert of a token receives gradient from it; the others receive nothing:  */
 /*   dW[e, o, i] = sum_{t : e*(t) = e} d_out[t, o] * x[t, i]                  */
 /*   db[e, o]    = sum_{t : e*(t) = e} d_out[t, o].                           */
 /* Tokens are visited in ascending t. An expert with no tokens gets exactly 0.*/
