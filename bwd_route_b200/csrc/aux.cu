@@ -13,8 +13,9 @@
 //
 // The logit gradient of token t needs only its own softmax row and the global
 // frac, so one streaming pass reads the logits once, writes d_logits and leaves
-// per-block sums of p; a one-block kernel then sums those in a fixed order
-// (mean_p, aux, loss, stats). No atomics: every bit is reproducible.
+// per-block sums of p (warps work on 32-token chunks staged in their own shared
+// buffers); a one-block kernel then sums those in a fixed order (mean_p, aux,
+// loss, stats). No atomics: every bit is reproducible.
 #include <cstdint>
 
 #include "common.cuh"
@@ -23,67 +24,134 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = kAuxTokPerBlk;  // one token per thread
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = 32;                                   // tokens a warp handles at a time
+constexpr int kChunksPerWarp = kAuxTokPerBlk / (kWarps * kChunk);  // 4
 
+// Shared-memory slot of float4 q (experts 4q..4q+3) of token row t when a row
+// holds Q = EMAX / 4 float4s: the XOR swizzle spreads the 8 rows read by one
+// quarter-warp over distinct banks, so row reads and writes are conflict-free.
 template <int EMAX>
-__global__ void __launch_bounds__(kThreads, 1) aux_kernel(const float* __restrict__ logits,
+__device__ __forceinline__ int row_slot(int t, int q) {
+    constexpr int Q = EMAX / 4;
+    if (Q == 1) return t;
+    constexpr int SH = (Q == 2) ? 2 : (Q == 4) ? 1 : 0;
+    return t * Q + (q ^ ((t >> SH) & (Q - 1)));
+}
+
+// One block per 1024 consecutive tokens; warp w handles chunks w, w + 8, w + 16,
+// w + 24 of 32 tokens. The warp stages all four chunks' logits in its own
+// shared buffer (128-bit loads, every load in flight before the first use, no
+// block barrier for the data), lane t computes token t of each chunk reading
+// its row as float4s, and the gradients go back out with 128-bit stores. When
+// E is not a multiple of 4 the rows are moved one float at a time.
+template <int EMAX>
+__global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__ logits,
                                                       const int32_t* __restrict__ counts, int64_t T, int E,
                                                       const float* __restrict__ lambda_eff,
                                                       float* __restrict__ d_logits, float* __restrict__ blk_psum) {
-    extern __shared__ float4 s_tile4[];  // kAuxTokPerBlk * E floats (logits, then gradients)
-    float* s_tile = reinterpret_cast<float*>(s_tile4);
-    __shared__ float s_frac[32];
+    constexpr int Q = EMAX / 4;          // float4s per staged row
+    constexpr int BUF4 = kChunk * Q;     // float4s per chunk buffer
+    extern __shared__ float4 s_dyn4[];   // kWarps x kChunksPerWarp chunk buffers
+    __shared__ float s_frac[EMAX];
     __shared__ float s_part[kWarps][EMAX];
-    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kAuxTokPerBlk;
-    const int64_t ntok = (T - t0 < kAuxTokPerBlk) ? (T - t0) : kAuxTokPerBlk;
-    const int64_t nflt = ntok * E;
-    const float* src = logits + t0 * E;
-    // coalesced 128-bit staging (the block's first float is 16-byte aligned: 1024 * E * 4 bytes per block)
-    const int64_t n4 = nflt / 4;
-    stage_f4<2>(s_tile4, reinterpret_cast<const float4*>(src), static_cast<int>(n4), threadIdx.x, kThreads);
-    for (int64_t i = n4 * 4 + threadIdx.x; i < nflt; i += kThreads) s_tile[i] = __ldg(src + i);
-    if (threadIdx.x < E) s_frac[threadIdx.x] = static_cast<float>(counts[threadIdx.x]) / static_cast<float>(T);
-    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < EMAX)
+        s_frac[threadIdx.x] = threadIdx.x < E ? static_cast<float>(counts[threadIdx.x]) / static_cast<float>(T) : 0.0f;
     const float lam = *lambda_eff;
     const float scale = lam * static_cast<float>(E) / static_cast<float>(T);
+    const bool vec = (E == EMAX);        // rows move as whole float4s
+    float4* wbuf = s_dyn4 + warp * kChunksPerWarp * BUF4;
+    int64_t c0[kChunksPerWarp];
+    int n[kChunksPerWarp];
+#pragma unroll
+    for (int j = 0; j < kChunksPerWarp; ++j) {
+        c0[j] = static_cast<int64_t>(blockIdx.x) * kAuxTokPerBlk + (j * kWarps + warp) * kChunk;
+        n[j] = c0[j] >= T ? 0 : static_cast<int>((T - c0[j] < kChunk) ? (T - c0[j]) : kChunk);
+    }
+#pragma unroll
+    for (int j = 0; j < kChunksPerWarp; ++j) {
+        float4* buf = wbuf + j * BUF4;
+        if (vec) {  // c0 * E * 4 bytes is a multiple of 16
+            const float4* src4 = reinterpret_cast<const float4*>(logits + c0[j] * E);
+            for (int i = lane; i < n[j] * Q; i += 32) buf[row_slot<EMAX>(i / Q, i % Q)] = __ldg(src4 + i);
+        } else {
+            float* b = reinterpret_cast<float*>(buf);
+            for (int i = lane; i < n[j] * E; i += 32) {
+                const int t = i / E, e = i % E;
+                b[row_slot<EMAX>(t, e / 4) * 4 + (e & 3)] = __ldg(logits + c0[j] * E + i);
+            }
+        }
+    }
+    __syncthreads();  // s_frac (the chunk buffers are per warp)
     float psum[EMAX];
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) psum[e] = 0.0f;
-    const int tl = threadIdx.x;  // this thread's token in the block
-    if (tl < ntok) {
-        float* row = s_tile + static_cast<int64_t>(tl) * E;
-        float p[EMAX];
-        float m = row[0];
 #pragma unroll
-        for (int e = 1; e < EMAX; ++e)
-            if (e < E && row[e] > m) m = row[e];
-        float s = 0.0f;
+    for (int j = 0; j < kChunksPerWarp; ++j) {
+        if (lane < n[j]) {
+            float4* buf = wbuf + j * BUF4;
+            float x[EMAX];
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-            if (e < E) {
-                p[e] = expf(row[e] - m);
-                s += p[e];
+            for (int q = 0; q < Q; ++q) {
+                const float4 v = buf[row_slot<EMAX>(lane, q)];
+                x[4 * q] = v.x;
+                x[4 * q + 1] = v.y;
+                x[4 * q + 2] = v.z;
+                x[4 * q + 3] = v.w;
             }
-        }
-        float g = 0.0f;
+            float m = x[0];
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-            if (e < E) {
-                p[e] = p[e] / s;
-                g += s_frac[e] * p[e];
+            for (int e = 1; e < EMAX; ++e)
+                if (e < E && x[e] > m) m = x[e];
+            float sum = 0.0f;
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) {
+                if (e < E) {
+                    x[e] = expf(x[e] - m);
+                    sum += x[e];
+                }
             }
-        }
+            const float rs = __frcp_rn(sum);  // correctly rounded 1 / sum
+            float g = 0.0f;
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-            if (e < E) {
-                psum[e] = p[e];
-                row[e] = scale * (p[e] * (s_frac[e] - g));
+            for (int e = 0; e < EMAX; ++e) {
+                if (e < E) {
+                    x[e] = x[e] * rs;
+                    g += s_frac[e] * x[e];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) {
+                if (e < E) {
+                    psum[e] += x[e];
+                    x[e] = scale * (x[e] * (s_frac[e] - g));
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < Q; ++q)
+                buf[row_slot<EMAX>(lane, q)] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+        }
+    }
+    __syncwarp();
+    if (d_logits) {
+#pragma unroll
+        for (int j = 0; j < kChunksPerWarp; ++j) {
+            const float4* buf = wbuf + j * BUF4;
+            if (vec) {
+                float4* dst4 = reinterpret_cast<float4*>(d_logits + c0[j] * E);
+                for (int i = lane; i < n[j] * Q; i += 32) dst4[i] = buf[row_slot<EMAX>(i / Q, i % Q)];
+            } else {
+                const float* b = reinterpret_cast<const float*>(buf);
+                for (int i = lane; i < n[j] * E; i += 32) {
+                    const int t = i / E, e = i % E;
+                    d_logits[c0[j] * E + i] = b[row_slot<EMAX>(t, e / 4) * 4 + (e & 3)];
+                }
             }
         }
     }
     // fixed-order block sum of p: xor-butterfly inside each warp, then warps in order
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) {
         float v = psum[e];
@@ -97,54 +165,65 @@ __global__ void __launch_bounds__(kThreads, 1) aux_kernel(const float* __restric
         for (int w = 1; w < kWarps; ++w) acc += s_part[w][threadIdx.x];
         blk_psum[static_cast<int64_t>(blockIdx.x) * E + threadIdx.x] = acc;
     }
-    if (d_logits) {
-        float* dst = d_logits + t0 * E;
-        for (int64_t i = threadIdx.x; i < n4; i += kThreads) reinterpret_cast<float4*>(dst)[i] = s_tile4[i];
-        for (int64_t i = n4 * 4 + threadIdx.x; i < nflt; i += kThreads) dst[i] = s_tile[i];
-    }
 }
 
-// One block: mean_p from the per-block sums (double, fixed order: warp e sums
-// expert e with lane-strided partials and an xor butterfly), then aux, loss and
-// stats.
+// One block: mean_p from the per-block sums (double, fixed order), then aux,
+// loss, stats. Expert e's partial sums are split over the warps of group e
+// (32 / E warps; block b of the expert goes to thread b mod the group's
+// threads), summed per thread in block order, by an xor butterfly per warp and
+// across the group's warps in order.
 __global__ void __launch_bounds__(1024) aux_finalize_kernel(const float* __restrict__ blk_psum, int64_t nblk,
                                                            const int32_t* __restrict__ counts, int64_t T, int E,
                                                            const float* __restrict__ lambda_eff,
                                                            float* __restrict__ loss_out, float* __restrict__ mean_p,
                                                            float* __restrict__ stats) {
+    __shared__ double s_wsum[32];
     __shared__ float s_mean[32];
     __shared__ double s_hf[32], s_hm[32];
+    __shared__ int s_cnt[32];
+    __shared__ float s_lam;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp < E) {
-        double acc = 0.0;
-        for (int64_t b0 = 0; b0 < nblk; b0 += 8 * 32) {
+    const int wpe = 32 / E;                 // warps per expert
+    const int e = warp / wpe;               // expert of this warp (e >= E: idle)
+    const int g = (warp % wpe) * 32 + lane; // thread index inside the expert's group
+    const int G = wpe * 32;
+    if (threadIdx.x == 0) s_lam = *lambda_eff;
+    if (threadIdx.x < E) s_cnt[threadIdx.x] = counts[threadIdx.x];
+    double acc = 0.0;
+    if (e < E) {
+        for (int64_t b0 = g; b0 < nblk; b0 += 8 * static_cast<int64_t>(G)) {
             float v[8];  // eight independent loads, then added in block order
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t b = b0 + u * 32 + lane;
-                v[u] = (b < nblk) ? blk_psum[b * E + warp] : 0.0f;
+                const int64_t b = b0 + static_cast<int64_t>(u) * G;
+                v[u] = (b < nblk) ? blk_psum[b * E + e] : 0.0f;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                if (b0 + u * 32 + lane < nblk) acc += static_cast<double>(v[u]);
+                if (b0 + static_cast<int64_t>(u) * G < nblk) acc += static_cast<double>(v[u]);
         }
+    }
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) {
-            const float m = T > 0 ? static_cast<float>(acc / static_cast<double>(T)) : 0.0f;
-            s_mean[warp] = m;
-            // entropy terms of expert `warp` (0 ln 0 = 0)
-            const double f = T > 0 ? static_cast<double>(counts[warp]) / static_cast<double>(T) : 0.0;
-            s_hf[warp] = f > 0.0 ? f * log(f) : 0.0;
-            s_hm[warp] = m > 0.0f ? static_cast<double>(m) * log(static_cast<double>(m)) : 0.0;
-        }
+    for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) s_wsum[warp] = acc;
+    __syncthreads();
+    if (threadIdx.x < E) {
+        const int x = threadIdx.x;
+        double tot = 0.0;
+        for (int w = 0; w < wpe; ++w) tot += s_wsum[x * wpe + w];
+        const float m = T > 0 ? static_cast<float>(tot / static_cast<double>(T)) : 0.0f;
+        s_mean[x] = m;
+        // entropy terms of expert x (0 ln 0 = 0)
+        const double f = T > 0 ? static_cast<double>(s_cnt[x]) / static_cast<double>(T) : 0.0;
+        s_hf[x] = f > 0.0 ? f * log(f) : 0.0;
+        s_hm[x] = m > 0.0f ? static_cast<double>(m) * log(static_cast<double>(m)) : 0.0;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        const float lam = *lambda_eff;
+        const float lam = s_lam;
         double acc = 0.0, hf = 0.0, hm = 0.0;
         for (int e = 0; e < E; ++e) {
-            acc += static_cast<double>(counts[e]) * static_cast<double>(s_mean[e]);
+            acc += static_cast<double>(s_cnt[e]) * static_cast<double>(s_mean[e]);
             hf -= s_hf[e];
             hm -= s_hm[e];
         }
@@ -154,9 +233,9 @@ __global__ void __launch_bounds__(1024) aux_finalize_kernel(const float* __restr
         for (int e = 0; e < E; ++e) mean_p[e] = s_mean[e];
         if (stats) {
             for (int e = 0; e < E; ++e) {
-                stats[e] = T > 0 ? static_cast<float>(counts[e]) / static_cast<float>(T) : 0.0f;
+                stats[e] = T > 0 ? static_cast<float>(s_cnt[e]) / static_cast<float>(T) : 0.0f;
                 stats[E + e] = s_mean[e];
-                stats[2 * E + e] = static_cast<float>(counts[e]);
+                stats[2 * E + e] = static_cast<float>(s_cnt[e]);
             }
             stats[3 * E + 0] = aux_raw;
             stats[3 * E + 1] = lam;
@@ -180,7 +259,7 @@ cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, in
                        cudaStream_t s) {
     const int64_t nblk = T > 0 ? (T + kAuxTokPerBlk - 1) / kAuxTokPerBlk : 0;
     if (T > 0) {
-        const size_t smem = sizeof(float) * kAuxTokPerBlk * E;
+        const size_t smem = sizeof(float) * kWarps * kChunksPerWarp * kChunk * (E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32);
         if (E <= 4)
             aux_kernel<4><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum);
         else if (E <= 8)
@@ -203,11 +282,12 @@ cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float la
 }
 
 cudaError_t aux_set_smem_limits() {
+    // 8 warps x 4 chunks x 32 tokens x 32 experts x 4 bytes = 128 KiB for the widest instance
     cudaError_t e = cudaFuncSetAttribute(aux_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(float) * kAuxTokPerBlk * 16));
+                                         static_cast<int>(sizeof(float) * kWarps * kChunksPerWarp * kChunk * 16));
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(aux_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(float) * kAuxTokPerBlk * 32));
+                                static_cast<int>(sizeof(float) * kWarps * kChunksPerWarp * kChunk * 32));
 }
 
 }  // namespace moe

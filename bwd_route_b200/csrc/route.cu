@@ -5,14 +5,16 @@
 // Transformer"), kernel list and PERFORMANCE: the expert of a token is the
 // argmax of its gate logits, picked by one thread scanning e = 0, 1, ... and
 // moving only on a strictly greater value. Here a group of lanes shares one
-// token and reduces (value, index) pairs with a combiner that yields exactly
-// that scan's result: NaN entries are never chosen, equal values keep the lower
-// index, and a NaN at e = 0 pins the result to 0.
+// token: a shuffle butterfly finds the maximum over the non-NaN entries and a
+// ballot picks the lowest expert index holding it, which is exactly that
+// scan's result (equal values, -0 / +0 included, keep the lower index; NaN
+// entries are never chosen; a NaN at e = 0 pins the result to 0).
 //
 // Three launches, all integer-exact and deterministic:
-//   1. route_count   : the block's 1024 x E logits are staged in shared memory
-//                      with 128-bit loads; lane groups reduce (value, index)
-//                      pairs with warp shuffles; per-block expert counts come
+//   1. route_count   : each warp loads its 128 tokens' logits (a lane group of
+//                      LPT lanes per token, 16 steps in flight), takes the
+//                      group maximum with xor shuffles and the lowest index
+//                      holding it with a ballot; per-block expert counts come
 //                      from warp ballots (no atomics).
 //   2. route_scan    : one block, one warp per expert: counts, offsets and every
 //                      block's base position inside each expert's segment.
@@ -26,74 +28,67 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;                 // route_scatter
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kTokPerWarp = kRouteTokPerBlk / kWarps;  // 128
-constexpr int kCountThreads = 1024;           // route_count: one block of 32 warps per 1024 tokens
-constexpr int kCountWarps = kCountThreads / 32;
-
-__device__ __forceinline__ void combine(float& v, int& e, bool& ok, float ov, int oe, bool ook) {
-    const bool take = ook && (!ok || ov > v || (ov == v && oe < e));
-    if (take) {
-        v = ov;
-        e = oe;
-        ok = true;
-    }
-}
 
 template <int LPT>  // lanes per token: a power of two >= E
-__global__ void __launch_bounds__(kCountThreads, 1) route_count_kernel(const float* __restrict__ logits, int64_t T, int E,
+__global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __restrict__ logits, int64_t T, int E,
                                                               int32_t* __restrict__ expert_idx,
                                                               int32_t* __restrict__ blk_counts) {
-    extern __shared__ float4 s_lg4[];  // the block's logits, kRouteTokPerBlk * E floats
-    const float* s_lg = reinterpret_cast<const float*>(s_lg4);
     __shared__ int s_idx[kRouteTokPerBlk];
-    __shared__ int s_wcnt[kCountWarps][32];
+    __shared__ int s_wcnt[kWarps][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokPerBlk;
     const int ntok = static_cast<int>((T - t0 < kRouteTokPerBlk) ? (T - t0) : kRouteTokPerBlk);
-    {
-        // coalesced 128-bit staging; the block's first float is 16-byte aligned (1024 * E * 4 bytes per block)
-        const int nflt = ntok * E, n4 = nflt / 4;
-        stage_f4<2>(s_lg4, reinterpret_cast<const float4*>(logits + t0 * E), n4, threadIdx.x, kCountThreads);
-        float* s_w = reinterpret_cast<float*>(s_lg4);
-        for (int i = n4 * 4 + threadIdx.x; i < nflt; i += kCountThreads) s_w[i] = __ldg(logits + t0 * E + i);
-    }
-    __syncthreads();
-    constexpr int TPW = 32 / LPT;  // tokens per warp per step
+    constexpr int TPW = 32 / LPT;              // tokens per warp per step
+    constexpr int STEPS = kTokPerWarp / TPW;   // steps for the warp's 128 consecutive tokens
+    constexpr int BATCH = STEPS < 16 ? STEPS : 16;
     const int sub = lane % LPT;
-    for (int base = warp * TPW; base < kRouteTokPerBlk; base += kCountWarps * TPW) {
-        const int tl = base + lane / LPT;
-        const bool in = (tl < ntok) && (sub < E);
-        const float raw = in ? s_lg[tl * E + sub] : 0.0f;
-        float v = raw;
-        int e = sub;
-        bool ok = in && !isnan(raw);
-        const bool nan0 = __shfl_sync(0xffffffffu, in && isnan(raw), lane & ~(LPT - 1));
+    const int wt0 = warp * kTokPerWarp;
+    const int g0 = (lane / LPT) * LPT;            // first lane of this token's group
+    const uint32_t gmask = (LPT == 32 ? 0xffffffffu : ((1u << LPT) - 1u)) << g0;
+    for (int b0 = 0; b0 < STEPS; b0 += BATCH) {
+        float v[BATCH];
 #pragma unroll
-        for (int off = LPT / 2; off >= 1; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, v, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, e, off);
-            const bool ook = __shfl_xor_sync(0xffffffffu, ok, off);
-            combine(v, e, ok, ov, oe, ook);
+        for (int j = 0; j < BATCH; ++j) {  // all loads of the batch first
+            const int tl = wt0 + (b0 + j) * TPW + lane / LPT;
+            v[j] = (tl < ntok && sub < E) ? __ldg(logits + (t0 + tl) * E + sub) : __int_as_float(0x7fc00000);
         }
-        if (sub == 0) s_idx[tl] = (tl < ntok) ? (nan0 ? 0 : e) : -1;
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {
+            const int tl = wt0 + (b0 + j) * TPW + lane / LPT;
+            // the group's maximum over its valid entries (fmaxf skips NaN; padding lanes hold NaN)
+            float m = v[j];
+#pragma unroll
+            for (int off = LPT / 2; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            // the lowest expert index holding that maximum (-0 == +0 tie); a NaN at
+            // e = 0 wins outright, as in a scan that never moves off its NaN start
+            const bool nan0 = (sub == 0) && isnan(v[j]) && (tl < ntok);
+            const uint32_t hit = __ballot_sync(0xffffffffu, v[j] == m) & gmask;
+            const uint32_t n0 = __ballot_sync(0xffffffffu, nan0) & gmask;
+            const int k = (n0 || !hit) ? 0 : __ffs(hit >> g0) - 1;
+            if (sub == 0) s_idx[tl] = (tl < ntok) ? k : -1;
+        }
     }
     __syncthreads();
-    // write expert_idx coalesced; per-warp counts over the warp's 32 consecutive
-    // tokens; lane e keeps expert e
-    const int k = s_idx[threadIdx.x];
-    if (threadIdx.x < ntok) expert_idx[t0 + threadIdx.x] = k;
+    // expert_idx written coalesced; per-warp counts over its 128 tokens, lane e keeps expert e
     int cnt = 0;
-    for (int e = 0; e < E; ++e) {
-        const int c = __popc(__ballot_sync(0xffffffffu, k == e));
-        if (lane == e) cnt = c;
+#pragma unroll
+    for (int it = 0; it < kTokPerWarp / 32; ++it) {
+        const int tl = wt0 + it * 32 + lane;
+        const int k = s_idx[tl];
+        if (tl < ntok) expert_idx[t0 + tl] = k;
+        for (int e = 0; e < E; ++e) {
+            const int c = __popc(__ballot_sync(0xffffffffu, k == e));
+            if (lane == e) cnt += c;
+        }
     }
     s_wcnt[warp][lane] = cnt;
     __syncthreads();
     if (threadIdx.x < E) {
         int total = 0;
-        for (int w = 0; w < kCountWarps; ++w) total += s_wcnt[w][threadIdx.x];
+        for (int w = 0; w < kWarps; ++w) total += s_wcnt[w][threadIdx.x];
         blk_counts[static_cast<int64_t>(blockIdx.x) * E + threadIdx.x] = total;
     }
 }
@@ -210,26 +205,21 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
                          int32_t* offsets, int32_t* perm, int32_t* blk_counts, int32_t* blk_base,
                          cudaStream_t s) {
     const int64_t nblk = (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk;
-    const size_t smem = sizeof(float) * kRouteTokPerBlk * E;
     if (E <= 4)
-        route_count_kernel<4><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<4><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
     else if (E <= 8)
-        route_count_kernel<8><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<8><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
     else if (E <= 16)
-        route_count_kernel<16><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<16><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
     else
-        route_count_kernel<32><<<(unsigned)nblk, kCountThreads, smem, s>>>(logits, T, E, expert_idx, blk_counts);
+        route_count_kernel<32><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
     route_scan_kernel<<<1, 1024, 0, s>>>(blk_counts, nblk, E, counts, offsets, blk_base);
     route_scatter_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(expert_idx, T, E, blk_base, perm);
     return cudaGetLastError();
 }
 
-cudaError_t route_set_smem_limits() {
-    cudaError_t e = cudaFuncSetAttribute(route_count_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(float) * kRouteTokPerBlk * 16));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(route_count_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(float) * kRouteTokPerBlk * 32));
-}
+// The routing kernels use static shared memory only; kept so that callers that
+// prepare a device once have a single place to do it.
+cudaError_t route_set_smem_limits() { return cudaSuccess; }
 
 }  // namespace moe
