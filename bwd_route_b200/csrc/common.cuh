@@ -105,6 +105,13 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
+// The same with a 256-byte L2 prefetch size: a miss fills the aligned 256-byte
+// block around the address, so the row segment next to it is in L2 when it is
+// fetched a stage later.
+__device__ __forceinline__ void cp_async_16_l2_256(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
 // The mbarrier receives one arrival once every cp.async issued so far by this
 // thread has landed (the arrival counts against the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {

@@ -194,7 +194,7 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                     const int r = it * 16 + prow;
                     const int t = tok[it];
                     const float* gsrc = src + static_cast<int64_t>(t < 0 ? 0 : t) * H + kc * 32 + pg * 4;
-                    cp_async_16(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), gsrc, t < 0 ? 0u : 16u);
+                    cp_async_16_l2_256(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), gsrc, t < 0 ? 0u : 16u);
                 }
                 cp_async_arrive_noinc(&ctl->afull[sa]);
                 if (++sa == C::A_STAGES) {
