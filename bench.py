@@ -114,6 +114,24 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The maximum of a per-rank time over all ranks (one all-reduce; a no-op for
+    a single process). Used for every multi-GPU time: the job is as slow as its
+    slowest replica."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job routed tokens/s: every replica routes its own batch per step."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def cpu_oracle_tokens_per_s(inp, n_tokens: int):
     """The CPU oracle, as it stands, on the first n_tokens tokens of the workload."""
     import oracle
@@ -242,11 +260,7 @@ def main():
             step(per_call[k])
         end.record(stream)
         barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dev)
     ms_per_step = ms / args.steps
     names = ["route", "fwd", "d_x", "wgrad", "aux+lambda"]
     call_ms = {n: sum(per_call[k][i].elapsed_time(per_call[k][i + 1]) for k in range(args.steps)) / args.steps
@@ -270,11 +284,7 @@ def main():
         h_loss.copy_(gate.loss, non_blocking=True)
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
@@ -282,7 +292,7 @@ def main():
         hbm = float(peaks["hbm_gbs"])
         tf32_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * TF32_OVER_BF16
         t_roof = max(step_bytes / (hbm * 1e9), step_flops / (tf32_sus * 1e12))
-        value = world * T / (ms_per_step * 1e-3)
+        value = job_throughput(world, T, ms_per_step)
         dominant = max(["fwd", "d_x", "wgrad"], key=lambda n: call_ms[n])
         achieved = kbytes[dominant] / (call_ms[dominant] * 1e-3) / 1e9
         line = {
@@ -299,7 +309,7 @@ def main():
                               "peaks": {"hbm_gbs": hbm, "tf32_tflops": tf32_sus,
                                         "source": f"{peak_kind}; tf32 = bf16_tflops_sustained x 1.1/2.25"}},
             "per_call_ms": call_ms,
-            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
+            "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
                     "h2d_bytes_per_step": T * (E + 2 * H) * 4, "d2h_bytes_per_step": 8},
             "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode),
             "clocks": clocks.summary(),

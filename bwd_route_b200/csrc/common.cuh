@@ -53,22 +53,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Waits for the phase with the given parity to complete. Returns false if the
-// wait ran past kWaitLimitCycles or another role of the CTA already gave up
+// wait ran past limit_cycles or another role of the CTA already gave up
 // (*abort != 0); in the first case it sets *abort and the device flag bit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* dev_flags) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint32_t* dev_flags, long long limit_cycles) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit_cycles) {
             *abort = 1;
             if (dev_flags) atomicOr(dev_flags, MOE_FLAG_WAIT_TIMEOUT);
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t* dev_flags) {
+    return mbar_wait_limit(bar, parity, abort, dev_flags, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------------------- TMA

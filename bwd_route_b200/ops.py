@@ -28,7 +28,7 @@ _STATUS = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED_SHAPE", "MOE_ER
 EXPORTED = [
     "moe_top1_workspace_bytes", "moe_top1_workspace_init", "moe_top1_route", "moe_top1_fwd",
     "moe_top1_bwd", "moe_aux_loss_fwd_bwd", "moe_lambda_eff_update", "moe_top1_device_flags",
-    "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc",
+    "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc", "moe_top1_selftest_wait_timeout",
 ]
 MOE_NOALLOC_MAX_TOKENS = 2097152
 
@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.argtypes = [I32]
         L.moe_top1_abi_version.restype = I32
         L.moe_top1_abi_version.argtypes = []
+        L.moe_top1_selftest_wait_timeout.restype = I32
+        L.moe_top1_selftest_wait_timeout.argtypes = [P, SZ, I64, P]
         L.moe_top1_route_noalloc.restype = I32
         L.moe_top1_route_noalloc.argtypes = [P, I64, I64, I32, ctypes.POINTER(RoutingC), P]
         _lib = L
@@ -194,6 +196,12 @@ def moe_lambda_eff_update(ent_ema, lambda_floor: float, lambda_max_extra: float,
     _check("moe_lambda_eff_update",
            lib().moe_lambda_eff_update(_ptr(ent_ema, f), lambda_floor, lambda_max_extra, ent_target,
                                        _ptr(lambda_eff, f), _stream(stream)))
+
+
+def moe_top1_selftest_wait_timeout(ws: torch.Tensor, limit_cycles: int, stream=None):
+    """Runs one bounded wait that must time out (diagnostic of the failure path)."""
+    _check("moe_top1_selftest_wait_timeout",
+           lib().moe_top1_selftest_wait_timeout(_ptr(ws), ws.numel(), limit_cycles, _stream(stream)))
 
 
 def moe_top1_device_flags(ws: torch.Tensor, stream=None) -> int:

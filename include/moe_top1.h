@@ -205,6 +205,15 @@ moe_status_t moe_lambda_eff_update(const float* ent_ema, float lambda_floor,
                                    float lambda_max_extra, float ent_target, float* lambda_eff,
                                    void* stream);
 
+/* Diagnostic (no counterpart on the pages): launches one thread that waits on
+ * a barrier nothing arrives on, through the same bounded wait as the tensor-core
+ * kernels, with a limit of limit_cycles SM clock cycles (1 .. 4e9). The wait
+ * gives up, sets MOE_FLAG_WAIT_TIMEOUT in the workspace flag word and the
+ * kernel returns; no fault, the context stays usable. Lets a test check the
+ * failure path end to end: afterwards moe_top1_device_flags reports the bit. */
+moe_status_t moe_top1_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
+                                            void* stream);
+
 /* Synchronises `stream`, returns the workspace flag word in *flags_out and
  * clears it. MOE_ERR_DEVICE_CHECK if any bit was set. (Debug / tests.) */
 moe_status_t moe_top1_device_flags(void* workspace, size_t workspace_bytes, void* stream,

@@ -35,24 +35,28 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declares the C signatures on a loaded copy of the oracle library."""
+    P = ctypes.c_void_p
+    i64, i32 = ctypes.c_int64, ctypes.c_int32
+    lib.oracle_tf32_round.restype = ctypes.c_float
+    lib.oracle_tf32_round.argtypes = [ctypes.c_float, i32]
+    lib.oracle_route.argtypes = [P, i64, i32, P, P, P, P]
+    lib.oracle_fwd.argtypes = [P, P, P, P, i64, i32, i32, i32, P]
+    lib.oracle_bwd_dx.argtypes = [P, P, P, i64, i32, i32, i32, P]
+    lib.oracle_bwd_dw.argtypes = [P, P, P, i64, i32, i32, i32, P, P, P, P]
+    lib.oracle_bwd_db.argtypes = [P, P, i64, i32, i32, P, P]
+    lib.oracle_bwd_dw_entries.argtypes = [P, P, P, i64, i32, i32, i64, P, P, P, P, P]
+    lib.oracle_aux.argtypes = [P, P, i64, i32, ctypes.c_float, P, P, P, P, P]
+    lib.oracle_lambda_eff.restype = ctypes.c_double
+    lib.oracle_lambda_eff.argtypes = [ctypes.c_double] * 4
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        i64, i32 = ctypes.c_int64, ctypes.c_int32
-        lib.oracle_tf32_round.restype = ctypes.c_float
-        lib.oracle_tf32_round.argtypes = [ctypes.c_float, i32]
-        lib.oracle_route.argtypes = [P, i64, i32, P, P, P, P]
-        lib.oracle_fwd.argtypes = [P, P, P, P, i64, i32, i32, i32, P]
-        lib.oracle_bwd_dx.argtypes = [P, P, P, i64, i32, i32, i32, P]
-        lib.oracle_bwd_dw.argtypes = [P, P, P, i64, i32, i32, i32, P, P, P, P]
-        lib.oracle_bwd_db.argtypes = [P, P, i64, i32, i32, P, P]
-        lib.oracle_bwd_dw_entries.argtypes = [P, P, P, i64, i32, i32, i64, P, P, P, P, P]
-        lib.oracle_aux.argtypes = [P, P, i64, i32, ctypes.c_float, P, P, P, P, P]
-        lib.oracle_lambda_eff.restype = ctypes.c_double
-        lib.oracle_lambda_eff.argtypes = [ctypes.c_double] * 4
-        _lib = lib
+        _lib = configure(ctypes.CDLL(build()))
     return _lib
 
 
