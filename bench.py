@@ -54,12 +54,35 @@ def algorithmic(spec):
     per_kernel_bytes = {
         # x read, routed written, perm read; W and bias
         "fwd": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
-        # d_out read, d_x written, perm read; W^T
+        # d_out read, d_x written, perm read; W
         "d_x": T * (8 * H + 4) + E * H * H * 4,
         # x and d_out read, perm read; dW and db written
         "wgrad": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
     }
     return step_bytes, step_flops, per_kernel_bytes
+
+
+TRAFFIC_RECORD = os.path.join(HERE, "profiles", "launch_list_large_b65536_e8_h256.md")
+
+
+def recorded_traffic(call: str, workload: str, math_name: str):
+    """DRAM bytes (read + write) of one launch of `call` from the committed ncu
+    launch list, or None when there is no record for this workload and math
+    mode, or when the kernel sources changed since the counters were taken."""
+    import hashlib
+    try:
+        text = open(TRAFFIC_RECORD).read()
+        rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
+        h = hashlib.sha1()
+        for f in rec["source_files"]:
+            with open(os.path.join(HERE, f), "rb") as fh:
+                h.update(fh.read())
+    except (OSError, IndexError, KeyError, ValueError):
+        return None
+    if rec.get("workload") != workload or rec.get("math") != math_name or h.hexdigest() != rec.get("source_sha1"):
+        return None
+    v = rec.get("traffic_bytes_per_call", {}).get(call)
+    return int(v) if v is not None else None
 
 
 class ClockSampler:
@@ -303,7 +326,8 @@ def main():
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (x, d_out, routed, d_x: 4 x %.2f GB), no flush" % (T * H * 4 / 1e9)},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": None, "peak_source": f"{peak_kind} hbm_gbs"},
+                         "frac": achieved / hbm, "traffic": recorded_traffic(dominant, spec.name, args.math),
+                         "algorithmic_bytes": kbytes[dominant], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "flops": step_flops, "t_roofline_ms": t_roof * 1e3,
                               "frac": t_roof * 1e3 / ms_per_step,
                               "peaks": {"hbm_gbs": hbm, "tf32_tflops": tf32_sus,

@@ -235,7 +235,7 @@ moe_status_t moe_top1_fwd(const float* x, const float* W, const float* bias, con
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (math == MOE_MATH_TF32)
-        return cuda_status(launch_grouped_tf32(x, W, bias, routing->offsets, routing->perm, T, E, H, 0, routed,
+        return cuda_status(launch_grouped_tf32(x, W, bias, routing->offsets, routing->perm, T, E, H, 0, 0, routed,
                                                static_cast<uint32_t*>(workspace), dev->num_sms, s));
     return cuda_status(launch_grouped_ffma(x, W, bias, routing->offsets, routing->perm, T, E, H, 1, 0, routed, s));
 }
@@ -269,7 +269,7 @@ moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out, co
                           {workspace, workspace ? workspace_bytes : 0}};
     if (any_alias(outs, 3, ins, 6)) return MOE_ERR_ALIAS;
     const WsLayout L = ws_layout(T, E, H);
-    const bool need_ws = (dW || db) || (d_x && math == MOE_MATH_TF32);
+    const bool need_ws = (dW || db) || (d_x && math == MOE_MATH_TF32);  // TF32 d_x: the flag word
     if (need_ws) {
         if (!workspace) return MOE_ERR_WORKSPACE;
         if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
@@ -292,11 +292,8 @@ moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out, co
     uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
     if (d_x) {
         if (math == MOE_MATH_TF32) {
-            float* wt = reinterpret_cast<float*>(ws + L.w_t);
-            e = launch_transpose_w(W, E, H, wt, s);
-            if (e == cudaSuccess)
-                e = launch_grouped_tf32(d_out, wt, nullptr, routing->offsets, routing->perm, T, E, H, acc_dx, d_x,
-                                        flags, dev->num_sms, s);
+            e = launch_grouped_tf32(d_out, W, nullptr, routing->offsets, routing->perm, T, E, H, 1, acc_dx, d_x,
+                                    flags, dev->num_sms, s);
         } else {
             e = launch_grouped_ffma(d_out, W, nullptr, routing->offsets, routing->perm, T, E, H, 0, acc_dx, d_x, s);
         }

@@ -1,6 +1,5 @@
 // gemm_ffma.cu -- FP32 fused-multiply-add variants of the expert contractions,
-// the fixed-order reduction of the weight-gradient partial sums, and the
-// expert-weight transpose.
+// and the fixed-order reduction of the weight-gradient partial sums.
 //
 // foxhunt commit 11b96dac6a ("Top-1 Mixture-of-Experts gate per Switch
 // Transformer"): forward routed[t,o] = sum_i W[e*,o,i] x[t,i] + b[e*,o]
@@ -323,16 +322,6 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
     }
 }
 
-// ---------------------------------------------------------------- transpose
-__global__ void transpose_w_kernel(const float* __restrict__ W, int H, float* __restrict__ Wt) {
-    __shared__ float tile[32][33];
-    const int64_t base = static_cast<int64_t>(blockIdx.z) * H * H;
-    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-    for (int r = threadIdx.y; r < 32; r += 8) tile[r][threadIdx.x] = W[base + static_cast<int64_t>(r0 + r) * H + c0 + threadIdx.x];
-    __syncthreads();
-    for (int r = threadIdx.y; r < 32; r += 8) Wt[base + static_cast<int64_t>(c0 + r) * H + r0 + threadIdx.x] = tile[threadIdx.x][r];
-}
-
 }  // namespace
 
 cudaError_t launch_grouped_ffma(const float* src, const float* Wsrc, const float* bias, const int32_t* offsets,
@@ -359,12 +348,6 @@ cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const i
     const int nb_w = static_cast<int>((HH / 4 + 255) / 256);
     dim3 grid(nb_w + 1, E);
     wgrad_reduce_kernel<<<grid, 256, 0, s>>>(part, part_db, offsets, T, E, H, P, dW, db, acc_dw, acc_db);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_transpose_w(const float* W, int E, int H, float* Wt, cudaStream_t s) {
-    dim3 grid(H / 32, H / 32, E), block(32, 8);
-    transpose_w_kernel<<<grid, block, 0, s>>>(W, H, Wt);
     return cudaGetLastError();
 }
 

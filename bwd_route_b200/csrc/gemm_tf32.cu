@@ -112,7 +112,11 @@ __device__ __forceinline__ int find_expert(const int* tstart, int E, int tile) {
     return e;
 }
 
-template <int H>
+// B_MN = false: the weight operand is K-major in memory (B_e[n][k] = W[e][n][k],
+// the forward). B_MN = true: it is read MN-major straight from W (B_e[n][k] =
+// W[e][k][n], the input gradient), in 32-row x 128-byte boxes with the 32-byte
+// granule swizzle that tcgen05 requires for an MN-major TF32 operand.
+template <int H, bool B_MN>
 __global__ void __launch_bounds__(kThreadsGrouped, 1)
 grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUtensorMap tm_b,
                     const float* __restrict__ bias, const int32_t* __restrict__ offsets,
@@ -216,7 +220,15 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                 for (int kc = 0; kc < C::KCH; ++kc) {
                     if (!(ok = mbar_wait(&ctl->bempty[sb], pb ^ 1, abort, dev_flags))) break;
                     mbar_arrive_expect_tx(&ctl->bfull[sb], C::B_BYTES);
-                    tma_load_2d(bring + sb * C::B_BYTES, &tm_b, kc * 32, e * H, &ctl->bfull[sb]);
+                    if (B_MN) {
+                        // k-chunk = rows kc*32 .. +31 of W[e]; one box per 32 output columns
+#pragma unroll
+                        for (int g = 0; g < H / 32; ++g)
+                            tma_load_2d(bring + sb * C::B_BYTES + g * 32 * 128, &tm_b, g * 32, e * H + kc * 32,
+                                        &ctl->bfull[sb]);
+                    } else {
+                        tma_load_2d(bring + sb * C::B_BYTES, &tm_b, kc * 32, e * H, &ctl->bfull[sb]);
+                    }
                     if (++sb == C::B_STAGES) {
                         sb = 0;
                         pb ^= 1;
@@ -228,7 +240,7 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
     } else if (warp == kGMmaWarp) {
         // ---------------- MMA issuer (one thread)
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_tf32(128, H, 0, 0);
+            constexpr uint32_t idesc = idesc_tf32(128, H, 0, B_MN ? 1 : 0);
             int sa = 0, sb = 0;
             uint32_t pa = 0, pb = 0;
             int acc = 0;
@@ -246,9 +258,11 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                     const uint32_t a_addr = smem_u32(aring + sa * C::A_BYTES);
                     const uint32_t b_addr = smem_u32(bring + sb * C::B_BYTES);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_tf32(d, sw128_desc(a_addr + ks * 32, 16, 1024), sw128_desc(b_addr + ks * 32, 16, 1024),
-                                 idesc, (kc | ks) != 0 ? 1u : 0u);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t bdesc = B_MN ? sw128_32b_mn_desc(b_addr + ks * 1024, 32 * 128, 512)
+                                                    : sw128_desc(b_addr + ks * 32, 16, 1024);
+                        mma_tf32(d, sw128_desc(a_addr + ks * 32, 16, 1024), bdesc, idesc, (kc | ks) != 0 ? 1u : 0u);
+                    }
                     mma_commit(&ctl->aempty[sa]);
                     mma_commit(&ctl->bempty[sb]);
                     if (++sa == C::A_STAGES) {
@@ -566,26 +580,35 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 }  // namespace
 
-cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float* bias, const int32_t* offsets,
-                                const int32_t* perm, int64_t T, int E, int H, int accumulate, float* out,
-                                uint32_t* dev_flags, int num_sms, cudaStream_t s) {
+template <int H, bool B_MN>
+cudaError_t launch_grouped_tf32_t(const float* src, const CUtensorMap& tm_b, const float* bias,
+                                  const int32_t* offsets, const int32_t* perm, int E, int accumulate, float* out,
+                                  uint32_t* dev_flags, int grid, cudaStream_t s) {
+    const cudaError_t err = set_smem(grouped_tf32_kernel<H, B_MN>, GCfg<H>::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    grouped_tf32_kernel<H, B_MN><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
+                                                                                  accumulate, out, dev_flags);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_tf32(const float* src, const float* W, const float* bias, const int32_t* offsets,
+                                const int32_t* perm, int64_t T, int E, int H, int w_transposed, int accumulate,
+                                float* out, uint32_t* dev_flags, int num_sms, cudaStream_t s) {
     CUtensorMap tm_b;
-    if (!make_map_2d(&tm_b, Bsrc, static_cast<uint64_t>(E) * H, H, 32, H)) return cudaErrorInvalidValue;
+    const bool ok = w_transposed ? make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, 32, true)
+                                 : make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, H);
+    if (!ok) return cudaErrorInvalidValue;
     const int64_t tiles = (T + 127) / 128 + E;
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    cudaError_t err;
-    if (H == 256) {
-        err = set_smem(grouped_tf32_kernel<256>, GCfg<256>::SMEM_BYTES);
-        if (err != cudaSuccess) return err;
-        grouped_tf32_kernel<256><<<grid, kThreadsGrouped, GCfg<256>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
-                                                                               accumulate, out, dev_flags);
-    } else {
-        err = set_smem(grouped_tf32_kernel<128>, GCfg<128>::SMEM_BYTES);
-        if (err != cudaSuccess) return err;
-        grouped_tf32_kernel<128><<<grid, kThreadsGrouped, GCfg<128>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
-                                                                               accumulate, out, dev_flags);
-    }
-    return cudaGetLastError();
+    if (H == 256)
+        return w_transposed ? launch_grouped_tf32_t<256, true>(src, tm_b, bias, offsets, perm, E, accumulate, out,
+                                                               dev_flags, grid, s)
+                            : launch_grouped_tf32_t<256, false>(src, tm_b, bias, offsets, perm, E, accumulate, out,
+                                                                dev_flags, grid, s);
+    return w_transposed ? launch_grouped_tf32_t<128, true>(src, tm_b, bias, offsets, perm, E, accumulate, out, dev_flags,
+                                                           grid, s)
+                        : launch_grouped_tf32_t<128, false>(src, tm_b, bias, offsets, perm, E, accumulate, out,
+                                                            dev_flags, grid, s);
 }
 
 cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,

@@ -33,7 +33,6 @@ struct WsLayout {
     size_t route_counts = 0; // int32 [nblk_route][E]
     size_t route_base = 0;   // int32 [nblk_route][E]
     size_t aux_psum = 0;     // float [nblk_aux][E]
-    size_t w_t = 0;          // float [E][H][H]  transposed expert weights (TF32 d_x)
     size_t wg_part = 0;      // float [P + E][H][H] dW partial sums
     size_t wg_part_db = 0;   // float [P + E][H]    db partial sums
     size_t route_end = 0;    // bytes the routing / aux calls need
@@ -58,8 +57,6 @@ inline WsLayout ws_layout(int64_t T, int E, int H) {
     off = align_up(off + sizeof(float) * na * E, 256);
     L.route_end = off;
     if (H > 0) {
-        L.w_t = off;
-        off = align_up(off + sizeof(float) * static_cast<size_t>(E) * H * H, 256);
         L.wg_part = off;
         off = align_up(off + sizeof(float) * static_cast<size_t>(P + E) * H * H, 256);
         L.wg_part_db = off;
@@ -89,13 +86,12 @@ cudaError_t launch_grouped_ffma(const float* src, const float* Wsrc, const float
                                 const int32_t* perm, int64_t T, int E, int H, int b_kmajor, int accumulate,
                                 float* out, cudaStream_t s);
 
-// Same contraction on tcgen05 (TF32 in, FP32 accumulate). Bsrc is [E][H][H]
-// with Bsrc[e][n][k] = B_e[n, k] (K-major).
-cudaError_t launch_grouped_tf32(const float* src, const float* Bsrc, const float* bias, const int32_t* offsets,
-                                const int32_t* perm, int64_t T, int E, int H, int accumulate, float* out,
-                                uint32_t* dev_flags, int num_sms, cudaStream_t s);
-
-cudaError_t launch_transpose_w(const float* W, int E, int H, float* Wt, cudaStream_t s);
+// Same contraction on tcgen05 (TF32 in, FP32 accumulate), straight from W
+// [E][H][H]: w_transposed = 0: B_e[n, k] = W[e][n][k] (forward);
+// w_transposed = 1: B_e[n, k] = W[e][k][n] (input gradient).
+cudaError_t launch_grouped_tf32(const float* src, const float* W, const float* bias, const int32_t* offsets,
+                                const int32_t* perm, int64_t T, int E, int H, int w_transposed, int accumulate,
+                                float* out, uint32_t* dev_flags, int num_sms, cudaStream_t s);
 
 // Per-range partial sums of dW / db into the slot buffers (see wgrad_splits).
 cudaError_t launch_wgrad_ffma(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,

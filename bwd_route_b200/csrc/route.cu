@@ -101,48 +101,62 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
                                                          int E, int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ blk_base) {
-    __shared__ int s_tot[32];
-    __shared__ int s_off[33];
+    // Each expert gets Q = 32 / E warps; warp q of expert e owns a contiguous
+    // run of routing blocks. Pass 1 sums each run, one thread turns the run sums
+    // into the expert totals, the offsets and each run's starting base, and pass
+    // 2 scans each run from its base. The first batch of a run stays in
+    // registers between the passes, so a run of up to 256 blocks (every expert at
+    // 262144 tokens for E = 8) reads the per-block counts once.
+    __shared__ int s_part[32];
+    __shared__ int s_base[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Q = 32 / E;
+    const int e = warp / Q, q = warp - e * Q;
     constexpr int kBatch = 8;  // chunks of 32 blocks loaded before they are used
-    if (warp < E) {
-        int tot = 0;
-        for (int64_t c0 = 0; c0 < nblk; c0 += 32 * kBatch) {
-            int v[kBatch];
+    const int64_t run = (nblk + Q - 1) / Q;
+    const int64_t lo = q * run;
+    const int64_t hi = lo + run < nblk ? lo + run : nblk;
+    auto load = [&](int64_t c0, int (&v)[kBatch]) {
 #pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int64_t b = c0 + j * 32 + lane;
-                v[j] = (b < nblk) ? blk_counts[b * E + warp] : 0;
-            }
+        for (int j = 0; j < kBatch; ++j) {
+            const int64_t b = c0 + j * 32 + lane;
+            v[j] = (b < hi) ? blk_counts[b * E + e] : 0;
+        }
+    };
+    int v0[kBatch];
+    if (e < E) {
+        int tot = 0;
+        load(lo, v0);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) tot += v0[j];
+        for (int64_t c0 = lo + 32 * kBatch; c0 < hi; c0 += 32 * kBatch) {
+            int v[kBatch];
+            load(c0, v);
 #pragma unroll
             for (int j = 0; j < kBatch; ++j) tot += v[j];
         }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
-        if (lane == 0) s_tot[warp] = tot;
+        if (lane == 0) s_part[warp] = tot;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            counts[e] = s_tot[e];
-            offsets[e] = run;
-            s_off[e] = run;
-            run += s_tot[e];
+        int acc = 0;
+        for (int ee = 0; ee < E; ++ee) {
+            offsets[ee] = acc;
+            const int first = acc;
+            for (int qq = 0; qq < Q; ++qq) {
+                s_base[ee * Q + qq] = acc;
+                acc += s_part[ee * Q + qq];
+            }
+            counts[ee] = acc - first;
         }
-        offsets[E] = run;
+        offsets[E] = acc;
     }
     __syncthreads();
-    if (warp < E) {
-        const int e = warp;
-        int carry = s_off[e];
-        for (int64_t c0 = 0; c0 < nblk; c0 += 32 * kBatch) {
-            int v[kBatch];
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int64_t b = c0 + j * 32 + lane;
-                v[j] = (b < nblk) ? blk_counts[b * E + e] : 0;
-            }
+    if (e < E) {
+        int carry = s_base[warp];
+        auto scan = [&](int64_t c0, const int (&v)[kBatch]) {
 #pragma unroll
             for (int j = 0; j < kBatch; ++j) {
                 int incl = v[j];
@@ -152,9 +166,15 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
                     if (lane >= off) incl += u;
                 }
                 const int64_t b = c0 + j * 32 + lane;
-                if (b < nblk) blk_base[b * E + e] = carry + incl - v[j];
+                if (b < hi) blk_base[b * E + e] = carry + incl - v[j];
                 carry += __shfl_sync(0xffffffffu, incl, 31);
             }
+        };
+        scan(lo, v0);
+        for (int64_t c0 = lo + 32 * kBatch; c0 < hi; c0 += 32 * kBatch) {
+            int v[kBatch];
+            load(c0, v);
+            scan(c0, v);
         }
     }
 }

@@ -20,11 +20,11 @@ from . import ops
 
 
 class MoETop1Gate:
-    # kernels launched per step() with T > 0: route 3, fwd 1, bwd (TF32: transpose +
-    # d_x + wgrad + reduce = 4; FFMA: d_x + wgrad + reduce = 3), aux 2, lambda 1
+    # kernels launched per step() with T > 0: route 3, fwd 1, bwd (d_x + wgrad +
+    # reduce) 3, aux 2, lambda 1 -- the same for both math modes
     @staticmethod
     def launches_per_step(math: int) -> int:
-        return 3 + 1 + (4 if math == ops.MOE_MATH_TF32 else 3) + 2 + 1
+        return 3 + 1 + 3 + 2 + 1
 
     def __init__(self, W: torch.Tensor, bias: torch.Tensor, B: int, N_H: int, math: int = ops.MOE_MATH_TF32,
                  lambda_floor: float = 0.01, lambda_max_extra: float = 0.09, ent_target: float = 1.0,
