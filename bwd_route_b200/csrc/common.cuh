@@ -1,5 +1,5 @@
 // common.cuh -- device helpers for the sm_100a kernels of the top-1 MoE gate:
-// mbarriers with bounded waits, TMA loads (2D tile and tile::gather4), tcgen05
+// mbarriers with bounded waits, TMA 2D tile loads, cp.async gathers, tcgen05
 // tensor-memory allocation, MMA, commit and loads, and the shared-memory matrix
 // descriptors the MMA reads its operands through.
 #pragma once
@@ -88,19 +88,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Row gather: four rows r0..r3 of a 2D tensor (box one row high, box width from
-// the map) starting at inner coordinate c0, written to dst as four consecutive
-// box rows. A row index outside the tensor reads zeros.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int32_t c0, int32_t r0,
-                                            int32_t r1, int32_t r2, int32_t r3, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -253,28 +240,26 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, int a_mn, int b_
 }
 
 // ---------------------------------------------------------------- misc
-// Global -> shared copy of n4 float4 by nthreads threads, BATCH independent
-// 128-bit loads in flight per thread before any store.
-template <int BATCH>
-__device__ __forceinline__ void stage_f4(float4* dst, const float4* __restrict__ src, int n4, int tid,
-                                         int nthreads) {
-    for (int base = 0; base < n4; base += BATCH * nthreads) {
-        float4 v[BATCH];
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int i = base + u * nthreads + tid;
-            if (i < n4) v[u] = __ldg(src + i);
-        }
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int i = base + u * nthreads + tid;
-            if (i < n4) dst[i] = v[u];
-        }
-    }
+// Predicated streaming store: no branch around the store, so a loop of them
+// has no control dependence on the (shuffled) predicate.
+__device__ __forceinline__ void st_global_cs_v4_pred(float* p, float4 v, bool pred) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.u32 q, %5, 0;\n\t"
+        "@q st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};\n\t}" ::"l"(p),
+        "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(static_cast<uint32_t>(pred)));
 }
 
-__device__ __forceinline__ void st_global_cs_v4(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+// Explicit shared-memory vector accesses (a pointer carved out of the dynamic
+// shared buffer by integer arithmetic would otherwise be accessed generically).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d));
+}
+__device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
 
-__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 }  // namespace moe

@@ -287,22 +287,33 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
         constexpr int HALF = H / 2;
         const int q = warp & 3;
         const int c0 = (warp >> 2) * HALF;
-        float* my = stg + warp * 32 * 32;
+        const uint32_t my_u32 = smem_u32(stg + warp * 32 * 32);  // this warp's 32 x 32 transpose buffer
         const int j = lane & 7;
+        const int myrow = 32 * q + lane;
+        // This lane's token of a tile: loaded one tile ahead, so that the DRAM
+        // latency of perm[] is never exposed between two tiles.
+        auto tile_token = [&](int tile) -> int {
+            const int e = find_expert(ctl->tstart, E, tile);
+            const int row0 = ctl->off[e] + (tile - ctl->tstart[e]) * C::BM;
+            return (myrow < ctl->off[e + 1] - row0) ? perm[row0 + myrow] : -1;
+        };
+        int tok_next = static_cast<int>(blockIdx.x) < ntiles ? tile_token(blockIdx.x) : -1;
+        // the bias this lane adds in each 32-column chunk; reloaded only when the expert changes
+        float4 bv[HALF / 32];
+        int bias_e = -1;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
             const int e = find_expert(ctl->tstart, E, tile);
-            const int row0 = ctl->off[e] + (tile - ctl->tstart[e]) * C::BM;
-            const int nrows = min(C::BM, ctl->off[e + 1] - row0);
-            const int myrow = 32 * q + lane;
-            const int tok_mine = (myrow < nrows) ? perm[row0 + myrow] : -1;
-            // the bias this lane adds in each 32-column chunk, loaded before the wait
-            float4 bv[HALF / 32];
+            const int tok_mine = tok_next;
+            if (tile + static_cast<int>(gridDim.x) < ntiles) tok_next = tile_token(tile + gridDim.x);
+            if (e != bias_e) {
 #pragma unroll
-            for (int c = 0; c < HALF / 32; ++c)
-                bv[c] = bias ? __ldg(reinterpret_cast<const float4*>(bias + static_cast<int64_t>(e) * H + c0 + c * 32) + j)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int c = 0; c < HALF / 32; ++c)
+                    bv[c] = bias ? __ldg(reinterpret_cast<const float4*>(bias + static_cast<int64_t>(e) * H + c0 + c * 32) + j)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                bias_e = e;
+            }
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, abort, dev_flags)) break;
             __syncwarp();
             tc_fence_after();
@@ -316,31 +327,40 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                     const int c = cc * 2 + h;  // 32-column chunk within the half
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj)
-                        *reinterpret_cast<float4*>(my + lane * 32 + ((jj ^ (lane & 7)) * 4)) =
-                            make_float4(v[32 * h + 4 * jj], v[32 * h + 4 * jj + 1], v[32 * h + 4 * jj + 2],
-                                        v[32 * h + 4 * jj + 3]);
+                        st_shared_v4(my_u32 + 4 * (lane * 32 + ((jj ^ (lane & 7)) * 4)), v[32 * h + 4 * jj],
+                                     v[32 * h + 4 * jj + 1], v[32 * h + 4 * jj + 2], v[32 * h + 4 * jj + 3]);
                     __syncwarp();
+                    if (accumulate) {
 #pragma unroll
-                    for (int it = 0; it < 8; ++it) {
-                        const int R = it * 4 + (lane >> 3);
-                        float4 val = *reinterpret_cast<const float4*>(my + R * 32 + ((j ^ (R & 7)) * 4));
-                        const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
-                        if (tok >= 0) {
+                        for (int it = 0; it < 8; ++it) {
+                            const int R = it * 4 + (lane >> 3);
+                            const float4 val = ld_shared_v4(my_u32 + 4 * (R * 32 + ((j ^ (R & 7)) * 4)));
+                            const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
+                            if (tok >= 0) {
+                                float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(tok) * H + c0 +
+                                                                        c * 32 + j * 4);
+                                float4 o = *dst;
+                                o.x += val.x + bv[c].x;
+                                o.y += val.y + bv[c].y;
+                                o.z += val.z + bv[c].z;
+                                o.w += val.w + bv[c].w;
+                                *dst = o;
+                            }
+                        }
+                    } else {
+                        // padding rows (tok < 0) only occur in an expert's last tile; the
+                        // stores are predicated rather than branched around
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int R = it * 4 + (lane >> 3);
+                            float4 val = ld_shared_v4(my_u32 + 4 * (R * 32 + ((j ^ (R & 7)) * 4)));
+                            const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
                             val.x += bv[c].x;
                             val.y += bv[c].y;
                             val.z += bv[c].z;
                             val.w += bv[c].w;
-                            float* dst = out + static_cast<int64_t>(tok) * H + c0 + c * 32 + j * 4;
-                            if (accumulate) {
-                                const float4 o = *reinterpret_cast<const float4*>(dst);
-                                val.x += o.x;
-                                val.y += o.y;
-                                val.z += o.z;
-                                val.w += o.w;
-                                *reinterpret_cast<float4*>(dst) = val;
-                            } else {
-                                st_global_cs_v4(dst, val);
-                            }
+                            st_global_cs_v4_pred(out + static_cast<int64_t>(tok < 0 ? 0 : tok) * H + c0 + c * 32 + j * 4,
+                                                 val, tok >= 0);
                         }
                     }
                     __syncwarp();
@@ -428,10 +448,17 @@ wgrad_tf32_kernel(const float* __restrict__ g_src, const float* __restrict__ x_s
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
+        // perm[] of the next stage is loaded one stage ahead (the range's sorted
+        // positions are contiguous, so the next stage starts at p0 + KT or, past
+        // an expert boundary, at that boundary; entries past hi are not loaded)
+        int next_lane = (lo + lane < hi) ? perm[lo + lane] : -1;
+        int next_p0 = lo;
         for (int e = 0; e < E && ok; ++e) {
             const int s = max(lo, ctl->off[e]), t = min(hi, ctl->off[e + 1]);
             for (int p0 = s; p0 < t; p0 += C::KT) {
-                const int tok_lane = (p0 + lane < t) ? perm[p0 + lane] : -1;
+                int tok_lane = (p0 + lane >= t) ? -1 : (p0 == next_p0) ? next_lane : perm[p0 + lane];
+                next_p0 = (p0 + C::KT < t) ? p0 + C::KT : t;
+                next_lane = (next_p0 + lane < hi) ? perm[next_p0 + lane] : -1;
                 if (!(ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags))) break;
                 const uint32_t base = smem_u32(stages + stage * C::STAGE_BYTES);
 #pragma unroll

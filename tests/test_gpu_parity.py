@@ -35,6 +35,10 @@ EDGE = [
     wl.make_spec("max_experts_b2000_e32_h128", 2000, 3, 32, 128, 15),
     wl.make_spec("h256_b1500_e8_h256", 1500, 3, 8, 256, 16),
     wl.make_spec("h256_skewed_b777_e3_h256", 777, 1, 3, 256, 17, skew_expert=1, skew_value=3.0),
+    # H = 256 with more 256-token tiles than CTA pairs: pairs run several tiles
+    # and change expert inside their run (the expert weights are reloaded).
+    wl.make_spec("h256_b4096_e8_h256", 4096, 8, 8, 256, 18),
+    wl.make_spec("h256_max_experts_b4000_e32_h256", 4000, 5, 32, 256, 19),
 ]
 
 
@@ -140,9 +144,11 @@ def test_tf32_operand_rounding_rule():
     assert matches[tf32_mode(ops.MOE_MATH_TF32)], matches
 
 
+@pytest.mark.parametrize("name", ["skewed_b4096_e8_h128", "h256"])
 @pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
-def test_deterministic_bitwise(math_mode):
-    inp = wl.generate(wl.WORKLOADS["skewed_b4096_e8_h128"])
+def test_deterministic_bitwise(math_mode, name):
+    spec = wl.make_spec("det_b4096_e8_h256", 4096, 4, 8, 256, 22) if name == "h256" else wl.WORKLOADS[name]
+    inp = wl.generate(spec)
     a = run_gpu(inp, math_mode, 0.02)
     b = run_gpu(inp, math_mode, 0.02)
     for k in ["expert_idx", "perm", "routed", "d_x", "dW", "db", "d_logits", "loss", "mean_p", "stats"]:
@@ -162,9 +168,10 @@ def test_uniform_logits_aux_is_exactly_one():
     assert np.all(np.abs(g["d_logits"].sum(axis=1)) <= 1e-6 * np.abs(g["d_logits"]).sum(axis=1) + 1e-12)
 
 
+@pytest.mark.parametrize("H", [128, 256])
 @pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
-def test_accumulate_flags(math_mode):
-    inp = wl.generate(wl.make_spec("acc_b600_e4_h128", 600, 2, 4, 128, 21))
+def test_accumulate_flags(math_mode, H):
+    inp = wl.generate(wl.make_spec(f"acc_b600_e4_h{H}", 600, 2, 4, H, 21))
     rng = np.random.default_rng(0)
     T, E, H = inp.spec.T, inp.spec.E, inp.spec.H
     pre = {"d_x": rng.standard_normal((T, H)).astype(np.float32),
