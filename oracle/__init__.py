@@ -50,6 +50,7 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_aux.argtypes = [P, P, i64, i32, ctypes.c_float, P, P, P, P, P]
     lib.oracle_lambda_eff.restype = ctypes.c_double
     lib.oracle_lambda_eff.argtypes = [ctypes.c_double] * 4
+    lib.oracle_usage_entropy_ema.argtypes = [P, i64, i32, ctypes.c_double, i32, P, P, P]
     return lib
 
 
@@ -159,6 +160,18 @@ def aux(gate_logits, counts, lambda_eff: float):
 
 def lambda_eff(ent_ema: float, lambda_floor: float, lambda_max_extra: float, ent_target: float) -> float:
     return float(_load().oracle_lambda_eff(ent_ema, lambda_floor, lambda_max_extra, ent_target))
+
+
+def usage_entropy_ema(counts, T: int, alpha: float, reset: bool, usage_ema, ent_ema: float):
+    """One update of the gate-entropy producer: returns (usage_ema', ent_ema', H of this step)."""
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    E = c.shape[0]
+    u = np.array(usage_ema, dtype=np.float64).reshape(E).copy()
+    ent = ctypes.c_double(float(ent_ema))
+    h = ctypes.c_double(0.0)
+    _load().oracle_usage_entropy_ema(_p(c), int(T), E, float(alpha), int(bool(reset)), _p(u), ctypes.byref(ent),
+                                     ctypes.byref(h))
+    return u, ent.value, h.value
 
 
 def step(inp, lambda_eff_value: float | None = None, tf32_mode: int = TF32_NONE, with_dw: bool = True):

@@ -14,7 +14,8 @@
  *   [P1] foxhunt commit 11b96dac6a, "Top-1 Mixture-of-Experts gate per Switch
  *        Transformer": kernel list, ARCHITECTURE, PERFORMANCE.
  *   [P2] foxhunt commit 2d0e6b6bdc, "Replace static moe_lambda=0.01 with a
- *        GPU-driven controller": the lambda_eff formula and its unit test.
+ *        GPU-driven controller": the lambda_eff formula and its unit test; the
+ *        constructor bootstrap and fold-boundary reset of the controller state.
  *   [P4] foxhunt commit 6cfd7e6691, "Per-(batch, horizon) softmax + cross-entropy
  *        loss + gradient": Kernel section (numerically stable softmax).
  *
@@ -285,4 +286,39 @@ double oracle_lambda_eff(double ent_ema, double lambda_floor, double lambda_max_
     double deficit = ent_target - ent_ema;
     if (!(deficit > 0.0)) deficit = 0.0;
     return lambda_floor + lambda_max_extra * deficit / ent_target;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Producer of ent_ema, the gate-entropy signal the lambda controller reads.  */
+/* [P2] opening paragraph and Wiring: ent_ema comes from an existing          */
+/* producer; the constructor puts 1/K in every per-expert usage slot and ln K */
+/* in the entropy slot (cold start), and the lambda slot goes back to its     */
+/* floor at a fold boundary. The pages name neither the entropy's input nor   */
+/* the averaging weight. Reading used: the entropy of this step's argmax      */
+/* usage fractions frac_e = counts[e] / T,                                    */
+/*   H = - sum_e frac_e ln frac_e          (a term with frac_e = 0 is 0),     */
+/* averaged with a caller-set weight alpha of the newest step:                */
+/*   usage_ema[e] <- (1 - alpha) usage_ema[e] + alpha frac_e                  */
+/*   ent_ema      <- (1 - alpha) ent_ema      + alpha H                       */
+/* reset != 0 writes the cold-start state instead (1/E per expert, ln E).     */
+/* T == 0 is no observation: the state is left as it is and H is 0.           */
+/* ------------------------------------------------------------------------- */
+void oracle_usage_entropy_ema(const int32_t* counts, int64_t T, int32_t E, double alpha, int32_t reset,
+                              double* usage_ema, double* ent_ema, double* ent_step)
+{
+    double h = 0.0;
+    for (int32_t e = 0; e < E && T > 0; ++e) {
+        const double f = (double)counts[e] / (double)T;
+        if (f > 0.0) h -= f * log(f);
+    }
+    *ent_step = h;
+    if (reset) {
+        for (int32_t e = 0; e < E; ++e) usage_ema[e] = 1.0 / (double)E;
+        *ent_ema = log((double)E);
+        return;
+    }
+    if (T <= 0) return;
+    for (int32_t e = 0; e < E; ++e)
+        usage_ema[e] = (1.0 - alpha) * usage_ema[e] + alpha * ((double)counts[e] / (double)T);
+    *ent_ema = (1.0 - alpha) * *ent_ema + alpha * h;
 }

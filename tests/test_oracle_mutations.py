@@ -45,6 +45,12 @@ MUTATIONS = [
     ("lambda deficit not normalised", "return lambda_floor + lambda_max_extra * deficit / ent_target;",
      "return lambda_floor + lambda_max_extra * deficit;"),
     ("tf32 keeps all bits", "    u &= 0xFFFFE000u;", "    u &= 0xFFFFFFFFu;"),
+    ("usage entropy sign flipped", "if (f > 0.0) h -= f * log(f);", "if (f > 0.0) h += f * log(f);"),
+    ("entropy average weights swapped", "*ent_ema = (1.0 - alpha) * *ent_ema + alpha * h;",
+     "*ent_ema = alpha * *ent_ema + (1.0 - alpha) * h;"),
+    ("usage average from the wrong expert", "usage_ema[e] = (1.0 - alpha) * usage_ema[e] + alpha * ((double)counts[e] / (double)T);",
+     "usage_ema[e] = (1.0 - alpha) * usage_ema[e] + alpha * ((double)counts[0] / (double)T);"),
+    ("cold start entropy wrong", "*ent_ema = log((double)E);", "*ent_ema = 1.0 / (double)E;"),
 ]
 
 

@@ -421,3 +421,76 @@ def test_lambda_eff_five_regimes():
 def test_lambda_eff_cold_start_is_floor():
     for K in (2, 4, 8, 32):
         assert oracle.lambda_eff(math.log(K), 0.01, 0.09, 0.7 * math.log(K)) == 0.01
+
+
+# --------------------------------------------------------------------------- entropy producer
+
+def _scipy_entropy(p):
+    from scipy.stats import entropy
+    return float(entropy(p))
+
+
+def test_usage_entropy_matches_scipy_and_closed_forms():
+    rng = np.random.default_rng(5)
+    for E in (1, 2, 3, 8, 17, 32):
+        counts = rng.integers(0, 1000, E).astype(np.int32)
+        counts[rng.integers(0, E)] = 0                    # an inactive expert contributes 0 ln 0 = 0
+        T = int(counts.sum())
+        if T == 0:
+            continue
+        _, _, h = oracle.usage_entropy_ema(counts, T, 0.5, False, np.full(E, 1.0 / E), 0.0)
+        assert abs(h - _scipy_entropy(counts / T)) <= 1e-12 * max(1.0, h)
+    for E in (2, 4, 8, 32):                               # uniform usage: ln E
+        _, _, h = oracle.usage_entropy_ema(np.full(E, 7, np.int32), 7 * E, 0.1, False, np.full(E, 1.0 / E), 0.0)
+        assert abs(h - math.log(E)) <= 1e-14
+    _, _, h = oracle.usage_entropy_ema(np.array([0, 0, 9, 0], np.int32), 9, 0.1, False, np.full(4, 0.25), 1.0)
+    assert h == 0.0                                       # everything on one expert
+    _, _, h = oracle.usage_entropy_ema(np.array([3, 0, 3, 0], np.int32), 6, 0.1, False, np.full(4, 0.25), 1.0)
+    assert abs(h - math.log(2)) <= 1e-15                  # two equal halves
+
+
+def test_usage_entropy_ema_weights_and_limits():
+    counts = np.array([10, 30, 0, 60], np.int32)
+    T = 100
+    frac = counts / T
+    h = _scipy_entropy(frac)
+    u0, e0 = np.array([0.1, 0.2, 0.3, 0.4]), 0.9
+    u, e, _ = oracle.usage_entropy_ema(counts, T, 1.0, False, u0, e0)      # weight 1: the step itself
+    np.testing.assert_allclose(u, frac, rtol=0, atol=1e-15)
+    assert abs(e - h) <= 1e-15
+    u, e, _ = oracle.usage_entropy_ema(counts, T, 0.0, False, u0, e0)      # weight 0: unchanged
+    np.testing.assert_array_equal(u, u0)
+    assert e == e0
+    u, e, _ = oracle.usage_entropy_ema(counts, T, 0.25, False, u0, e0)     # the weighted mean
+    np.testing.assert_allclose(u, 0.75 * u0 + 0.25 * frac, rtol=0, atol=1e-15)
+    assert abs(e - (0.75 * e0 + 0.25 * h)) <= 1e-15
+    assert abs(u.sum() - 1.0) <= 1e-15                                      # still a distribution
+
+
+def test_usage_entropy_ema_geometric_approach():
+    """n updates with the same counts: ent_n = H + (ent_0 - H) (1 - alpha)^n."""
+    counts = np.array([50, 25, 25], np.int32)
+    alpha = 0.2
+    h = _scipy_entropy(counts / 100)
+    u, e = np.full(3, 1.0 / 3), math.log(3)
+    for n in range(1, 40):
+        u, e, _ = oracle.usage_entropy_ema(counts, 100, alpha, False, u, e)
+        assert abs(e - (h + (math.log(3) - h) * (1 - alpha) ** n)) <= 1e-13
+        np.testing.assert_allclose(u, counts / 100 + (1.0 / 3 - counts / 100) * (1 - alpha) ** n, rtol=0, atol=1e-14)
+
+
+def test_usage_entropy_reset_is_the_cold_start_and_gives_the_floor():
+    """The pages' bootstrap (usage 1/K, entropy ln K) and fold-boundary reset (lambda at its floor)."""
+    for E in (2, 4, 8, 32):
+        u, e, _ = oracle.usage_entropy_ema(np.arange(E, dtype=np.int32), E * (E - 1) // 2, 0.3, True,
+                                           np.zeros(E), 0.123)
+        np.testing.assert_array_equal(u, np.full(E, 1.0 / E))
+        assert e == math.log(E)
+        assert oracle.lambda_eff(e, 0.01, 0.09, 0.7 * math.log(E)) == 0.01
+
+
+def test_usage_entropy_no_tokens_is_no_observation():
+    u0 = np.array([0.5, 0.5])
+    u, e, h = oracle.usage_entropy_ema(np.zeros(2, np.int32), 0, 0.5, False, u0, 0.3)
+    np.testing.assert_array_equal(u, u0)
+    assert e == 0.3 and h == 0.0
