@@ -358,4 +358,22 @@ moe_status_t moe_lambda_eff_update(const float* ent_ema, float lambda_floor, flo
                                          static_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_usage_entropy_ema_update(const int32_t* counts, int64_t T, int32_t E, float alpha,
+                                          int32_t reset, float* usage_ema, float* ent_ema, float* ent_step,
+                                          void* stream) {
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || E > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!counts || !usage_ema || !ent_ema) return MOE_ERR_INVALID_ARG;
+    if (!(alpha >= 0.0f && alpha <= 1.0f)) return MOE_ERR_INVALID_ARG;  // NaN fails too
+    if (!aligned(counts, 4) || !aligned(usage_ema, 4) || !aligned(ent_ema, 4) || (ent_step && !aligned(ent_step, 4)))
+        return MOE_ERR_MISALIGNED;
+    const Range outs[3] = {{usage_ema, sizeof(float) * static_cast<size_t>(E)},
+                           {ent_ema, sizeof(float)},
+                           {ent_step, ent_step ? sizeof(float) : 0}};
+    const Range ins[1] = {{counts, sizeof(int32_t) * static_cast<size_t>(E)}};
+    if (any_alias(outs, 3, ins, 1)) return MOE_ERR_ALIAS;
+    return cuda_status(launch_usage_entropy_ema(counts, T, E, alpha, reset ? 1 : 0, usage_ema, ent_ema, ent_step,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -252,7 +252,38 @@ __global__ void lambda_eff_kernel(const float* __restrict__ ent_ema, float lambd
     *lambda_eff = lambda_floor + lambda_max_extra * deficit / ent_target;
 }
 
+// Producer of the gate-entropy signal the lambda controller reads (one warp;
+// lane e owns expert e): H = -sum_e frac_e ln frac_e over this step's argmax
+// usage fractions, then the caller-weighted moving averages of frac and H, or
+// the cold-start state on a reset. Double inside, fp32 in memory; the sum over
+// experts is one fixed xor butterfly, read from lane 0.
+__global__ void usage_entropy_ema_kernel(const int32_t* __restrict__ counts, int64_t T, int E, float alpha,
+                                         int reset, float* __restrict__ usage_ema, float* __restrict__ ent_ema,
+                                         float* __restrict__ ent_step) {
+    const int lane = threadIdx.x;
+    const bool on = lane < E;
+    const double f = (on && T > 0) ? static_cast<double>(counts[lane]) / static_cast<double>(T) : 0.0;
+    double h = f > 0.0 ? -f * log(f) : 0.0;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) h += __shfl_xor_sync(0xffffffffu, h, off);
+    if (reset) {
+        if (on) usage_ema[lane] = static_cast<float>(1.0 / static_cast<double>(E));
+        if (lane == 0) *ent_ema = static_cast<float>(log(static_cast<double>(E)));
+    } else if (T > 0) {
+        const double a = alpha;
+        if (on) usage_ema[lane] = static_cast<float>((1.0 - a) * static_cast<double>(usage_ema[lane]) + a * f);
+        if (lane == 0) *ent_ema = static_cast<float>((1.0 - a) * static_cast<double>(*ent_ema) + a * h);
+    }
+    if (lane == 0 && ent_step) *ent_step = static_cast<float>(h);
+}
+
 }  // namespace
+
+cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, float alpha, int reset,
+                                     float* usage_ema, float* ent_ema, float* ent_step, cudaStream_t s) {
+    usage_entropy_ema_kernel<<<1, 32, 0, s>>>(counts, T, E, alpha, reset, usage_ema, ent_ema, ent_step);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, int E, const float* lambda_eff,
                        float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,

@@ -76,6 +76,9 @@ cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, in
                        float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,
                        cudaStream_t s);
 
+cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, float alpha, int reset,
+                                     float* usage_ema, float* ent_ema, float* ent_step, cudaStream_t s);
+
 cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float lambda_max_extra, float ent_target,
                               float* lambda_eff, cudaStream_t s);
 

@@ -49,6 +49,8 @@ class MoETop1Gate:
         self.stats = torch.zeros(3 * E + 4, dtype=f32, device=dev) if stats else None
         self.lambda_eff = torch.full((1,), lambda_floor, dtype=f32, device=dev)
         self.ent_ema = torch.full((1,), ent_ema, dtype=f32, device=dev)
+        self.usage_ema = torch.full((E,), 1.0 / E, dtype=f32, device=dev)
+        self.ent_step = torch.zeros(1, dtype=f32, device=dev)
         self.ws = ops.new_workspace(T, E, H, dev)
 
     def route(self, gate_logits, stream=None):
@@ -69,6 +71,14 @@ class MoETop1Gate:
     def update_lambda(self, stream=None):
         ops.moe_lambda_eff_update(self.ent_ema, self.lambda_floor, self.lambda_max_extra, self.ent_target,
                                   self.lambda_eff, stream)
+
+    def update_controller(self, alpha: float, reset: bool = False, stream=None):
+        """Closes the lambda loop after a step: the gate-entropy producer folds
+        this step's usage into ent_ema (or resets it at a fold boundary), then
+        lambda_eff is recomputed from it for the next step."""
+        ops.moe_usage_entropy_ema_update(self.routing.counts, self.T, self.E, alpha, reset, self.usage_ema,
+                                         self.ent_ema, self.ent_step, stream)
+        self.update_lambda(stream)
 
     def step(self, gate_logits, x, d_out, stream=None):
         self.route(gate_logits, stream)

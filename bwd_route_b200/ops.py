@@ -29,6 +29,7 @@ EXPORTED = [
     "moe_top1_workspace_bytes", "moe_top1_workspace_init", "moe_top1_route", "moe_top1_fwd",
     "moe_top1_bwd", "moe_aux_loss_fwd_bwd", "moe_lambda_eff_update", "moe_top1_device_flags",
     "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc", "moe_top1_selftest_wait_timeout",
+    "moe_usage_entropy_ema_update",
 ]
 MOE_NOALLOC_MAX_TOKENS = 2097152
 
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.moe_top1_abi_version.argtypes = []
         L.moe_top1_selftest_wait_timeout.restype = I32
         L.moe_top1_selftest_wait_timeout.argtypes = [P, SZ, I64, P]
+        L.moe_usage_entropy_ema_update.restype = I32
+        L.moe_usage_entropy_ema_update.argtypes = [P, I64, I32, ctypes.c_float, I32, P, P, P, P]
         L.moe_top1_route_noalloc.restype = I32
         L.moe_top1_route_noalloc.argtypes = [P, I64, I64, I32, ctypes.POINTER(RoutingC), P]
         _lib = L
@@ -196,6 +199,17 @@ def moe_lambda_eff_update(ent_ema, lambda_floor: float, lambda_max_extra: float,
     _check("moe_lambda_eff_update",
            lib().moe_lambda_eff_update(_ptr(ent_ema, f), lambda_floor, lambda_max_extra, ent_target,
                                        _ptr(lambda_eff, f), _stream(stream)))
+
+
+def moe_usage_entropy_ema_update(counts, T: int, E: int, alpha: float, reset: bool, usage_ema, ent_ema,
+                                 ent_step=None, stream=None):
+    """Gate-entropy producer for the lambda controller: updates usage_ema [E] and
+    ent_ema [1] in place from this step's counts (or resets them to 1/E, ln E)."""
+    f = torch.float32
+    _check("moe_usage_entropy_ema_update",
+           lib().moe_usage_entropy_ema_update(_ptr(counts, torch.int32), T, E, alpha, int(bool(reset)),
+                                              _ptr(usage_ema, f), _ptr(ent_ema, f), _ptr(ent_step, f),
+                                              _stream(stream)))
 
 
 def moe_top1_selftest_wait_timeout(ws: torch.Tensor, limit_cycles: int, stream=None):

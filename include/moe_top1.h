@@ -205,6 +205,28 @@ moe_status_t moe_lambda_eff_update(const float* ent_ema, float lambda_floor,
                                    float lambda_max_extra, float ent_target, float* lambda_eff,
                                    void* stream);
 
+/*
+ * Producer of the gate-entropy signal ent_ema that moe_lambda_eff_update reads.
+ * [P2] opening paragraph (ent_ema comes from an existing producer) and Wiring
+ * (the constructor puts 1/K in every per-expert usage slot and ln K in the
+ * entropy slot; lambda returns to its floor at a fold boundary). The pages name
+ * neither the entropy's input nor the averaging weight; this call uses the
+ * entropy of the step's argmax usage fractions and a caller-set weight:
+ *   frac[e] = counts[e] / T,   H = -sum_e frac[e] ln frac[e]   (0 ln 0 = 0)
+ *   usage_ema[e] <- (1 - alpha) usage_ema[e] + alpha frac[e]
+ *   ent_ema      <- (1 - alpha) ent_ema      + alpha H
+ * reset != 0 writes the cold-start state instead: usage_ema[e] = 1/E,
+ * ent_ema = ln E (so the next lambda is the floor). T = 0 leaves the state as it
+ * is (no observation). counts [E] int32 (the routing's counts), usage_ema [E]
+ * and ent_ema (device scalar) float, read and written in place; ent_step
+ * (device scalar) receives H, or NULL. alpha in [0, 1]; 1 <= E <= 32; outputs
+ * must not overlap each other or counts. Computed in double, stored as float;
+ * one warp, deterministic. No workspace.
+ */
+moe_status_t moe_usage_entropy_ema_update(const int32_t* counts, int64_t T, int32_t E, float alpha,
+                                          int32_t reset, float* usage_ema, float* ent_ema, float* ent_step,
+                                          void* stream);
+
 /* Diagnostic (no counterpart on the pages): launches one thread that waits on
  * a barrier nothing arrives on, through the same bounded wait as the tensor-core
  * kernels, with a limit of limit_cycles SM clock cycles (1 .. 4e9). The wait

@@ -143,6 +143,23 @@ def test_aux_and_lambda_reject_bad_arguments(L):
     assert u(_p(A + 2), 0.01, 0.09, 1.0, out, None) == MISALIGNED
 
 
+def test_usage_entropy_update_rejects_bad_arguments(L):
+    u = L.moe_usage_entropy_ema_update
+    cnt, ue, ee, hs = _p(A), _p(A + 0x100), _p(A + 0x200), _p(A + 0x300)
+    assert u(cnt, 100, 0, 0.1, 0, ue, ee, hs, None) == SHAPE
+    assert u(cnt, 100, 33, 0.1, 0, ue, ee, hs, None) == SHAPE
+    assert u(cnt, -1, 8, 0.1, 0, ue, ee, hs, None) == INVALID
+    assert u(None, 100, 8, 0.1, 0, ue, ee, hs, None) == INVALID
+    assert u(cnt, 100, 8, 0.1, 0, None, ee, hs, None) == INVALID
+    assert u(cnt, 100, 8, 0.1, 0, ue, None, hs, None) == INVALID
+    for bad in (-0.1, 1.5, float("nan")):
+        assert u(cnt, 100, 8, bad, 0, ue, ee, hs, None) == INVALID
+    assert u(cnt, 100, 8, 0.1, 0, _p(A + 0x102), ee, hs, None) == MISALIGNED
+    assert u(cnt, 100, 8, 0.1, 0, ue, _p(A + 0x104), hs, None) == ALIAS      # ent_ema inside usage_ema [8]
+    assert u(cnt, 100, 8, 0.1, 0, ue, ee, _p(A + 0x200), None) == ALIAS      # ent_step on ent_ema
+    assert u(cnt, 100, 8, 0.1, 0, _p(A + 0x10), ee, hs, None) == ALIAS      # usage_ema over counts [8]
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
