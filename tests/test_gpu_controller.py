@@ -88,12 +88,12 @@ def test_closed_loop_follows_the_oracle_and_is_deterministic():
         prev_u, prev_e = gate.usage_ema.cpu().numpy().astype(np.float64), float(gate.ent_ema.item())
         rng = np.random.default_rng(7)
         trace = []
-        for step in range(12):
+        for step in range(20):
             logits = inp.gate_logits + rng.normal(0, 0.5, inp.gate_logits.shape).astype(np.float32)
             gate.route(torch.from_numpy(logits).cuda())
-            gate.update_controller(0.1)
+            gate.update_controller(0.2)
             counts = oracle.route(logits)[1]
-            ou, oe, _ = oracle.usage_entropy_ema(counts, T, 0.1, False, prev_u, prev_e)
+            ou, oe, _ = oracle.usage_entropy_ema(counts, T, 0.2, False, prev_u, prev_e)
             torch.cuda.synchronize()
             gu = gate.usage_ema.cpu().numpy()
             ge = float(gate.ent_ema.item())
