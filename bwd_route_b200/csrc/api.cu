@@ -13,6 +13,7 @@ namespace moe {
 
 cudaError_t aux_set_smem_limits();
 cudaError_t route_set_smem_limits();
+cudaError_t tf32_set_smem_limits();
 
 namespace {
 
@@ -40,6 +41,7 @@ cudaError_t device_info(DeviceInfo** out) {
     if (!d.aux_ready) {
         e = aux_set_smem_limits();
         if (e == cudaSuccess) e = route_set_smem_limits();
+        if (e == cudaSuccess) e = tf32_set_smem_limits();
         if (e != cudaSuccess) return e;
         d.aux_ready = true;
     }
@@ -103,8 +105,52 @@ EncodeTiledFn get_encode_tiled() {
     return g_encode;
 }
 
+namespace {
+
+// Recently encoded tensor maps (a map depends only on the arguments and the
+// device, so the same weight tensor reuses its map on every call).
+struct MapKey {
+    const float* base;
+    uint64_t rows, cols;
+    uint32_t box_cols, box_rows;
+    bool atom32;
+    int dev;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && rows == o.rows && cols == o.cols && box_cols == o.box_cols &&
+               box_rows == o.box_rows && atom32 == o.atom32 && dev == o.dev;
+    }
+};
+constexpr int kMapCache = 16;
+MapKey g_map_key[kMapCache];
+CUtensorMap g_map_val[kMapCache];
+int g_map_n = 0, g_map_next = 0;
+std::mutex g_map_mu;
+
+}  // namespace
+
 bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                  uint32_t box_rows, bool atom32) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const MapKey key{base, rows, cols, box_cols, box_rows, atom32, dev};
+    {
+        std::lock_guard<std::mutex> lock(g_map_mu);
+        for (int i = 0; i < g_map_n; ++i)
+            if (g_map_key[i] == key) {
+                *map = g_map_val[i];
+                return true;
+            }
+    }
+    if (!encode_map_2d(map, base, rows, cols, box_cols, box_rows, atom32)) return false;
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    const int slot = g_map_n < kMapCache ? g_map_n++ : (g_map_next++ % kMapCache);
+    g_map_key[slot] = key;
+    g_map_val[slot] = *map;
+    return true;
+}
+
+bool encode_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                   uint32_t box_rows, bool atom32) {
     EncodeTiledFn enc = get_encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cols, rows};

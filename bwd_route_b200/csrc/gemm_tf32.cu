@@ -611,8 +611,6 @@ template <int H, bool B_MN>
 cudaError_t launch_grouped_tf32_t(const float* src, const CUtensorMap& tm_b, const float* bias,
                                   const int32_t* offsets, const int32_t* perm, int E, int accumulate, float* out,
                                   uint32_t* dev_flags, int grid, cudaStream_t s) {
-    const cudaError_t err = set_smem(grouped_tf32_kernel<H, B_MN>, GCfg<H>::SMEM_BYTES);
-    if (err != cudaSuccess) return err;
     grouped_tf32_kernel<H, B_MN><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
                                                                                   accumulate, out, dev_flags);
     return cudaGetLastError();
@@ -642,21 +640,28 @@ cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t*
                               int64_t T, int E, int H, float* part, float* part_db, uint32_t* dev_flags,
                               cudaStream_t s) {
     const int P = wgrad_splits(T);
-    cudaError_t err;
     if (H == 256) {
-        err = set_smem(wgrad_tf32_kernel<256>, WCfg<256>::SMEM_BYTES);
-        if (err != cudaSuccess) return err;
         wgrad_tf32_kernel<256><<<P, kThreads, WCfg<256>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
                                                                          static_cast<int>(T), E, P, part, part_db,
                                                                          dev_flags);
     } else {
-        err = set_smem(wgrad_tf32_kernel<128>, WCfg<128>::SMEM_BYTES);
-        if (err != cudaSuccess) return err;
         wgrad_tf32_kernel<128><<<P, kThreads, WCfg<128>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
                                                                          static_cast<int>(T), E, P, part, part_db,
                                                                          dev_flags);
     }
     return cudaGetLastError();
+}
+
+// The dynamic shared-memory limits of every tcgen05 kernel, set once per device
+// (before the first launch there) instead of at every launch.
+cudaError_t tf32_set_smem_limits() {
+    cudaError_t e = set_smem(grouped_tf32_kernel<256, false>, GCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<256, true>, GCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, false>, GCfg<128>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, true>, GCfg<128>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(wgrad_tf32_kernel<256>, WCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(wgrad_tf32_kernel<128>, WCfg<128>::SMEM_BYTES);
+    return e;
 }
 
 }  // namespace moe

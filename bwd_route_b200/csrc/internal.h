@@ -114,8 +114,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 EncodeTiledFn get_encode_tiled();
 
 // 2D fp32 tensor [rows][cols] with a 128-byte-swizzled box of box_cols x box_rows
-// (16-byte granules, or 32-byte granules when atom32 is set).
+// (16-byte granules, or 32-byte granules when atom32 is set). make_map_2d returns
+// a cached copy when the same map was encoded before on this device;
+// encode_map_2d always encodes.
 bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                  uint32_t box_rows, bool atom32 = false);
+bool encode_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                   uint32_t box_rows, bool atom32);
 
 }  // namespace moe
