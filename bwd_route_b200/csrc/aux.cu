@@ -27,7 +27,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 32;                                   // tokens a warp handles at a time
-constexpr int kChunksPerWarp = kAuxTokPerBlk / (kWarps * kChunk);  // 4
+constexpr int kChunksPerWarp = kAuxTokPerBlk / (kWarps * kChunk);  // 2
 
 // Shared-memory slot of float4 q (experts 4q..4q+3) of token row t when a row
 // holds Q = EMAX / 4 float4s: the XOR swizzle spreads the 8 rows read by one
@@ -40,8 +40,9 @@ __device__ __forceinline__ int row_slot(int t, int q) {
     return t * Q + (q ^ ((t >> SH) & (Q - 1)));
 }
 
-// One block per 1024 consecutive tokens; warp w handles chunks w, w + 8, w + 16,
-// w + 24 of 32 tokens. The warp stages all four chunks' logits in its own
+// One block per 512 consecutive tokens; warp w handles chunks w and w + 8 of 32
+// tokens (blocks small enough that several waves overlap one another's loads,
+// math and stores). The warp stages both chunks' logits in its own
 // shared buffer (128-bit loads, every load in flight before the first use, no
 // block barrier for the data), lane t computes token t of each chunk reading
 // its row as float4s, and the gradients go back out with 128-bit stores. When
@@ -70,13 +71,28 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
         c0[j] = static_cast<int64_t>(blockIdx.x) * kAuxTokPerBlk + (j * kWarps + warp) * kChunk;
         n[j] = c0[j] >= T ? 0 : static_cast<int>((T - c0[j] < kChunk) ? (T - c0[j]) : kChunk);
     }
+    if (vec) {
+        // cp.async straight into the swizzled rows: all of the warp's copies (Q per
+        // lane per chunk) are in flight before the warp waits once; rows past the
+        // end of a ragged chunk are zero-filled and never used.
 #pragma unroll
-    for (int j = 0; j < kChunksPerWarp; ++j) {
+        for (int j = 0; j < kChunksPerWarp; ++j) {
+            const float4* src4 = reinterpret_cast<const float4*>(logits + (n[j] > 0 ? c0[j] : 0) * E);
+            const uint32_t b32 = smem_u32(wbuf + j * BUF4);
+#pragma unroll
+            for (int u = 0; u < Q; ++u) {
+                const int i = lane + 32 * u;  // float4 i of the chunk: row i / Q, quarter i % Q
+                cp_async_16(b32 + 16 * row_slot<EMAX>(i / Q, i % Q), src4 + (i < n[j] * Q ? i : 0),
+                            i < n[j] * Q ? 16u : 0u);
+            }
+        }
+        cp_async_wait_all();
+        __syncwarp();
+    }
+#pragma unroll
+    for (int j = 0; j < kChunksPerWarp && !vec; ++j) {
         float4* buf = wbuf + j * BUF4;
-        if (vec) {  // c0 * E * 4 bytes is a multiple of 16
-            const float4* src4 = reinterpret_cast<const float4*>(logits + c0[j] * E);
-            for (int i = lane; i < n[j] * Q; i += 32) buf[row_slot<EMAX>(i / Q, i % Q)] = __ldg(src4 + i);
-        } else {
+        {
             float* b = reinterpret_cast<float*>(buf);
             for (int i = lane; i < n[j] * E; i += 32) {
                 const int t = i / E, e = i % E;
@@ -313,7 +329,7 @@ cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float la
 }
 
 cudaError_t aux_set_smem_limits() {
-    // 8 warps x 4 chunks x 32 tokens x 32 experts x 4 bytes = 128 KiB for the widest instance
+    // 8 warps x 2 chunks x 32 tokens x 32 experts x 4 bytes = 64 KiB for the widest instance
     cudaError_t e = cudaFuncSetAttribute(aux_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(float) * kWarps * kChunksPerWarp * kChunk * 16));
     if (e != cudaSuccess) return e;

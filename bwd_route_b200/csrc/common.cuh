@@ -104,6 +104,10 @@ __device__ __forceinline__ void cp_async_16_l2_256(uint32_t dst, const void* src
     asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                  : "memory");
 }
+// Waits until every cp.async this thread issued has landed in shared memory.
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 // The mbarrier receives one arrival once every cp.async issued so far by this
 // thread has landed (the arrival counts against the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {

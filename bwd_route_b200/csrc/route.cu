@@ -11,15 +11,16 @@
 // entries are never chosen; a NaN at e = 0 pins the result to 0).
 //
 // Three launches, all integer-exact and deterministic:
-//   1. route_count   : each warp loads its 128 tokens' logits (a lane group of
-//                      LPT lanes per token, 16 steps in flight), takes the
-//                      group maximum with xor shuffles and the lowest index
-//                      holding it with a ballot; per-block expert counts come
-//                      from warp ballots (no atomics).
+//   1. route_count   : E a multiple of 4: one thread per token scans its row
+//                      (128-bit loads); other E: each warp loads its 128
+//                      tokens' logits (a lane group of LPT lanes per token, 16
+//                      steps in flight), takes the group maximum with xor
+//                      shuffles and the lowest index holding it with a ballot.
+//                      Per-block expert counts (exact integer sums).
 //   2. route_scan    : one block, one warp per expert: counts, offsets and every
 //                      block's base position inside each expert's segment.
-//   3. route_scatter : per-token rank inside its block (warp ballots in token
-//                      order), perm[base + rank] = t.
+//   3. route_scatter : per-token rank inside its block (lanes grouped by
+//                      expert in token order), perm[base + rank] = t.
 #include <cstdint>
 
 #include "common.cuh"
@@ -91,6 +92,64 @@ __global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __re
         for (int w = 0; w < kWarps; ++w) total += s_wcnt[w][threadIdx.x];
         blk_counts[static_cast<int64_t>(blockIdx.x) * E + threadIdx.x] = total;
     }
+}
+
+// The same result when E is a multiple of 4 (E = 4, 8, 16, 32): one thread per
+// token reads its row with 128-bit loads and runs the pages' scan as written
+// (start at e = 0, move only on a strictly greater value), which fixes ties,
+// -0 / +0 and NaN exactly as the definition does. Thread i of the block takes
+// tokens i, i + 256, i + 512, i + 768 (rows of neighbouring lanes are
+// contiguous, so every load instruction is coalesced); TOK of them have their
+// rows in flight at once, few enough that 8 blocks fit on an SM. Per-block expert counts: per-warp aggregated integer
+// adds into shared memory (exact, order-free).
+template <int E>
+__global__ void __launch_bounds__(kThreads, 8) route_count_vec_kernel(const float* __restrict__ logits, int64_t T,
+                                                                  int32_t* __restrict__ expert_idx,
+                                                                  int32_t* __restrict__ blk_counts) {
+    constexpr int Q = E / 4;                               // float4s per row
+    constexpr int TOK = (Q == 1) ? 4 : (Q == 2 ? 2 : 1);   // tokens in flight per thread
+    constexpr int PER = kRouteTokPerBlk / kThreads;         // 4 tokens per thread
+    __shared__ int s_cnt[E];
+    if (threadIdx.x < E) s_cnt[threadIdx.x] = 0;
+    __syncthreads();
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokPerBlk;
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int p0 = 0; p0 < PER; p0 += TOK) {
+        float4 v[TOK][Q];
+#pragma unroll
+        for (int j = 0; j < TOK; ++j) {
+            const int64_t t = t0 + (p0 + j) * kThreads + threadIdx.x;
+            const float4* row = reinterpret_cast<const float4*>(logits + (t < T ? t : 0) * E);
+#pragma unroll
+            for (int q = 0; q < Q; ++q) v[j][q] = __ldg(row + q);
+        }
+#pragma unroll
+        for (int j = 0; j < TOK; ++j) {
+            const int64_t t = t0 + (p0 + j) * kThreads + threadIdx.x;
+            float best = v[j][0].x;
+            int k = 0;
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+                const float x[4] = {v[j][q].x, v[j][q].y, v[j][q].z, v[j][q].w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (q == 0 && r == 0) continue;
+                    if (x[r] > best) {
+                        best = x[r];
+                        k = 4 * q + r;
+                    }
+                }
+            }
+            const bool valid = t < T;
+            if (valid) expert_idx[t] = k;
+            const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+            const unsigned same = __match_any_sync(0xffffffffu, valid ? k : -1) & vmask;
+            if (valid && lane == __ffs(same) - 1) atomicAdd(&s_cnt[k], __popc(same));
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < E) blk_counts[static_cast<int64_t>(blockIdx.x) * E + threadIdx.x] = s_cnt[threadIdx.x];
 }
 
 // One block, warp e scans the per-block counts of expert e: blk_base[b][e] =
@@ -182,40 +241,47 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
 __global__ void __launch_bounds__(kThreads) route_scatter_kernel(const int32_t* __restrict__ expert_idx, int64_t T,
                                                                 int E, const int32_t* __restrict__ blk_base,
                                                                 int32_t* __restrict__ perm) {
-    __shared__ int s_wcnt[kWarps][32];
+    // s_pos[w][e]: first the number of warp w's tokens on expert e, then warp w's
+    // next free position in expert e's segment. Lanes holding the same expert are
+    // grouped with __match_any_sync: a token's rank is the number of lower lanes
+    // in its group, and the group's lowest lane advances the position.
+    __shared__ int s_pos[kWarps][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    s_pos[warp][lane] = 0;
+    __syncwarp();
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokPerBlk + warp * kTokPerWarp;
     constexpr int IT = kTokPerWarp / 32;
+    const unsigned lt = (1u << lane) - 1u;
     int k[IT];
-    int cnt = 0;
 #pragma unroll
     for (int it = 0; it < IT; ++it) {
         const int64_t t = t0 + it * 32 + lane;
         k[it] = (t < T) ? expert_idx[t] : -1;
-        for (int e = 0; e < E; ++e) {
-            const int c = __popc(__ballot_sync(0xffffffffu, k[it] == e));
-            if (lane == e) cnt += c;
-        }
     }
-    s_wcnt[warp][lane] = cnt;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+        const unsigned same = __match_any_sync(0xffffffffu, k[it]);
+        if (k[it] >= 0 && (same & lt) == 0) s_pos[warp][k[it]] += __popc(same);
+        __syncwarp();
+    }
     __syncthreads();
-    // lane e: first free position of expert e for this warp
     int run = 0;
     if (lane < E) {
         run = blk_base[static_cast<int64_t>(blockIdx.x) * E + lane];
-        for (int w = 0; w < warp; ++w) run += s_wcnt[w][lane];
+        for (int w = 0; w < warp; ++w) run += s_pos[w][lane];
     }
-    const unsigned lt = (1u << lane) - 1u;
+    __syncthreads();
+    if (lane < E) s_pos[warp][lane] = run;
+    __syncwarp();
 #pragma unroll
     for (int it = 0; it < IT; ++it) {
         const int kk = k[it];
         const unsigned same = __match_any_sync(0xffffffffu, kk);
-        const int base = __shfl_sync(0xffffffffu, run, kk < 0 ? 0 : kk);
+        const int base = kk >= 0 ? s_pos[warp][kk] : 0;
         if (kk >= 0) perm[base + __popc(same & lt)] = static_cast<int32_t>(t0 + it * 32 + lane);
-        for (int e = 0; e < E; ++e) {
-            const int c = __popc(__ballot_sync(0xffffffffu, kk == e));
-            if (lane == e) run += c;
-        }
+        __syncwarp();
+        if (kk >= 0 && (same & lt) == 0) s_pos[warp][kk] = base + __popc(same);
+        __syncwarp();
     }
 }
 
@@ -225,7 +291,15 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
                          int32_t* offsets, int32_t* perm, int32_t* blk_counts, int32_t* blk_base,
                          cudaStream_t s) {
     const int64_t nblk = (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk;
-    if (E <= 4)
+    if (E == 4)
+        route_count_vec_kernel<4><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+    else if (E == 8)
+        route_count_vec_kernel<8><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+    else if (E == 16)
+        route_count_vec_kernel<16><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+    else if (E == 32)
+        route_count_vec_kernel<32><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+    else if (E <= 4)
         route_count_kernel<4><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
     else if (E <= 8)
         route_count_kernel<8><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
