@@ -27,7 +27,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 32;                                   // tokens a warp handles at a time
-constexpr int kChunksPerWarp = kAuxTokPerBlk / (kWarps * kChunk);  // 2
+constexpr int kChunksPerWarp = kAuxTokPerBlk / (kWarps * kChunk);  // 4
 
 // Shared-memory slot of float4 q (experts 4q..4q+3) of token row t when a row
 // holds Q = EMAX / 4 float4s: the XOR swizzle spreads the 8 rows read by one
@@ -40,9 +40,8 @@ __device__ __forceinline__ int row_slot(int t, int q) {
     return t * Q + (q ^ ((t >> SH) & (Q - 1)));
 }
 
-// One block per 512 consecutive tokens; warp w handles chunks w and w + 8 of 32
-// tokens (blocks small enough that several waves overlap one another's loads,
-// math and stores). The warp stages both chunks' logits in its own
+// One block per 1024 consecutive tokens; warp w handles chunks w, w + 8, w + 16,
+// w + 24 of 32 tokens. The warp stages all four chunks' logits in its own
 // shared buffer (128-bit loads, every load in flight before the first use, no
 // block barrier for the data), lane t computes token t of each chunk reading
 // its row as float4s, and the gradients go back out with 128-bit stores. When
@@ -329,7 +328,7 @@ cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float la
 }
 
 cudaError_t aux_set_smem_limits() {
-    // 8 warps x 2 chunks x 32 tokens x 32 experts x 4 bytes = 64 KiB for the widest instance
+    // 8 warps x 4 chunks x 32 tokens x 32 experts x 4 bytes = 128 KiB for the widest instance
     cudaError_t e = cudaFuncSetAttribute(aux_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(float) * kWarps * kChunksPerWarp * kChunk * 16));
     if (e != cudaSuccess) return e;

@@ -10,7 +10,7 @@ namespace moe {
 
 // Tokens handled by one block of the routing and aux kernels.
 constexpr int kRouteTokPerBlk = 1024;
-constexpr int kAuxTokPerBlk = 512;
+constexpr int kAuxTokPerBlk = 1024;
 
 // Weight-gradient contraction: the expert-sorted token list is cut into
 // `wgrad_splits(T)` equal ranges (further cut at expert boundaries); range c
