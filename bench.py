@@ -46,11 +46,24 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic(spec):
-    """Bytes and flops the method itself must move / compute for one step."""
-    T, E, H = spec.T, spec.E, spec.H
-    step_bytes = T * (4 * (5 * H + 3 * E) + 16) + 2 * E * H * H * 4
+def algorithmic(spec, grad: str = "token"):
+    """Bytes and flops the method itself must move / compute for one step.
+    grad = "mean_collapse": the output gradient arrives as [B, H] (the gradient
+    of the horizon mean) instead of [T, H]."""
+    T, E, H, B = spec.T, spec.E, spec.H, spec.B
     step_flops = 6 * H * H * T
+    if grad == "mean_collapse":
+        g_bytes = B * H * 4
+        step_bytes = T * (4 * (4 * H + 3 * E) + 16) + g_bytes + 2 * E * H * H * 4
+        per_kernel_bytes = {
+            "fwd": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
+            # grad_ctx_mean read once, d_x written, perm read; W
+            "d_x": T * (4 * H + 4) + g_bytes + E * H * H * 4,
+            # x and grad_ctx_mean read, perm read; dW and db written
+            "wgrad": T * (4 * H + 4) + g_bytes + E * H * H * 4 + E * H * 4,
+        }
+        return step_bytes, step_flops, per_kernel_bytes
+    step_bytes = T * (4 * (5 * H + 3 * E) + 16) + 2 * E * H * H * 4
     per_kernel_bytes = {
         # x read, routed written, perm read; W and bias
         "fwd": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
@@ -203,6 +216,8 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--grad", choices=["token", "mean_collapse"], default="token",
+                    help="output gradient per token [T, H] (default) or of the horizon mean [B, H]")
     args = ap.parse_args()
     spec = wl.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -230,7 +245,11 @@ def main():
     T, E, H = spec.T, spec.E, spec.H
     logits = torch.from_numpy(inp.gate_logits).to(dev)
     x = torch.from_numpy(inp.x).to(dev)
-    d_out = torch.from_numpy(inp.d_out).to(dev)
+    collapse = args.grad == "mean_collapse"
+    # the gradient of the horizon mean: one row per batch row (a seeded draw of its own)
+    g_host = (np.random.default_rng(spec.seed + 7).standard_normal((spec.B, spec.H), dtype=np.float32)
+              if collapse else inp.d_out)
+    d_out = torch.from_numpy(g_host).to(dev)
     W = torch.from_numpy(inp.W).to(dev)
     bias = torch.from_numpy(inp.bias).to(dev)
     gate = MoETop1Gate(W, bias, spec.B, spec.N_H, math_mode, inp.lambda_floor, inp.lambda_max_extra,
@@ -248,11 +267,12 @@ def main():
         gate.forward(x)
         if ev:
             ev[2].record(stream)
-        ops.moe_top1_bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, gate.d_x, None, None, 0,
+        bwd = ops.moe_top1_bwd_mean_collapse if collapse else ops.moe_top1_bwd
+        bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, gate.d_x, None, None, 0,
                          gate.ws)
         if ev:
             ev[3].record(stream)
-        ops.moe_top1_bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, None, gate.dW, gate.db, 0,
+        bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, None, gate.dW, gate.db, 0,
                          gate.ws)
         if ev:
             ev[4].record(stream)
@@ -293,7 +313,7 @@ def main():
     # end to end through the public API: inputs from pinned host memory, loss back to the host
     h_logits = torch.from_numpy(inp.gate_logits).pin_memory()
     h_x = torch.from_numpy(inp.x).pin_memory()
-    h_dout = torch.from_numpy(inp.d_out).pin_memory()
+    h_dout = torch.from_numpy(g_host).pin_memory()
     h_loss = torch.empty(2, dtype=torch.float32).pin_memory()
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
     barrier()
@@ -303,7 +323,14 @@ def main():
         logits.copy_(h_logits, non_blocking=True)
         x.copy_(h_x, non_blocking=True)
         d_out.copy_(h_dout, non_blocking=True)
-        gate.step(logits, x, d_out)
+        if collapse:
+            gate.route(logits)
+            gate.forward(x)
+            gate.backward_mean_collapse(x, d_out)
+            gate.aux(logits)
+            gate.update_lambda()
+        else:
+            gate.step(logits, x, d_out)
         h_loss.copy_(gate.loss, non_blocking=True)
     e1.record(stream)
     barrier()
@@ -311,7 +338,7 @@ def main():
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
-        step_bytes, step_flops, kbytes = algorithmic(spec)
+        step_bytes, step_flops, kbytes = algorithmic(spec, args.grad)
         hbm = float(peaks["hbm_gbs"])
         tf32_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * TF32_OVER_BF16
         t_roof = max(step_bytes / (hbm * 1e9), step_flops / (tf32_sus * 1e12))
@@ -322,11 +349,15 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": spec.name, "B": spec.B, "N_H": spec.N_H, "E": E, "H": H, "tokens": T,
+            "config": {"workload": spec.name + ("+mean_collapse_bwd" if collapse else ""), "B": spec.B,
+                       "N_H": spec.N_H, "E": E, "H": H, "tokens": T, "grad": args.grad,
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (x, d_out, routed, d_x: 4 x %.2f GB), no flush" % (T * H * 4 / 1e9)},
+                       "l2": ("inputs larger than L2 (x, routed, d_x: 3 x %.2f GB; the [B, H] gradient, %.0f MB, "
+                              "stays in L2), no flush" % (T * H * 4 / 1e9, spec.B * H * 4 / 1e6)) if collapse else
+                             ("inputs larger than L2 (x, d_out, routed, d_x: 4 x %.2f GB), no flush" % (T * H * 4 / 1e9))},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": recorded_traffic(dominant, spec.name, args.math),
+                         "frac": achieved / hbm,
+                         "traffic": None if collapse else recorded_traffic(dominant, spec.name, args.math),
                          "algorithmic_bytes": kbytes[dominant], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "flops": step_flops, "t_roofline_ms": t_roof * 1e3,
                               "frac": t_roof * 1e3 / ms_per_step,
@@ -334,7 +365,7 @@ def main():
                                         "source": f"{peak_kind}; tf32 = bf16_tflops_sustained x 1.1/2.25"}},
             "per_call_ms": call_ms,
             "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
-                    "h2d_bytes_per_step": T * (E + 2 * H) * 4, "d2h_bytes_per_step": 8},
+                    "h2d_bytes_per_step": (T * (E + H) + g_host.shape[0] * H) * 4, "d2h_bytes_per_step": 8},
             "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode),
             "clocks": clocks.summary(),
             "device_flags": flags,

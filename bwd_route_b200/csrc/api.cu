@@ -165,6 +165,83 @@ bool encode_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
+// Body of both backward entry points: token t's output gradient is
+// g_scale * d_out[t / g_div] (d_out has g_rows rows).
+moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_t g_rows, int g_div, float g_scale,
+                      const moe_routing_t* routing,
+                          int64_t B, int64_t N_H, int32_t E, int32_t H, moe_math_t math, float* d_x, float* dW,
+                          float* db, uint32_t accumulate_flags, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    int64_t T = 0;
+    moe_status_t st = tokens(B, N_H, &T);
+    if (st != MOE_OK) return st;
+    if (math != MOE_MATH_TF32 && math != MOE_MATH_FFMA) return MOE_ERR_INVALID_ARG;
+    if (accumulate_flags & ~(MOE_ACC_DX | MOE_ACC_DW | MOE_ACC_DB)) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || E > 32 || !h_supported(H, math)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!routing) return MOE_ERR_INVALID_ARG;
+    if (!d_x && !dW && !db) return MOE_OK;
+    if (T > 0 && (!d_out || !routing->offsets || !routing->perm)) return MOE_ERR_INVALID_ARG;
+    if (d_x && !W) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (dW || db) && !x) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(W, 16) || !aligned(d_out, 16) || !aligned(d_x, 16) || !aligned(dW, 16) ||
+        !aligned(db, 16))
+        return MOE_ERR_MISALIGNED;
+    const size_t act = sizeof(float) * T * H;
+    const size_t wbytes = sizeof(float) * E * H * H;
+    const Range outs[3] = {{d_x, act}, {dW, wbytes}, {db, sizeof(float) * E * H}};
+    const Range ins[6] = {{x, act},
+                          {W, wbytes},
+                          {d_out, sizeof(float) * static_cast<size_t>(g_rows) * H},
+                          {routing->offsets, sizeof(int32_t) * (E + 1)},
+                          {routing->perm, sizeof(int32_t) * T},
+                          {workspace, workspace ? workspace_bytes : 0}};
+    if (any_alias(outs, 3, ins, 6)) return MOE_ERR_ALIAS;
+    const WsLayout L = ws_layout(T, E, H);
+    const bool need_ws = (dW || db) || (d_x && math == MOE_MATH_TF32);  // TF32 d_x: the flag word
+    if (need_ws) {
+        if (!workspace) return MOE_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
+        if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int acc_dx = (accumulate_flags & MOE_ACC_DX) ? 1 : 0;
+    const int acc_dw = (accumulate_flags & MOE_ACC_DW) ? 1 : 0;
+    const int acc_db = (accumulate_flags & MOE_ACC_DB) ? 1 : 0;
+    if (T == 0) {
+        cudaError_t e = cudaSuccess;
+        if (dW && !acc_dw) e = cudaMemsetAsync(dW, 0, wbytes, s);
+        if (e == cudaSuccess && db && !acc_db) e = cudaMemsetAsync(db, 0, sizeof(float) * E * H, s);
+        return cuda_status(e);
+    }
+    DeviceInfo* dev = nullptr;
+    cudaError_t e = device_info(&dev);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
+    if (d_x) {
+        if (math == MOE_MATH_TF32) {
+            e = launch_grouped_tf32(d_out, W, nullptr, routing->offsets, routing->perm, T, E, H, 1, acc_dx, g_div,
+                                    g_scale, d_x, flags, dev->num_sms, s);
+        } else {
+            e = launch_grouped_ffma(d_out, W, nullptr, routing->offsets, routing->perm, T, E, H, 0, acc_dx, g_div,
+                                    g_scale, d_x, s);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (dW || db) {
+        float* part = reinterpret_cast<float*>(ws + L.wg_part);
+        float* part_db = reinterpret_cast<float*>(ws + L.wg_part_db);
+        if (math == MOE_MATH_TF32)
+            e = launch_wgrad_tf32(x, d_out, routing->offsets, routing->perm, T, E, H, g_div, part, part_db, flags, s);
+        else
+            e = launch_wgrad_ffma(x, d_out, routing->offsets, routing->perm, T, E, H, g_div, part, part_db, s);
+        if (e == cudaSuccess)
+            e = launch_wgrad_reduce(part, part_db, routing->offsets, T, E, H, g_scale, dW, db, acc_dw, acc_db, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -281,9 +358,9 @@ moe_status_t moe_top1_fwd(const float* x, const float* W, const float* bias, con
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (math == MOE_MATH_TF32)
-        return cuda_status(launch_grouped_tf32(x, W, bias, routing->offsets, routing->perm, T, E, H, 0, 0, routed,
+        return cuda_status(launch_grouped_tf32(x, W, bias, routing->offsets, routing->perm, T, E, H, 0, 0, 1, 1.0f, routed,
                                                static_cast<uint32_t*>(workspace), dev->num_sms, s));
-    return cuda_status(launch_grouped_ffma(x, W, bias, routing->offsets, routing->perm, T, E, H, 1, 0, routed, s));
+    return cuda_status(launch_grouped_ffma(x, W, bias, routing->offsets, routing->perm, T, E, H, 1, 0, 1, 1.0f, routed, s));
 }
 
 moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out, const moe_routing_t* routing,
@@ -293,70 +370,22 @@ moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out, co
     int64_t T = 0;
     moe_status_t st = tokens(B, N_H, &T);
     if (st != MOE_OK) return st;
-    if (math != MOE_MATH_TF32 && math != MOE_MATH_FFMA) return MOE_ERR_INVALID_ARG;
-    if (accumulate_flags & ~(MOE_ACC_DX | MOE_ACC_DW | MOE_ACC_DB)) return MOE_ERR_INVALID_ARG;
-    if (E < 1 || E > 32 || !h_supported(H, math)) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (!routing) return MOE_ERR_INVALID_ARG;
-    if (!d_x && !dW && !db) return MOE_OK;
-    if (T > 0 && (!d_out || !routing->offsets || !routing->perm)) return MOE_ERR_INVALID_ARG;
-    if (d_x && !W) return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (dW || db) && !x) return MOE_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(W, 16) || !aligned(d_out, 16) || !aligned(d_x, 16) || !aligned(dW, 16) ||
-        !aligned(db, 16))
-        return MOE_ERR_MISALIGNED;
-    const size_t act = sizeof(float) * T * H;
-    const size_t wbytes = sizeof(float) * E * H * H;
-    const Range outs[3] = {{d_x, act}, {dW, wbytes}, {db, sizeof(float) * E * H}};
-    const Range ins[6] = {{x, act},
-                          {W, wbytes},
-                          {d_out, act},
-                          {routing->offsets, sizeof(int32_t) * (E + 1)},
-                          {routing->perm, sizeof(int32_t) * T},
-                          {workspace, workspace ? workspace_bytes : 0}};
-    if (any_alias(outs, 3, ins, 6)) return MOE_ERR_ALIAS;
-    const WsLayout L = ws_layout(T, E, H);
-    const bool need_ws = (dW || db) || (d_x && math == MOE_MATH_TF32);  // TF32 d_x: the flag word
-    if (need_ws) {
-        if (!workspace) return MOE_ERR_WORKSPACE;
-        if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
-        if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
-    }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int acc_dx = (accumulate_flags & MOE_ACC_DX) ? 1 : 0;
-    const int acc_dw = (accumulate_flags & MOE_ACC_DW) ? 1 : 0;
-    const int acc_db = (accumulate_flags & MOE_ACC_DB) ? 1 : 0;
-    if (T == 0) {
-        cudaError_t e = cudaSuccess;
-        if (dW && !acc_dw) e = cudaMemsetAsync(dW, 0, wbytes, s);
-        if (e == cudaSuccess && db && !acc_db) e = cudaMemsetAsync(db, 0, sizeof(float) * E * H, s);
-        return cuda_status(e);
-    }
-    DeviceInfo* dev = nullptr;
-    cudaError_t e = device_info(&dev);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
-    if (d_x) {
-        if (math == MOE_MATH_TF32) {
-            e = launch_grouped_tf32(d_out, W, nullptr, routing->offsets, routing->perm, T, E, H, 1, acc_dx, d_x,
-                                    flags, dev->num_sms, s);
-        } else {
-            e = launch_grouped_ffma(d_out, W, nullptr, routing->offsets, routing->perm, T, E, H, 0, acc_dx, d_x, s);
-        }
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-    }
-    if (dW || db) {
-        float* part = reinterpret_cast<float*>(ws + L.wg_part);
-        float* part_db = reinterpret_cast<float*>(ws + L.wg_part_db);
-        if (math == MOE_MATH_TF32)
-            e = launch_wgrad_tf32(x, d_out, routing->offsets, routing->perm, T, E, H, part, part_db, flags, s);
-        else
-            e = launch_wgrad_ffma(x, d_out, routing->offsets, routing->perm, T, E, H, part, part_db, s);
-        if (e == cudaSuccess)
-            e = launch_wgrad_reduce(part, part_db, routing->offsets, T, E, H, dW, db, acc_dw, acc_db, s);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-    }
-    return MOE_OK;
+    return bwd_impl(x, W, d_out, T, 1, 1.0f, routing, B, N_H, E, H, math, d_x, dW, db, accumulate_flags, workspace,
+                    workspace_bytes, stream);
+}
+
+moe_status_t moe_top1_bwd_mean_collapse(const float* x, const float* W, const float* grad_ctx_mean,
+                                        const moe_routing_t* routing, int64_t B, int64_t N_H, int32_t E, int32_t H,
+                                        moe_math_t math, float* d_x, float* dW, float* db, uint32_t accumulate_flags,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+    int64_t T = 0;
+    moe_status_t st = tokens(B, N_H, &T);
+    if (st != MOE_OK) return st;
+    if (N_H > (int64_t{1} << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int g_div = T > 0 ? static_cast<int>(N_H) : 1;
+    const float g_scale = T > 0 ? static_cast<float>(1.0 / static_cast<double>(N_H)) : 1.0f;
+    return bwd_impl(x, W, grad_ctx_mean, B, g_div, g_scale, routing, B, N_H, E, H, math, d_x, dW, db,
+                    accumulate_flags, workspace, workspace_bytes, stream);
 }
 
 moe_status_t moe_aux_loss_fwd_bwd(const float* gate_logits, const int32_t* counts, int64_t B, int64_t N_H,

@@ -37,8 +37,8 @@ __global__ void __launch_bounds__(kGThreads) grouped_ffma_kernel(const float* __
                                                                 const float* __restrict__ bias,
                                                                 const int32_t* __restrict__ offsets,
                                                                 const int32_t* __restrict__ perm, int E, int H,
-                                                                int b_kmajor, int accumulate,
-                                                                float* __restrict__ out) {
+                                                                int b_kmajor, int accumulate, int src_div,
+                                                                float out_scale, float* __restrict__ out) {
     __shared__ int s_off[33];
     __shared__ int s_tstart[33];
     __shared__ int s_tok[kGBM];
@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(kGThreads) grouped_ffma_kernel(const float* __
             const int m = idx / 8, kq = idx % 8;
             const int tok = s_tok[m];
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (tok >= 0) v = __ldg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(tok) * H + k0) + kq);
+            if (tok >= 0)
+                v = __ldg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(tok / src_div) * H + k0) + kq);
             sA[kq * 4 + 0][m] = v.x;
             sA[kq * 4 + 1][m] = v.y;
             sA[kq * 4 + 2][m] = v.z;
@@ -121,7 +122,8 @@ __global__ void __launch_bounds__(kGThreads) grouped_ffma_kernel(const float* __
         const int m = tm * 4 + i;
         const int tok = s_tok[m];
         if (tok < 0) continue;
-        float4 v = make_float4(acc[i][0] + bvec.x, acc[i][1] + bvec.y, acc[i][2] + bvec.z, acc[i][3] + bvec.w);
+        float4 v = make_float4(acc[i][0] * out_scale + bvec.x, acc[i][1] * out_scale + bvec.y,
+                               acc[i][2] * out_scale + bvec.z, acc[i][3] * out_scale + bvec.w);
         float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(tok) * H + n0 + tn * 4);
         if (accumulate) {
             const float4 o = *dst;
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(kWThreads) wgrad_ffma_kernel(const float* __re
                                                               const float* __restrict__ d_out,
                                                               const int32_t* __restrict__ offsets,
                                                               const int32_t* __restrict__ perm, int64_t T, int E,
-                                                              int H, int P, float* __restrict__ part,
+                                                              int H, int P, int g_div, float* __restrict__ part,
                                                               float* __restrict__ part_db) {
     __shared__ __align__(16) float sG[kWChunk][kWT];  // d_out rows
     __shared__ __align__(16) float sX[kWChunk][kWT];  // x rows
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kWThreads) wgrad_ffma_kernel(const float* __re
                 const int tok = s_tok[r];
                 float4 g = make_float4(0.f, 0.f, 0.f, 0.f), v = g;
                 if (tok >= 0) {
-                    g = __ldg(reinterpret_cast<const float4*>(d_out + static_cast<int64_t>(tok) * H + o0) + q);
+                    g = __ldg(reinterpret_cast<const float4*>(d_out + static_cast<int64_t>(tok / g_div) * H + o0) + q);
                     v = __ldg(reinterpret_cast<const float4*>(x + static_cast<int64_t>(tok) * H + i0) + q);
                 }
                 *reinterpret_cast<float4*>(&sG[r][q * 4]) = g;
@@ -271,7 +273,7 @@ __device__ __forceinline__ float4 sum_slots(const float4* __restrict__ src, int6
 __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ part,
                                                           const float* __restrict__ part_db,
                                                           const int32_t* __restrict__ offsets, int64_t T, int E,
-                                                          int H, int P, float* __restrict__ dW,
+                                                          int H, int P, float scale, float* __restrict__ dW,
                                                           float* __restrict__ db, int acc_dw, int acc_db) {
     __shared__ int s_c[2];
     const int e = blockIdx.y;
@@ -301,6 +303,7 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
         if (j >= HH / 4) return;
         float4 r = sum_slots(reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c_lo) + e) * HH) + j,
                              HH / 4, c_hi - c_lo + 1);
+        r = make_float4(r.x * scale, r.y * scale, r.z * scale, r.w * scale);
         float4* dst = reinterpret_cast<float4*>(dW + e * HH) + j;
         if (acc_dw) {
             const float4 o = *dst;
@@ -313,6 +316,7 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
         if (j >= H / 4) return;
         float4 r = sum_slots(reinterpret_cast<const float4*>(part_db + (static_cast<int64_t>(c_lo) + e) * H) + j,
                              H / 4, c_hi - c_lo + 1);
+        r = make_float4(r.x * scale, r.y * scale, r.z * scale, r.w * scale);
         float4* dst = reinterpret_cast<float4*>(db + static_cast<int64_t>(e) * H) + j;
         if (acc_db) {
             const float4 o = *dst;
@@ -326,28 +330,30 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
 
 cudaError_t launch_grouped_ffma(const float* src, const float* Wsrc, const float* bias, const int32_t* offsets,
                                 const int32_t* perm, int64_t T, int E, int H, int b_kmajor, int accumulate,
-                                float* out, cudaStream_t s) {
+                                int src_div, float out_scale, float* out, cudaStream_t s) {
     const int64_t tiles = (T + kGBM - 1) / kGBM + E;  // upper bound; extra CTAs exit
     dim3 grid(static_cast<unsigned>(tiles), H / kGBN);
-    grouped_ffma_kernel<<<grid, kGThreads, 0, s>>>(src, Wsrc, bias, offsets, perm, E, H, b_kmajor, accumulate, out);
+    grouped_ffma_kernel<<<grid, kGThreads, 0, s>>>(src, Wsrc, bias, offsets, perm, E, H, b_kmajor, accumulate,
+                                                   src_div, out_scale, out);
     return cudaGetLastError();
 }
 
 cudaError_t launch_wgrad_ffma(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
-                              int64_t T, int E, int H, float* part, float* part_db, cudaStream_t s) {
+                              int64_t T, int E, int H, int g_div, float* part, float* part_db, cudaStream_t s) {
     const int P = wgrad_splits(T);
     dim3 grid(P, H / kWT, H / kWT);
-    wgrad_ffma_kernel<<<grid, kWThreads, 0, s>>>(x, d_out, offsets, perm, T, E, H, P, part, part_db);
+    wgrad_ffma_kernel<<<grid, kWThreads, 0, s>>>(x, d_out, offsets, perm, T, E, H, P, g_div, part, part_db);
     return cudaGetLastError();
 }
 
 cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const int32_t* offsets, int64_t T,
-                                int E, int H, float* dW, float* db, int acc_dw, int acc_db, cudaStream_t s) {
+                                int E, int H, float scale, float* dW, float* db, int acc_dw, int acc_db,
+                                cudaStream_t s) {
     const int P = wgrad_splits(T);
     const int64_t HH = static_cast<int64_t>(H) * H;
     const int nb_w = static_cast<int>((HH / 4 + 255) / 256);
     dim3 grid(nb_w + 1, E);
-    wgrad_reduce_kernel<<<grid, 256, 0, s>>>(part, part_db, offsets, T, E, H, P, dW, db, acc_dw, acc_db);
+    wgrad_reduce_kernel<<<grid, 256, 0, s>>>(part, part_db, offsets, T, E, H, P, scale, dW, db, acc_dw, acc_db);
     return cudaGetLastError();
 }
 

@@ -120,8 +120,8 @@ template <int H, bool B_MN>
 __global__ void __launch_bounds__(kThreadsGrouped, 1)
 grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUtensorMap tm_b,
                     const float* __restrict__ bias, const int32_t* __restrict__ offsets,
-                    const int32_t* __restrict__ perm, int E, int accumulate, float* __restrict__ out,
-                    uint32_t* __restrict__ dev_flags) {
+                    const int32_t* __restrict__ perm, int E, int accumulate, int src_div, float out_scale,
+                    float* __restrict__ out, uint32_t* __restrict__ dev_flags) {
     using C = GCfg<H>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -181,7 +181,7 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
                 const int r = it * 16 + prow;
-                t[it] = (r < nrows) ? perm[row0 + r] : -1;
+                t[it] = (r < nrows) ? perm[row0 + r] / src_div : -1;  // the source row of the token
             }
         };
         if (static_cast<int>(blockIdx.x) < ntiles) load_tokens(blockIdx.x, tok);
@@ -340,10 +340,10 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                                 float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(tok) * H + c0 +
                                                                         c * 32 + j * 4);
                                 float4 o = *dst;
-                                o.x += val.x + bv[c].x;
-                                o.y += val.y + bv[c].y;
-                                o.z += val.z + bv[c].z;
-                                o.w += val.w + bv[c].w;
+                                o.x += val.x * out_scale + bv[c].x;
+                                o.y += val.y * out_scale + bv[c].y;
+                                o.z += val.z * out_scale + bv[c].z;
+                                o.w += val.w * out_scale + bv[c].w;
                                 *dst = o;
                             }
                         }
@@ -355,10 +355,10 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                             const int R = it * 4 + (lane >> 3);
                             float4 val = ld_shared_v4(my_u32 + 4 * (R * 32 + ((j ^ (R & 7)) * 4)));
                             const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
-                            val.x += bv[c].x;
-                            val.y += bv[c].y;
-                            val.z += bv[c].z;
-                            val.w += bv[c].w;
+                            val.x = val.x * out_scale + bv[c].x;
+                            val.y = val.y * out_scale + bv[c].y;
+                            val.z = val.z * out_scale + bv[c].z;
+                            val.w = val.w * out_scale + bv[c].w;
                             st_global_cs_v4_pred(out + static_cast<int64_t>(tok < 0 ? 0 : tok) * H + c0 + c * 32 + j * 4,
                                                  val, tok >= 0);
                         }
@@ -405,7 +405,7 @@ template <int H>
 __global__ void __launch_bounds__(kThreads, 1)
 wgrad_tf32_kernel(const float* __restrict__ g_src, const float* __restrict__ x_src,
                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int T, int E, int P,
-                  float* __restrict__ part, float* __restrict__ part_db, uint32_t* __restrict__ dev_flags) {
+                  int g_div, float* __restrict__ part, float* __restrict__ part_db, uint32_t* __restrict__ dev_flags) {
     using C = WCfg<H>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -466,9 +466,11 @@ wgrad_tf32_kernel(const float* __restrict__ g_src, const float* __restrict__ x_s
                     const int r = it * ROWS_PER_PASS + rsub;
                     const int tk = __shfl_sync(0xffffffffu, tok_lane, r);
                     const uint32_t off = g * C::GROUP_BYTES + r * 128 + ((((q16 >> 1) ^ (r & 3)) << 5) | ((q16 & 1) << 4));
-                    const int64_t row = static_cast<int64_t>(tk < 0 ? 0 : tk) * H + g * 32 + q16 * 4;
+                    const int64_t col = g * 32 + q16 * 4;
+                    const int64_t row = static_cast<int64_t>(tk < 0 ? 0 : tk) * H + col;
+                    const int64_t grow = static_cast<int64_t>(tk < 0 ? 0 : tk / g_div) * H + col;  // gradient source row
                     const uint32_t nb = tk < 0 ? 0u : 16u;
-                    cp_async_16(base + off, g_src + row, nb);
+                    cp_async_16(base + off, g_src + grow, nb);
                     cp_async_16(base + C::OP_BYTES + off, x_src + row, nb);
                 }
                 cp_async_arrive_noinc(&ctl->full[stage]);
@@ -609,16 +611,17 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 template <int H, bool B_MN>
 cudaError_t launch_grouped_tf32_t(const float* src, const CUtensorMap& tm_b, const float* bias,
-                                  const int32_t* offsets, const int32_t* perm, int E, int accumulate, float* out,
-                                  uint32_t* dev_flags, int grid, cudaStream_t s) {
-    grouped_tf32_kernel<H, B_MN><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(src, tm_b, bias, offsets, perm, E,
-                                                                                  accumulate, out, dev_flags);
+                                  const int32_t* offsets, const int32_t* perm, int E, int accumulate, int src_div,
+                                  float out_scale, float* out, uint32_t* dev_flags, int grid, cudaStream_t s) {
+    grouped_tf32_kernel<H, B_MN><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(
+        src, tm_b, bias, offsets, perm, E, accumulate, src_div, out_scale, out, dev_flags);
     return cudaGetLastError();
 }
 
 cudaError_t launch_grouped_tf32(const float* src, const float* W, const float* bias, const int32_t* offsets,
                                 const int32_t* perm, int64_t T, int E, int H, int w_transposed, int accumulate,
-                                float* out, uint32_t* dev_flags, int num_sms, cudaStream_t s) {
+                                int src_div, float out_scale, float* out, uint32_t* dev_flags, int num_sms,
+                                cudaStream_t s) {
     CUtensorMap tm_b;
     const bool ok = w_transposed ? make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, 32, true)
                                  : make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, H);
@@ -626,27 +629,27 @@ cudaError_t launch_grouped_tf32(const float* src, const float* W, const float* b
     const int64_t tiles = (T + 127) / 128 + E;
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     if (H == 256)
-        return w_transposed ? launch_grouped_tf32_t<256, true>(src, tm_b, bias, offsets, perm, E, accumulate, out,
-                                                               dev_flags, grid, s)
-                            : launch_grouped_tf32_t<256, false>(src, tm_b, bias, offsets, perm, E, accumulate, out,
-                                                                dev_flags, grid, s);
-    return w_transposed ? launch_grouped_tf32_t<128, true>(src, tm_b, bias, offsets, perm, E, accumulate, out, dev_flags,
-                                                           grid, s)
-                        : launch_grouped_tf32_t<128, false>(src, tm_b, bias, offsets, perm, E, accumulate, out,
-                                                            dev_flags, grid, s);
+        return w_transposed ? launch_grouped_tf32_t<256, true>(src, tm_b, bias, offsets, perm, E, accumulate,
+                                                               src_div, out_scale, out, dev_flags, grid, s)
+                            : launch_grouped_tf32_t<256, false>(src, tm_b, bias, offsets, perm, E, accumulate,
+                                                                src_div, out_scale, out, dev_flags, grid, s);
+    return w_transposed ? launch_grouped_tf32_t<128, true>(src, tm_b, bias, offsets, perm, E, accumulate,
+                                                           src_div, out_scale, out, dev_flags, grid, s)
+                        : launch_grouped_tf32_t<128, false>(src, tm_b, bias, offsets, perm, E, accumulate,
+                                                            src_div, out_scale, out, dev_flags, grid, s);
 }
 
 cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
-                              int64_t T, int E, int H, float* part, float* part_db, uint32_t* dev_flags,
+                              int64_t T, int E, int H, int g_div, float* part, float* part_db, uint32_t* dev_flags,
                               cudaStream_t s) {
     const int P = wgrad_splits(T);
     if (H == 256) {
         wgrad_tf32_kernel<256><<<P, kThreads, WCfg<256>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
-                                                                         static_cast<int>(T), E, P, part, part_db,
+                                                                         static_cast<int>(T), E, P, g_div, part, part_db,
                                                                          dev_flags);
     } else {
         wgrad_tf32_kernel<128><<<P, kThreads, WCfg<128>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
-                                                                         static_cast<int>(T), E, P, part, part_db,
+                                                                         static_cast<int>(T), E, P, g_div, part, part_db,
                                                                          dev_flags);
     }
     return cudaGetLastError();

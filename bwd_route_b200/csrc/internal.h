@@ -82,29 +82,35 @@ cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, fl
 cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float lambda_max_extra, float ent_target,
                               float* lambda_eff, cudaStream_t s);
 
-// out[perm[r], n] = sum_k src[perm[r], k] * B_e[n, k] (+ bias[e, n]) for the
-// sorted rows r of expert e. b_kmajor = 1: B_e[n, k] = Wsrc[e][n][k] (forward);
+// out[perm[r], n] = out_scale * sum_k src[perm[r] / src_div, k] * B_e[n, k]
+// (+ bias[e, n]) for the sorted rows r of expert e (src_div = 1, out_scale = 1:
+// the plain contraction; src_div = N_H: every horizon token of a batch row reads
+// that row's gradient). b_kmajor = 1: B_e[n, k] = Wsrc[e][n][k] (forward);
 // b_kmajor = 0: B_e[n, k] = Wsrc[e][k][n] (input gradient).
 cudaError_t launch_grouped_ffma(const float* src, const float* Wsrc, const float* bias, const int32_t* offsets,
                                 const int32_t* perm, int64_t T, int E, int H, int b_kmajor, int accumulate,
-                                float* out, cudaStream_t s);
+                                int src_div, float out_scale, float* out, cudaStream_t s);
 
 // Same contraction on tcgen05 (TF32 in, FP32 accumulate), straight from W
 // [E][H][H]: w_transposed = 0: B_e[n, k] = W[e][n][k] (forward);
 // w_transposed = 1: B_e[n, k] = W[e][k][n] (input gradient).
 cudaError_t launch_grouped_tf32(const float* src, const float* W, const float* bias, const int32_t* offsets,
                                 const int32_t* perm, int64_t T, int E, int H, int w_transposed, int accumulate,
-                                float* out, uint32_t* dev_flags, int num_sms, cudaStream_t s);
+                                int src_div, float out_scale, float* out, uint32_t* dev_flags, int num_sms,
+                                cudaStream_t s);
 
-// Per-range partial sums of dW / db into the slot buffers (see wgrad_splits).
+// Per-range partial sums of dW / db into the slot buffers (see wgrad_splits);
+// token t's gradient row is d_out[t / g_div].
 cudaError_t launch_wgrad_ffma(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
-                              int64_t T, int E, int H, float* part, float* part_db, cudaStream_t s);
+                              int64_t T, int E, int H, int g_div, float* part, float* part_db, cudaStream_t s);
 cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t* offsets, const int32_t* perm,
-                              int64_t T, int E, int H, float* part, float* part_db, uint32_t* dev_flags,
+                              int64_t T, int E, int H, int g_div, float* part, float* part_db, uint32_t* dev_flags,
                               cudaStream_t s);
-// Fixed-order pairwise sum of the slots of each expert into dW / db (either may be null).
+// Fixed-order pairwise sum of the slots of each expert, times scale, into dW / db
+// (either may be null).
 cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const int32_t* offsets, int64_t T,
-                                int E, int H, float* dW, float* db, int acc_dw, int acc_db, cudaStream_t s);
+                                int E, int H, float scale, float* dW, float* db, int acc_dw, int acc_db,
+                                cudaStream_t s);
 
 // Driver entry point for tensor-map encoding (resolved at run time, so the
 // library does not link libcuda).

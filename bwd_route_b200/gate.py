@@ -64,6 +64,12 @@ class MoETop1Gate:
         ops.moe_top1_bwd(x, self.W, d_out, self.routing, self.B, self.N_H, self.E, self.H, self.math, self.d_x,
                          self.dW, self.db, 0, self.ws, stream)
 
+    def backward_mean_collapse(self, x, grad_ctx_mean, stream=None):
+        """Backward when the gate's output is averaged over the horizon axis:
+        grad_ctx_mean [B, H] is the gradient of that mean."""
+        ops.moe_top1_bwd_mean_collapse(x, self.W, grad_ctx_mean, self.routing, self.B, self.N_H, self.E, self.H,
+                                       self.math, self.d_x, self.dW, self.db, 0, self.ws, stream)
+
     def aux(self, gate_logits, stream=None):
         ops.moe_aux_loss_fwd_bwd(gate_logits, self.routing.counts, self.B, self.N_H, self.E, self.lambda_eff,
                                  self.d_logits, self.loss, self.mean_p, self.stats, self.ws, stream)

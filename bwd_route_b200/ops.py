@@ -29,7 +29,7 @@ EXPORTED = [
     "moe_top1_workspace_bytes", "moe_top1_workspace_init", "moe_top1_route", "moe_top1_fwd",
     "moe_top1_bwd", "moe_aux_loss_fwd_bwd", "moe_lambda_eff_update", "moe_top1_device_flags",
     "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc", "moe_top1_selftest_wait_timeout",
-    "moe_usage_entropy_ema_update",
+    "moe_usage_entropy_ema_update", "moe_top1_bwd_mean_collapse",
 ]
 MOE_NOALLOC_MAX_TOKENS = 2097152
 
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.moe_top1_bwd.restype = I32
         L.moe_top1_bwd.argtypes = [P, P, P, ctypes.POINTER(RoutingC), I64, I64, I32, I32, I32, P, P, P, U32,
                                    P, SZ, P]
+        L.moe_top1_bwd_mean_collapse.restype = I32
+        L.moe_top1_bwd_mean_collapse.argtypes = L.moe_top1_bwd.argtypes
         L.moe_aux_loss_fwd_bwd.restype = I32
         L.moe_aux_loss_fwd_bwd.argtypes = [P, P, I64, I64, I32, P, P, P, P, P, P, SZ, P]
         L.moe_lambda_eff_update.restype = I32
@@ -189,6 +191,17 @@ def moe_top1_bwd(x, W, d_out, routing: Routing, B: int, N_H: int, E: int, H: int
     _check("moe_top1_bwd", lib().moe_top1_bwd(_ptr(x, f), _ptr(W, f), _ptr(d_out, f), ctypes.byref(rc), B, N_H, E,
                                               H, math, _ptr(d_x, f), _ptr(dW, f), _ptr(db, f),
                                               accumulate_flags, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_top1_bwd_mean_collapse(x, W, grad_ctx_mean, routing: Routing, B: int, N_H: int, E: int, H: int, math: int,
+                               d_x, dW, db, accumulate_flags: int, ws: torch.Tensor, stream=None):
+    """moe_top1_bwd with d_out[b * N_H + h] = grad_ctx_mean[b] / N_H (grad_ctx_mean is [B, H])."""
+    rc = routing.c()
+    f = torch.float32
+    _check("moe_top1_bwd_mean_collapse",
+           lib().moe_top1_bwd_mean_collapse(_ptr(x, f), _ptr(W, f), _ptr(grad_ctx_mean, f), ctypes.byref(rc), B, N_H,
+                                            E, H, math, _ptr(d_x, f), _ptr(dW, f), _ptr(db, f), accumulate_flags,
+                                            _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def moe_aux_loss_fwd_bwd(gate_logits, counts, B: int, N_H: int, E: int, lambda_eff, d_logits, loss_out, mean_p,

@@ -171,6 +171,27 @@ moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out,
                           void* stream);
 
 /*
+ * Backward with the horizon mean-collapse folded in. [P5] MHA additions and the
+ * horizon_mean_collapse kernel: the MoE output [B, N_H, H] is averaged over the
+ * horizon axis into ctx_mean [B, H], so the gradient reaching token (b, h) is
+ * grad_ctx_mean[b, :] / N_H. This call is moe_top1_bwd with
+ *   d_out[b * N_H + h, :] = grad_ctx_mean[b, :] / N_H
+ * without that [T, H] array ever existing: the contraction kernels read row b of
+ * grad_ctx_mean [B, H] for every horizon token of batch row b, and the 1 / N_H
+ * is applied once to each result (exact when N_H is a power of two; otherwise
+ * within one rounding of the definition). Same arguments, outputs, flags,
+ * workspace and errors as moe_top1_bwd; grad_ctx_mean must not overlap any
+ * output. No counterpart of the forward half: a token's N_H horizon siblings go
+ * to different experts, so a fused forward collapse would need a cross-CTA sum
+ * that is not deterministic.
+ */
+moe_status_t moe_top1_bwd_mean_collapse(const float* x, const float* W, const float* grad_ctx_mean,
+                                        const moe_routing_t* routing, int64_t B, int64_t N_H, int32_t E,
+                                        int32_t H, moe_math_t math, float* d_x, float* dW, float* db,
+                                        uint32_t accumulate_flags, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
+/*
  * Load-balance auxiliary loss and its logit gradient. [P1] kernel list (a
  * softmax of the gate logits feeds a balance loss built from the usage
  * fraction, the mean probability and the expert count), ARCHITECTURE (the

@@ -130,6 +130,24 @@ def bwd_db(d_out, expert_idx, E: int):
     return db, sb
 
 
+def bwd_mean_collapse(x, W, grad_ctx_mean, expert_idx, N_H: int, E: int, tf32_mode: int = TF32_NONE,
+                      with_dw: bool = True):
+    """Backward of the gate followed by the horizon mean [B, N_H, H] -> [B, H]
+    ("Single source of truth for the attention path" page, MHA additions and the
+    horizon_mean_collapse kernel): every horizon token h of batch row b receives
+    grad_ctx_mean[b] / N_H. Computed as the plain backward on the broadcast rows
+    grad_ctx_mean[b] (the contraction's operand; TF32 mode rounds it), each
+    result divided by N_H in double.
+    -> dict d_x [T,H], and with_dw: dW, db, dW_scale, db_scale (float64)."""
+    g = _f32(grad_ctx_mean)
+    g_rep = np.repeat(g, int(N_H), axis=0)
+    out = {"d_x": bwd_dx(W, g_rep, expert_idx, tf32_mode) / N_H}
+    if with_dw:
+        dW, db, sW, sb = bwd_dw(x, g_rep, expert_idx, E, tf32_mode)
+        out.update(dW=dW / N_H, db=db / N_H, dW_scale=sW / N_H, db_scale=sb / N_H)
+    return out
+
+
 def bwd_dw_entries(x, d_out, expert_idx, e_list, o_list, i_list, tf32_mode: int = TF32_NONE):
     """dW at single entries (e, o, i) -> (values, scales), float64 [n]."""
     x, d_out, idx = _f32(x), _f32(d_out), _i32(expert_idx)

@@ -143,6 +143,21 @@ def test_aux_and_lambda_reject_bad_arguments(L):
     assert u(_p(A + 2), 0.01, 0.09, 1.0, out, None) == MISALIGNED
 
 
+def test_bwd_mean_collapse_rejects_bad_arguments(L):
+    b = L.moe_top1_bwd_mean_collapse
+    R = ops.RoutingC(_p(A + 0x100000), _p(A + 0x200000), _p(A + 0x300000), _p(A + 0x400000))
+    x, W, g = _p(A + 0x1000000), _p(A + 0x2000000), _p(A + 0x3000000)
+    dx, dW, db = _p(A + 0x4000000), _p(A + 0x5000000), _p(A + 0x6000000)
+    ws, wsb = _p(A + 0x40000000), 1 << 30
+    args = lambda **k: [k.get("x", x), W, k.get("g", g), ctypes.byref(R), 8, 5, 4, k.get("H", 128), 0,
+                        k.get("dx", dx), dW, db, 0, ws, wsb, None]
+    assert b(*args(H=100)) == SHAPE
+    assert b(*args(g=None)) == INVALID
+    assert b(*args(g=_p(A + 0x3000004))) == MISALIGNED
+    # d_x overlapping the last row of grad_ctx_mean [B, H] = 8 x 128 floats
+    assert b(*args(dx=_p(A + 0x3000000 + 4 * 128 * 7))) == ALIAS
+
+
 def test_usage_entropy_update_rejects_bad_arguments(L):
     u = L.moe_usage_entropy_ema_update
     cnt, ue, ee, hs = _p(A), _p(A + 0x100), _p(A + 0x200), _p(A + 0x300)

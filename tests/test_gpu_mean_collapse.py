@@ -1,0 +1,101 @@
+"""GPU parity of the backward with the horizon mean folded in
+(moe_top1_bwd_mean_collapse) against the oracle, in both math modes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bwd_route_b200 import ops
+from bwd_route_b200 import workloads as wl
+from gpu_harness import TOL, Guarded, assert_close, dev, tf32_mode
+
+pytestmark = pytest.mark.gpu
+
+MATHS = [ops.MOE_MATH_FFMA, ops.MOE_MATH_TF32]
+MATH_ID = {ops.MOE_MATH_FFMA: "ffma", ops.MOE_MATH_TF32: "tf32"}
+
+SPECS = [
+    wl.make_spec("mc_b8_h5_e4_h128", 8, 5, 4, 128, 31),            # N_H not a power of two
+    wl.make_spec("mc_b1024_h5_e4_h128", 1024, 5, 4, 128, 32),
+    wl.make_spec("mc_b300_h1_e3_h128", 300, 1, 3, 128, 33),         # N_H = 1: the plain backward
+    wl.make_spec("mc_b777_h3_e8_h256", 777, 3, 8, 256, 34),
+    wl.make_spec("mc_b2048_h16_e8_h256", 2048, 16, 8, 256, 35),     # the throughput shape's N_H, 32k tokens
+    wl.make_spec("mc_b700_h7_e32_h128", 700, 7, 32, 128, 36, skew_expert=3, skew_value=1.5),
+]
+
+
+def _run(inp, g_host, math, acc_flags=0, preset=None):
+    s = inp.spec
+    B, N_H, E, H, T = s.B, s.N_H, s.E, s.H, s.T
+    out = {k: Guarded(n, shape=sh) for k, n, sh in
+           [("d_x", T * H, (T, H)), ("dW", E * H * H, (E, H, H)), ("db", E * H, (E, H))]}
+    if preset:
+        for k, v in preset.items():
+            out[k].t.copy_(dev(v).view_as(out[k].t))
+    r = ops.Routing.empty(T, E, "cuda")
+    ws = ops.new_workspace(T, E, H, "cuda")
+    ops.moe_top1_route(dev(inp.gate_logits), B, N_H, E, r, ws)
+    ops.moe_top1_bwd_mean_collapse(dev(inp.x), dev(inp.W), dev(g_host), r, B, N_H, E, H, math, out["d_x"].t,
+                                   out["dW"].t, out["db"].t, acc_flags, ws)
+    torch.cuda.synchronize()
+    assert ops.moe_top1_device_flags(ws) == 0
+    assert all(v.guards_intact() for v in out.values())
+    return {k: v.host() for k, v in out.items()}
+
+
+def _grad(spec):
+    rng = np.random.default_rng(spec.seed + 1000)
+    return rng.standard_normal((spec.B, spec.H)).astype(np.float32)
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+@pytest.mark.parametrize("spec", SPECS, ids=lambda s: s.name)
+def test_mean_collapse_backward_parity(spec, math_mode):
+    inp = wl.generate(spec)
+    g = _grad(spec)
+    got = _run(inp, g, math_mode)
+    idx = oracle.route(inp.gate_logits)[0]
+    want = oracle.bwd_mean_collapse(inp.x, inp.W, g, idx, spec.N_H, spec.E, tf32_mode(math_mode))
+    atol, rtol = TOL[math_mode]
+    assert_close("d_x", got["d_x"], want["d_x"], atol, rtol)
+    assert_close("dW", got["dW"], want["dW"], atol, rtol, scale=want["dW_scale"])
+    assert_close("db", got["db"], want["db"], atol, rtol, scale=want["db_scale"])
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_mean_collapse_matches_plain_backward_bitwise_for_power_of_two_horizons(math_mode):
+    """With N_H = 16, g / N_H is exact, so the two entry points must agree bit for
+    bit: the same kernels, only the gradient rows and the final scale differ."""
+    spec = wl.make_spec("mc_eq_b512_h16_e8_h256", 512, 16, 8, 256, 37)
+    inp = wl.generate(spec)
+    g = _grad(spec)
+    got = _run(inp, g, math_mode)
+    d_out = np.repeat(g / np.float32(spec.N_H), spec.N_H, axis=0).astype(np.float32)
+    s = spec
+    r = ops.Routing.empty(s.T, s.E, "cuda")
+    ws = ops.new_workspace(s.T, s.E, s.H, "cuda")
+    ops.moe_top1_route(dev(inp.gate_logits), s.B, s.N_H, s.E, r, ws)
+    d_x = torch.empty(s.T, s.H, device="cuda")
+    dW = torch.empty(s.E, s.H, s.H, device="cuda")
+    db = torch.empty(s.E, s.H, device="cuda")
+    ops.moe_top1_bwd(dev(inp.x), dev(inp.W), dev(d_out), r, s.B, s.N_H, s.E, s.H, math_mode, d_x, dW, db, 0, ws)
+    torch.cuda.synchronize()
+    assert got["d_x"].tobytes() == d_x.cpu().numpy().tobytes()
+    assert got["dW"].tobytes() == dW.cpu().numpy().tobytes()
+    assert got["db"].tobytes() == db.cpu().numpy().tobytes()
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_mean_collapse_accumulate_flags(math_mode):
+    spec = wl.make_spec("mc_acc_b200_h5_e4_h256", 200, 5, 4, 256, 38)
+    inp = wl.generate(spec)
+    g = _grad(spec)
+    rng = np.random.default_rng(1)
+    T, E, H = spec.T, spec.E, spec.H
+    pre = {"d_x": rng.standard_normal((T, H)).astype(np.float32),
+           "dW": rng.standard_normal((E, H, H)).astype(np.float32),
+           "db": rng.standard_normal((E, H)).astype(np.float32)}
+    plain = _run(inp, g, math_mode)
+    acc = _run(inp, g, math_mode, acc_flags=ops.MOE_ACC_DX | ops.MOE_ACC_DW | ops.MOE_ACC_DB, preset=pre)
+    for k in ("d_x", "dW", "db"):
+        np.testing.assert_array_equal(acc[k], (pre[k] + plain[k]).astype(np.float32), err_msg=k)

@@ -494,3 +494,66 @@ def test_usage_entropy_no_tokens_is_no_observation():
     u, e, h = oracle.usage_entropy_ema(np.zeros(2, np.int32), 0, 0.5, False, u0, 0.3)
     np.testing.assert_array_equal(u, u0)
     assert e == 0.3 and h == 0.0
+
+
+# --------------------------------------------------------------------------- backward through the horizon mean
+
+def _collapse_case(B=3, N_H=4, E=3, H=32, seed=11):
+    rng = np.random.default_rng(seed)
+    T = B * N_H
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    W = (rng.standard_normal((E, H, H)) / np.sqrt(H)).astype(np.float32)
+    bias = (0.1 * rng.standard_normal((E, H))).astype(np.float32)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    g = rng.standard_normal((B, H)).astype(np.float32)
+    idx = oracle.route(logits)[0]
+    return x, W, bias, g, idx, B, N_H, E, H
+
+
+def _collapsed_loss(x, W, bias, g, idx, B, N_H):
+    """L = sum_b g[b] . mean_h routed[b, h] in float64, straight from the definitions."""
+    xd, Wd, bd = x.astype(np.float64), W.astype(np.float64), bias.astype(np.float64)
+    routed = np.einsum("toi,ti->to", Wd[idx], xd) + bd[idx]
+    ctx_mean = routed.reshape(B, N_H, -1).mean(axis=1)
+    return float((g.astype(np.float64) * ctx_mean).sum())
+
+
+def test_bwd_mean_collapse_finite_differences():
+    x, W, bias, g, idx, B, N_H, E, H = _collapse_case()
+    got = oracle.bwd_mean_collapse(x, W, g, idx, N_H, E)
+    eps = 1e-3
+    rng = np.random.default_rng(3)
+    for _ in range(6):                                    # d_x entries
+        t, i = rng.integers(0, B * N_H), rng.integers(0, H)
+        xp, xm = x.astype(np.float64).copy(), x.astype(np.float64).copy()
+        xp[t, i] += eps
+        xm[t, i] -= eps
+        fd = (_collapsed_loss(xp, W, bias, g, idx, B, N_H) - _collapsed_loss(xm, W, bias, g, idx, B, N_H)) / (2 * eps)
+        assert abs(got["d_x"][t, i] - fd) <= 1e-8 * max(1.0, abs(fd)), (t, i)
+    for _ in range(6):                                    # dW entries, including untouched experts
+        e, o, i = rng.integers(0, E), rng.integers(0, H), rng.integers(0, H)
+        Wp, Wm = W.astype(np.float64).copy(), W.astype(np.float64).copy()
+        Wp[e, o, i] += eps
+        Wm[e, o, i] -= eps
+        fd = (_collapsed_loss(x, Wp, bias, g, idx, B, N_H) - _collapsed_loss(x, Wm, bias, g, idx, B, N_H)) / (2 * eps)
+        assert abs(got["dW"][e, o, i] - fd) <= 1e-8 * max(1.0, abs(fd)), (e, o, i)
+    for e in range(E):                                    # db: the mean of g over each expert's tokens' rows
+        o = rng.integers(0, H)
+        bp, bm = bias.astype(np.float64).copy(), bias.astype(np.float64).copy()
+        bp[e, o] += eps
+        bm[e, o] -= eps
+        fd = (_collapsed_loss(x, W, bp, g, idx, B, N_H) - _collapsed_loss(x, W, bm, g, idx, B, N_H)) / (2 * eps)
+        assert abs(got["db"][e, o] - fd) <= 1e-8 * max(1.0, abs(fd)), (e, o)
+
+
+def test_bwd_mean_collapse_equals_plain_backward_on_the_broadcast_gradient():
+    """With N_H a power of two, g / N_H is exact in fp32, so the collapsed backward
+    must equal the (separately pinned) plain backward fed d_out = g[b] / N_H."""
+    x, W, bias, g, idx, B, N_H, E, H = _collapse_case(N_H=8)
+    d_out = np.repeat(g / np.float32(N_H), N_H, axis=0).astype(np.float32)
+    for mode in (oracle.TF32_NONE, oracle.TF32_RZ):
+        got = oracle.bwd_mean_collapse(x, W, g, idx, N_H, E, mode)
+        np.testing.assert_allclose(got["d_x"], oracle.bwd_dx(W, d_out, idx, mode), rtol=1e-15, atol=1e-15)
+        dW, db, _, _ = oracle.bwd_dw(x, d_out, idx, E, mode)
+        np.testing.assert_allclose(got["dW"], dW, rtol=1e-15, atol=1e-15)
+        np.testing.assert_allclose(got["db"], db, rtol=1e-15, atol=1e-15)
