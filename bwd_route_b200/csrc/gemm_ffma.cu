@@ -36,8 +36,8 @@ __global__ void __launch_bounds__(kGThreads) grouped_ffma_kernel(const float* __
                                                                 const float* __restrict__ Wsrc,
                                                                 const float* __restrict__ bias,
                                                                 const int32_t* __restrict__ offsets,
-                                                                const int32_t* __restrict__ perm, int E, int H,
-                                                                int b_kmajor, int accumulate, int src_div,
+                                                                const int32_t* __restrict__ perm, int E,
+                                                                int H, int b_kmajor, int accumulate, int src_div,
                                                                 float out_scale, float* __restrict__ out) {
     __shared__ int s_off[33];
     __shared__ int s_tstart[33];
@@ -80,7 +80,8 @@ __global__ void __launch_bounds__(kGThreads) grouped_ffma_kernel(const float* __
             const int tok = s_tok[m];
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (tok >= 0)
-                v = __ldg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(tok / src_div) * H + k0) + kq);
+                v = __ldg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(src_div == 1 ? tok : tok / src_div) * H +
+                                                          k0) + kq);
             sA[kq * 4 + 0][m] = v.x;
             sA[kq * 4 + 1][m] = v.y;
             sA[kq * 4 + 2][m] = v.z;
@@ -175,7 +176,8 @@ __global__ void __launch_bounds__(kWThreads) wgrad_ffma_kernel(const float* __re
                 const int tok = s_tok[r];
                 float4 g = make_float4(0.f, 0.f, 0.f, 0.f), v = g;
                 if (tok >= 0) {
-                    g = __ldg(reinterpret_cast<const float4*>(d_out + static_cast<int64_t>(tok / g_div) * H + o0) + q);
+                    g = __ldg(reinterpret_cast<const float4*>(d_out + static_cast<int64_t>(g_div == 1 ? tok : tok / g_div) * H +
+                                                              o0) + q);
                     v = __ldg(reinterpret_cast<const float4*>(x + static_cast<int64_t>(tok) * H + i0) + q);
                 }
                 *reinterpret_cast<float4*>(&sG[r][q * 4]) = g;

@@ -116,7 +116,10 @@ __device__ __forceinline__ int find_expert(const int* tstart, int E, int tile) {
 // the forward). B_MN = true: it is read MN-major straight from W (B_e[n][k] =
 // W[e][k][n], the input gradient), in 32-row x 128-byte boxes with the 32-byte
 // granule swizzle that tcgen05 requires for an MN-major TF32 operand.
-template <int H, bool B_MN>
+// COLLAPSE: token t's source row is t / src_div and each result is multiplied
+// by out_scale (the backward through the horizon mean); without it both are 1
+// and the code is the plain contraction's.
+template <int H, bool B_MN, bool COLLAPSE>
 __global__ void __launch_bounds__(kThreadsGrouped, 1)
 grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUtensorMap tm_b,
                     const float* __restrict__ bias, const int32_t* __restrict__ offsets,
@@ -181,7 +184,8 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
                 const int r = it * 16 + prow;
-                t[it] = (r < nrows) ? perm[row0 + r] / src_div : -1;  // the source row of the token
+                const int tk = (r < nrows) ? perm[row0 + r] : -1;
+                t[it] = (COLLAPSE && tk >= 0) ? tk / src_div : tk;  // the token's source row
             }
         };
         if (static_cast<int>(blockIdx.x) < ntiles) load_tokens(blockIdx.x, tok);
@@ -322,6 +326,10 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                 float v[64];
                 tmem_ld_32x32b_x64(tmem + (static_cast<uint32_t>(32 * q) << 16) +
                                        static_cast<uint32_t>(acc * H + c0 + cc * 64), v);
+                if (COLLAPSE) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) v[i] *= out_scale;
+                }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int c = cc * 2 + h;  // 32-column chunk within the half
@@ -340,10 +348,10 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                                 float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(tok) * H + c0 +
                                                                         c * 32 + j * 4);
                                 float4 o = *dst;
-                                o.x += val.x * out_scale + bv[c].x;
-                                o.y += val.y * out_scale + bv[c].y;
-                                o.z += val.z * out_scale + bv[c].z;
-                                o.w += val.w * out_scale + bv[c].w;
+                                o.x += val.x + bv[c].x;
+                                o.y += val.y + bv[c].y;
+                                o.z += val.z + bv[c].z;
+                                o.w += val.w + bv[c].w;
                                 *dst = o;
                             }
                         }
@@ -355,10 +363,10 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                             const int R = it * 4 + (lane >> 3);
                             float4 val = ld_shared_v4(my_u32 + 4 * (R * 32 + ((j ^ (R & 7)) * 4)));
                             const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
-                            val.x = val.x * out_scale + bv[c].x;
-                            val.y = val.y * out_scale + bv[c].y;
-                            val.z = val.z * out_scale + bv[c].z;
-                            val.w = val.w * out_scale + bv[c].w;
+                            val.x += bv[c].x;
+                            val.y += bv[c].y;
+                            val.z += bv[c].z;
+                            val.w += bv[c].w;
                             st_global_cs_v4_pred(out + static_cast<int64_t>(tok < 0 ? 0 : tok) * H + c0 + c * 32 + j * 4,
                                                  val, tok >= 0);
                         }
@@ -457,6 +465,8 @@ wgrad_tf32_kernel(const float* __restrict__ g_src, const float* __restrict__ x_s
             const int s = max(lo, ctl->off[e]), t = min(hi, ctl->off[e + 1]);
             for (int p0 = s; p0 < t; p0 += C::KT) {
                 int tok_lane = (p0 + lane >= t) ? -1 : (p0 == next_p0) ? next_lane : perm[p0 + lane];
+                // the lane's gradient row, one division per lane and stage (none for g_div = 1)
+                const int gtok_lane = (g_div == 1 || tok_lane < 0) ? tok_lane : tok_lane / g_div;
                 next_p0 = (p0 + C::KT < t) ? p0 + C::KT : t;
                 next_lane = (next_p0 + lane < hi) ? perm[next_p0 + lane] : -1;
                 if (!(ok = mbar_wait(&ctl->empty[stage], phase ^ 1, abort, dev_flags))) break;
@@ -465,10 +475,11 @@ wgrad_tf32_kernel(const float* __restrict__ g_src, const float* __restrict__ x_s
                 for (int it = 0; it < C::PER_THREAD; ++it) {
                     const int r = it * ROWS_PER_PASS + rsub;
                     const int tk = __shfl_sync(0xffffffffu, tok_lane, r);
+                    const int gtk = __shfl_sync(0xffffffffu, gtok_lane, r);
                     const uint32_t off = g * C::GROUP_BYTES + r * 128 + ((((q16 >> 1) ^ (r & 3)) << 5) | ((q16 & 1) << 4));
                     const int64_t col = g * 32 + q16 * 4;
                     const int64_t row = static_cast<int64_t>(tk < 0 ? 0 : tk) * H + col;
-                    const int64_t grow = static_cast<int64_t>(tk < 0 ? 0 : tk / g_div) * H + col;  // gradient source row
+                    const int64_t grow = static_cast<int64_t>(tk < 0 ? 0 : gtk) * H + col;  // gradient source row
                     const uint32_t nb = tk < 0 ? 0u : 16u;
                     cp_async_16(base + off, g_src + grow, nb);
                     cp_async_16(base + C::OP_BYTES + off, x_src + row, nb);
@@ -613,8 +624,12 @@ template <int H, bool B_MN>
 cudaError_t launch_grouped_tf32_t(const float* src, const CUtensorMap& tm_b, const float* bias,
                                   const int32_t* offsets, const int32_t* perm, int E, int accumulate, int src_div,
                                   float out_scale, float* out, uint32_t* dev_flags, int grid, cudaStream_t s) {
-    grouped_tf32_kernel<H, B_MN><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(
-        src, tm_b, bias, offsets, perm, E, accumulate, src_div, out_scale, out, dev_flags);
+    if (src_div != 1 || out_scale != 1.0f)
+        grouped_tf32_kernel<H, B_MN, true><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(
+            src, tm_b, bias, offsets, perm, E, accumulate, src_div, out_scale, out, dev_flags);
+    else
+        grouped_tf32_kernel<H, B_MN, false><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(
+            src, tm_b, bias, offsets, perm, E, accumulate, 1, 1.0f, out, dev_flags);
     return cudaGetLastError();
 }
 
@@ -658,10 +673,14 @@ cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t*
 // The dynamic shared-memory limits of every tcgen05 kernel, set once per device
 // (before the first launch there) instead of at every launch.
 cudaError_t tf32_set_smem_limits() {
-    cudaError_t e = set_smem(grouped_tf32_kernel<256, false>, GCfg<256>::SMEM_BYTES);
-    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<256, true>, GCfg<256>::SMEM_BYTES);
-    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, false>, GCfg<128>::SMEM_BYTES);
-    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, true>, GCfg<128>::SMEM_BYTES);
+    cudaError_t e = set_smem(grouped_tf32_kernel<256, false, false>, GCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<256, true, false>, GCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<256, false, true>, GCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<256, true, true>, GCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, false, false>, GCfg<128>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, true, false>, GCfg<128>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, false, true>, GCfg<128>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(grouped_tf32_kernel<128, true, true>, GCfg<128>::SMEM_BYTES);
     if (e == cudaSuccess) e = set_smem(wgrad_tf32_kernel<256>, WCfg<256>::SMEM_BYTES);
     if (e == cudaSuccess) e = set_smem(wgrad_tf32_kernel<128>, WCfg<128>::SMEM_BYTES);
     return e;

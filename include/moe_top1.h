@@ -74,7 +74,13 @@ typedef enum {
 /* Bits of the device flag word. */
 #define MOE_FLAG_WAIT_TIMEOUT 0x1u  /* a pipeline wait ran past its bound */
 
-/* Routing result: caller-owned device buffers. */
+/* Routing result: caller-owned device buffers. The forward, backward and aux
+ * entry points take a routing as an input and trust it: it must be what
+ * moe_top1_route (or moe_top1_route_noalloc) wrote for the same tokens. The
+ * contraction kernels index activations with offsets and perm without checking
+ * them again (a check per token costs about 5 % of their time), so a routing
+ * from anywhere else -- an uninitialised buffer, another batch -- can make them
+ * read and write outside the arrays. */
 typedef struct {
     int32_t* expert_idx; /* [T]     selected expert of each token */
     int32_t* counts;     /* [E]     tokens routed to each expert */
