@@ -75,6 +75,50 @@ def algorithmic(spec, grad: str = "token"):
     return step_bytes, step_flops, per_kernel_bytes
 
 
+L2_BYTES = 126 * 1024 * 1024
+# FP32 SIMT peak of the FFMA path: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz (nominal)
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def l2_note(spec, collapse: bool, flushed: bool) -> str:
+    T, H, E, B = spec.T, spec.H, spec.E, spec.B
+    act = T * H * 4
+    if act * 2 > L2_BYTES:
+        if collapse:
+            return ("inputs larger than L2 (x, routed, d_x: 3 x %.2f GB; the [B, H] gradient, %.0f MB, stays in "
+                    "L2)%s" % (act / 1e9, B * H * 4 / 1e6, ", L2 also flushed between steps" if flushed else ", no flush"))
+        return "inputs larger than L2 (x, d_out, routed, d_x: 4 x %.2f GB)%s" % (
+            act / 1e9, ", L2 also flushed between steps" if flushed else ", no flush")
+    total = 4 * act + T * E * 8 + 2 * E * H * H * 4
+    if flushed:
+        return "inputs (%.1f MB) fit in L2; 256 MB written between steps to flush it" % (total / 1e6)
+    return "inputs (%.1f MB) fit in L2 and stay there (back-to-back steps)" % (total / 1e6)
+
+
+def simt_roofline(step_flops: float, ms_per_step: float) -> dict:
+    """The FFMA path against its own ceiling, FP32 on the CUDA cores."""
+    achieved = step_flops / (ms_per_step * 1e-3) / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
+            "frac": achieved / FP32_SIMT_TFLOPS, "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}
+
+
+def host_cpu() -> dict:
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = os.cpu_count()
+    return {"cpu_model": model, "cores_available": avail}
+
+
 TRAFFIC_RECORD = os.path.join(HERE, "profiles", "launch_list_large_b65536_e8_h256.md")
 
 
@@ -200,7 +244,7 @@ def run_reference(args, spec):
                    "tokens": spec.T, "math": "fp64 oracle"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"first {sample_tokens} tokens of {spec.name} per step (route, forward, "
-                                   f"d_x, dW/db, aux) in plain single-threaded C, fp64 accumulation"},
+                                   f"d_x, dW/db, aux) in plain single-threaded C, fp64 accumulation", **host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -218,6 +262,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--grad", choices=["token", "mean_collapse"], default="token",
                     help="output gradient per token [T, H] (default) or of the horizon mean [B, H]")
+    ap.add_argument("--graph", action="store_true",
+                    help="time K replays of one step captured in a CUDA graph (the per-call times then come "
+                         "from a separate un-captured loop); for launch-bound small workloads")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 256 MB buffer between timed steps (outside each step's events)")
     args = ap.parse_args()
     spec = wl.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -294,19 +343,48 @@ def main():
         raise RuntimeError(f"device flags set during warm-up: {flags:#x}")
 
     # timed region: K whole steps, events on the launching stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
     per_call = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph = None
+    if args.graph:
+        # one step through the same public calls, captured once
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        graph.replay()
+        torch.cuda.synchronize(dev)
     barrier()
     with ClockSampler(local) as clocks:
         start.record(stream)
         for k in range(args.steps):
-            step(per_call[k])
+            if flush is not None:
+                flush.fill_(k & 0xFF)
+            if graph is not None:
+                per_call[k][0].record(stream)
+                graph.replay()
+                per_call[k][5].record(stream)
+            else:
+                step(per_call[k])
         end.record(stream)
         barrier()
-    ms = max_over_ranks(start.elapsed_time(end), dev)
+    step_ms = sorted(per_call[k][0].elapsed_time(per_call[k][5]) for k in range(args.steps))
+    if flush is not None:  # the flushes sit between the steps' own events
+        ms = sum(step_ms)
+    else:
+        ms = start.elapsed_time(end)
+    ms = max_over_ranks(ms, dev)
     ms_per_step = ms / args.steps
+    pct = lambda f: step_ms[min(len(step_ms) - 1, int(f * len(step_ms)))]  # noqa: E731
     names = ["route", "fwd", "d_x", "wgrad", "aux+lambda"]
-    call_ms = {n: sum(per_call[k][i].elapsed_time(per_call[k][i + 1]) for k in range(args.steps)) / args.steps
+    if graph is not None:
+        # per-call times from a separate un-captured loop
+        per_call = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(min(args.steps, 20))]
+        for ev in per_call:
+            step(ev)
+        torch.cuda.synchronize(dev)
+    call_ms = {n: sum(ev[i].elapsed_time(ev[i + 1]) for ev in per_call) / len(per_call)
                for i, n in enumerate(names)}
     flags = ops.moe_top1_device_flags(gate.ws)
 
@@ -352,9 +430,7 @@ def main():
             "config": {"workload": spec.name + ("+mean_collapse_bwd" if collapse else ""), "B": spec.B,
                        "N_H": spec.N_H, "E": E, "H": H, "tokens": T, "grad": args.grad,
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
-                       "l2": ("inputs larger than L2 (x, routed, d_x: 3 x %.2f GB; the [B, H] gradient, %.0f MB, "
-                              "stays in L2), no flush" % (T * H * 4 / 1e9, spec.B * H * 4 / 1e6)) if collapse else
-                             ("inputs larger than L2 (x, d_out, routed, d_x: 4 x %.2f GB), no flush" % (T * H * 4 / 1e9))},
+                       "l2": l2_note(spec, collapse, flush is not None)},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm,
                          "traffic": None if collapse else recorded_traffic(dominant, spec.name, args.math),
@@ -364,6 +440,10 @@ def main():
                               "peaks": {"hbm_gbs": hbm, "tf32_tflops": tf32_sus,
                                         "source": f"{peak_kind}; tf32 = bf16_tflops_sustained x 1.1/2.25"}},
             "per_call_ms": call_ms,
+            **({"simt_roofline": simt_roofline(step_flops, ms_per_step)} if math_mode == ops.MOE_MATH_FFMA else {}),
+            "step_ms_percentiles": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9)},
+            "timing": ("CUDA graph of one step, replayed" if graph is not None else "stream launches")
+                      + ("; 256 MB written between steps, outside their events" if flush is not None else ""),
             "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
                     "h2d_bytes_per_step": (T * (E + H) + g_host.shape[0] * H) * 4, "d2h_bytes_per_step": 8},
             "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode),
@@ -374,7 +454,8 @@ def main():
             v, dt, n = cpu_oracle_tokens_per_s(inp, CPU_SAMPLE_TOKENS)
             line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                                     "sample": f"first {n} tokens of {spec.name}: route, forward, d_x, dW/db and "
-                                              f"aux in plain single-threaded C (fp64 accumulation), {dt:.1f} s"}
+                                              f"aux in plain single-threaded C (fp64 accumulation), {dt:.1f} s",
+                                    **host_cpu()}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
