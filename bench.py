@@ -303,6 +303,9 @@ def main():
     bias = torch.from_numpy(inp.bias).to(dev)
     gate = MoETop1Gate(W, bias, spec.B, spec.N_H, math_mode, inp.lambda_floor, inp.lambda_max_extra,
                        inp.ent_target, inp.ent_ema)
+    if args.graph:
+        # a CUDA graph is captured on a stream other than the default one: run everything there
+        torch.cuda.set_stream(torch.cuda.Stream(dev))
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
