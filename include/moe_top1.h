@@ -53,7 +53,10 @@
 extern "C" {
 #endif
 
-#define MOE_TOP1_ABI_VERSION 1
+/* 1: routing, forward, backward, aux loss, lambda update.
+ * 2: adds moe_usage_entropy_ema_update and moe_top1_bwd_mean_collapse (every
+ *    version-1 call is unchanged). */
+#define MOE_TOP1_ABI_VERSION 2
 
 typedef enum {
     MOE_OK = 0,

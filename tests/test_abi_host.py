@@ -53,7 +53,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_top1_abi_version() == 1
+    assert L.moe_top1_abi_version() == 2
     for s, name in enumerate(ops._STATUS):
         assert L.moe_status_string(s).decode() == name
     assert L.moe_status_string(99).decode() == "MOE_ERR_UNKNOWN"

@@ -1,0 +1,53 @@
+"""Host-side pieces of bench.py (no GPU): the algorithmic bytes and flops the
+roofline is computed from, the FP32 SIMT ceiling of the FFMA path, the L2 note
+and the traffic record lookup."""
+import json
+import os
+
+import bench
+from bwd_route_b200 import workloads as wl
+
+LARGE = wl.WORKLOADS["large_b65536_e8_h256"]
+
+
+def test_algorithmic_bytes_and_flops_of_the_throughput_workload():
+    T, E, H = LARGE.T, LARGE.E, LARGE.H
+    step_bytes, step_flops, per = bench.algorithmic(LARGE)
+    # x twice, d_out once, routed and d_x written: 5 H floats; logits twice and d_logits: 3 E floats;
+    # expert_idx written, perm written and read: 16 bytes; W read and dW written per step
+    assert step_bytes == T * (4 * (5 * H + 3 * E) + 16) + 2 * E * H * H * 4
+    assert abs(step_bytes - 5.49e9) < 0.01e9
+    assert step_flops == 6 * H * H * T
+    assert per["fwd"] == per["d_x"] + E * H * 4 == T * (8 * H + 4) + E * H * H * 4 + E * H * 4
+    # the step roofline quoted in the docs: HBM-bound at the measured 6541 GB/s
+    assert abs(step_bytes / 6541e9 * 1e6 - 839) < 1
+
+
+def test_algorithmic_bytes_with_the_horizon_mean_gradient():
+    T, E, H, B = LARGE.T, LARGE.E, LARGE.H, LARGE.B
+    full, flops, per = bench.algorithmic(LARGE)
+    coll, flops_c, per_c = bench.algorithmic(LARGE, "mean_collapse")
+    assert flops_c == flops
+    # d_out [T, H] is read once in the plain step; the [B, H] gradient replaces it
+    assert full - coll == T * H * 4 - B * H * 4
+    assert per["d_x"] - per_c["d_x"] == T * H * 4 - B * H * 4
+
+
+def test_fp32_simt_ceiling_and_l2_note():
+    r = bench.simt_roofline(74.44992e12 * 1e-3, 1.0)  # exactly the peak for 1 ms
+    assert abs(r["frac"] - 1.0) < 1e-9 and r["bound"] == "alu"
+    assert "larger than L2" in bench.l2_note(LARGE, False, False)
+    assert "fit in L2" in bench.l2_note(wl.WORKLOADS["tiny_b8_e4_h128"], False, False)
+    assert "256 MB" in bench.l2_note(wl.WORKLOADS["tiny_b8_e4_h128"], False, True)
+
+
+def test_traffic_record_is_well_formed_and_keyed_to_the_sources():
+    text = open(bench.TRAFFIC_RECORD).read()
+    rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
+    assert rec["workload"] == LARGE.name and rec["math"] == "tf32"
+    for f in rec["source_files"]:
+        assert os.path.exists(os.path.join(bench.HERE, f)), f
+    assert set(rec["traffic_bytes_per_call"]) == {"fwd", "d_x", "wgrad"}
+    # the lookup refuses other workloads and the FFMA path
+    assert bench.recorded_traffic("fwd", "mid_b16384_e8_h256", "tf32") is None
+    assert bench.recorded_traffic("fwd", LARGE.name, "ffma") is None
