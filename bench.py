@@ -122,21 +122,32 @@ def host_cpu() -> dict:
 TRAFFIC_RECORD = os.path.join(HERE, "profiles", "launch_list_large_b65536_e8_h256.md")
 
 
+def code_sha1(paths) -> str:
+    """sha1 of the code of the given source files with comments and blank space
+    removed, so that a change to a comment does not count as a kernel change."""
+    import hashlib
+    import re
+    h = hashlib.sha1()
+    for path in paths:
+        with open(path) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()
+
+
 def recorded_traffic(call: str, workload: str, math_name: str):
     """DRAM bytes (read + write) of one launch of `call` from the committed ncu
     launch list, or None when there is no record for this workload and math
-    mode, or when the kernel sources changed since the counters were taken."""
-    import hashlib
+    mode, or when the kernel code changed since the counters were taken."""
     try:
         text = open(TRAFFIC_RECORD).read()
         rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
-        h = hashlib.sha1()
-        for f in rec["source_files"]:
-            with open(os.path.join(HERE, f), "rb") as fh:
-                h.update(fh.read())
+        digest = code_sha1([os.path.join(HERE, f) for f in rec["source_files"]])
     except (OSError, IndexError, KeyError, ValueError):
         return None
-    if rec.get("workload") != workload or rec.get("math") != math_name or h.hexdigest() != rec.get("source_sha1"):
+    if rec.get("workload") != workload or rec.get("math") != math_name or digest != rec.get("code_sha1"):
         return None
     v = rec.get("traffic_bytes_per_call", {}).get(call)
     return int(v) if v is not None else None

@@ -18,12 +18,16 @@
 // ~2.0 TB/s. The dense expert-weight operand is loaded by TMA.
 //
 //   grouped_tf32_kernel : persistent, one CTA per SM; a tile is 128 sorted
-//     tokens x all H outputs. Warps 4-7 gather the tile's rows (K-major,
-//     128-byte swizzle) into a 6-deep ring; warp 9 streams the expert's weight
-//     slab by TMA into a 3-deep ring (it comes from L2); warp 8 issues tcgen05.mma kind::tf32 (M=128, N=H, K=8) into one of two
-//     TMEM accumulators; warps 0-3 drain the other accumulator (tcgen05.ld),
-//     add the bias and store the rows to their original token positions with
-//     coalesced 128-byte stores.
+//     tokens x all H outputs. Warps 8-11 gather the tile's rows (K-major,
+//     128-byte swizzle) into a 6-deep ring; warp 13 streams the expert's weight
+//     slab by TMA into a 3-deep ring (it comes from L2; K-major for the
+//     forward, MN-major straight from W for d_x); one thread of warp 12 issues
+//     tcgen05.mma kind::tf32 (M=128, N=H, K=8) into one of two TMEM
+//     accumulators; warps 0-7 drain the other accumulator (tcgen05.ld), add
+//     the bias, transpose through shared memory and store the rows to their
+//     original token positions, 4 rows x 128 bytes per warp instruction. The
+//     COLLAPSE instances serve the backward through the horizon mean (gradient
+//     row t / N_H, result scaled by 1 / N_H).
 //
 //   wgrad_tf32_kernel : one CTA per range of the sorted token list (range c of
 //     expert e -> partial-sum slot c + e). Tokens are the contraction index, so
