@@ -15,8 +15,9 @@ controller of foxhunt commit 2d0e6b6bdc at the end of the step.
 from __future__ import annotations
 
 import torch
+import torch.distributed as dist
 
-from . import ops
+from . import dp, ops
 
 
 class MoETop1Gate:
@@ -41,8 +42,12 @@ class MoETop1Gate:
         self.routing = ops.Routing.empty(T, E, dev)
         self.routed = torch.empty(T, H, dtype=f32, device=dev)
         self.d_x = torch.empty(T, H, dtype=f32, device=dev)
-        self.dW = torch.empty(E, H, H, dtype=f32, device=dev)
-        self.db = torch.empty(E, H, dtype=f32, device=dev)
+        # dW and db are views of one flat buffer, so that a data-parallel step sums
+        # both over the ranks with one collective (db starts E*H*H*4 bytes in: a
+        # multiple of 4 KiB for every supported H)
+        self.grads = torch.empty(E * H * H + E * H, dtype=f32, device=dev)
+        self.dW = self.grads[:E * H * H].view(E, H, H)
+        self.db = self.grads[E * H * H:].view(E, H)
         self.d_logits = torch.empty(T, E, dtype=f32, device=dev)
         self.loss = torch.zeros(2, dtype=f32, device=dev)
         self.mean_p = torch.zeros(E, dtype=f32, device=dev)
@@ -52,6 +57,9 @@ class MoETop1Gate:
         self.usage_ema = torch.full((E,), 1.0 / E, dtype=f32, device=dev)
         self.ent_step = torch.zeros(1, dtype=f32, device=dev)
         self.ws = ops.new_workspace(T, E, H, dev)
+        self.dp_group = None
+        self.dp_tokens = T
+        self.counts_global = None
 
     def route(self, gate_logits, stream=None):
         ops.moe_top1_route(gate_logits, self.B, self.N_H, self.E, self.routing, self.ws, stream)
@@ -81,10 +89,37 @@ class MoETop1Gate:
     def update_controller(self, alpha: float, reset: bool = False, stream=None):
         """Closes the lambda loop after a step: the gate-entropy producer folds
         this step's usage into ent_ema (or resets it at a fold boundary), then
-        lambda_eff is recomputed from it for the next step."""
-        ops.moe_usage_entropy_ema_update(self.routing.counts, self.T, self.E, alpha, reset, self.usage_ema,
+        lambda_eff is recomputed from it for the next step. Under data
+        parallelism the usage is that of the global batch (counts summed over
+        the ranks), so every rank holds the same ent_ema and lambda_eff."""
+        counts = self.routing.counts
+        if self.dp_group is not None:
+            self._dp_stream_check(stream)
+            counts = dp.global_counts(counts, self.counts_global, self.dp_group)
+        ops.moe_usage_entropy_ema_update(counts, self.dp_tokens, self.E, alpha, reset, self.usage_ema,
                                          self.ent_ema, self.ent_step, stream)
         self.update_lambda(stream)
+
+    def enable_data_parallel(self, group=None):
+        """Makes this gate one replica of a data-parallel job over the ranks of
+        group (torch.distributed, initialised by the caller; NCCL on GPUs).
+        Every rank must hold a shard of the same [B, N_H] shape."""
+        self.dp_tokens = dp.world_tokens(self.T, self.W.device, group)
+        self.counts_global = torch.zeros(self.E, dtype=torch.int32, device=self.W.device)
+        self.dp_group = group if group is not None else dist.group.WORLD
+
+    def allreduce_gradients(self, stream=None):
+        """After backward: dW and db of the global batch on every rank (their
+        sum over the ranks' shards). A no-op without data parallelism."""
+        if self.dp_group is None:
+            return
+        self._dp_stream_check(stream)
+        dp.allreduce_gradients(self.grads, self.dp_group)
+
+    @staticmethod
+    def _dp_stream_check(stream):
+        if stream is not None and stream != torch.cuda.current_stream():
+            raise ValueError("a data-parallel step runs on torch's current stream")
 
     def step(self, gate_logits, x, d_out, stream=None):
         self.route(gate_logits, stream)
