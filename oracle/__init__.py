@@ -47,6 +47,7 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_bwd_dw.argtypes = [P, P, P, i64, i32, i32, i32, P, P, P, P]
     lib.oracle_bwd_db.argtypes = [P, P, i64, i32, i32, P, P]
     lib.oracle_bwd_dw_entries.argtypes = [P, P, P, i64, i32, i32, i64, P, P, P, P, P]
+    lib.oracle_fwd_mean_collapse.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P]
     lib.oracle_aux.argtypes = [P, P, i64, i32, ctypes.c_float, P, P, P, P, P]
     lib.oracle_lambda_eff.restype = ctypes.c_double
     lib.oracle_lambda_eff.argtypes = [ctypes.c_double] * 4
@@ -128,6 +129,25 @@ def bwd_db(d_out, expert_idx, E: int):
     sb = np.empty((E, H), np.float64)
     _load().oracle_bwd_db(_p(d_out), _p(idx), T, E, H, _p(db), _p(sb))
     return db, sb
+
+
+def fwd_mean_collapse(x, W, bias, expert_idx, N_H: int):
+    """Forward of the gate followed by the horizon mean [B, N_H, H] -> [B, H]
+    ("Single source of truth for the attention path" page, MHA additions):
+    ctx_mean[b] = (1/N_H) sum_h routed[b*N_H + h], exact products in double.
+    -> (ctx_mean [B,H], mag [B,H]) float64; mag is (1/N_H) sum_h of the absolute
+    terms, sum_i |W x| + |bias|."""
+    x, W, bias, idx = _f32(x), _f32(W), _f32(bias), _i32(expert_idx)
+    T, H = x.shape
+    E = W.shape[0]
+    N_H = int(N_H)
+    if N_H < 1 or T % N_H:
+        raise ValueError("T must be a multiple of N_H >= 1")
+    B = T // N_H
+    out = np.empty((B, H), np.float64)
+    mag = np.empty((B, H), np.float64)
+    _load().oracle_fwd_mean_collapse(_p(x), _p(W), _p(bias), _p(idx), B, N_H, E, H, _p(out), _p(mag))
+    return out, mag
 
 
 def bwd_mean_collapse(x, W, grad_ctx_mean, expert_idx, N_H: int, E: int, tf32_mode: int = TF32_NONE,

@@ -114,6 +114,42 @@ void oracle_fwd(const float* x, const float* W, const float* bias, const int32_t
 }
 
 /* ------------------------------------------------------------------------- */
+/* Forward followed by the horizon mean. [P5] MHA additions: the gate's      */
+/* output [B, N_H, H] is averaged over the horizon axis into ctx_mean [B, H]: */
+/*   ctx_mean[b, o] = (1/N_H) sum_h routed[b*N_H + h, o],                     */
+/* routed being the forward above (exact products, no TF32 rounding), the    */
+/* horizon tokens visited in ascending h. Also returns the size of the terms,*/
+/*   mag[b, o] = (1/N_H) sum_h (sum_i |W[e,o,i] x[t,i]| + |bias[e,o]|),       */
+/* which bounds what rounding the inputs or the partial sums can change.     */
+/* ------------------------------------------------------------------------- */
+void oracle_fwd_mean_collapse(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
+                              int64_t B, int32_t N_H, int32_t E, int32_t H, double* ctx_mean, double* mag)
+{
+    (void)E;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int32_t o = 0; o < H; ++o) {
+            double sum = 0.0, size = 0.0;
+            for (int32_t h = 0; h < N_H; ++h) {
+                const int64_t t = b * N_H + h;
+                const int32_t e_t = expert_idx[t];
+                const float* w_row = W + ((int64_t)e_t * H + o) * H;
+                double acc = 0.0, acc_abs = 0.0;
+                for (int32_t i = 0; i < H; ++i) {
+                    const double term = (double)w_row[i] * (double)x[t * H + i];
+                    acc += term;
+                    acc_abs += fabs(term);
+                }
+                const double b_o = (double)bias[(int64_t)e_t * H + o];
+                sum += acc + b_o;
+                size += acc_abs + fabs(b_o);
+            }
+            ctx_mean[b * H + o] = sum / (double)N_H;
+            if (mag) mag[b * H + o] = size / (double)N_H;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
 /* Backward, input gradient. [P1] kernel list and PERFORMANCE: the chain rule */
 /* runs through the selected expert only, and the weight column lines up     */
 /* with the input index:  d_x[t, i] = sum_o W[e*, o, i] * d_out[t, o].        */

@@ -51,6 +51,15 @@ MUTATIONS = [
     ("usage average from the wrong expert", "usage_ema[e] = (1.0 - alpha) * usage_ema[e] + alpha * ((double)counts[e] / (double)T);",
      "usage_ema[e] = (1.0 - alpha) * usage_ema[e] + alpha * ((double)counts[0] / (double)T);"),
     ("cold start entropy wrong", "*ent_ema = log((double)E);", "*ent_ema = 1.0 / (double)E;"),
+    ("horizon mean not divided by N_H", "ctx_mean[b * H + o] = sum / (double)N_H;", "ctx_mean[b * H + o] = sum;"),
+    ("horizon mean drops the bias", "sum += acc + b_o;", "sum += acc;"),
+    ("horizon mean uses W transposed", "const double term = (double)w_row[i] * (double)x[t * H + i];",
+     "const double term = (double)W[((int64_t)e_t * H + i) * H + o] * (double)x[t * H + i];"),
+    ("horizon mean takes the first token's expert", "const int32_t e_t = expert_idx[t];",
+     "const int32_t e_t = expert_idx[b * N_H];"),
+    ("horizon mean reads token 0's input", "(double)w_row[i] * (double)x[t * H + i];",
+     "(double)w_row[i] * (double)x[b * N_H * H + i];"),
+    ("horizon mean magnitude keeps signs", "acc_abs += fabs(term);", "acc_abs += term;"),
 ]
 
 

@@ -557,3 +557,63 @@ def test_bwd_mean_collapse_equals_plain_backward_on_the_broadcast_gradient():
         dW, db, _, _ = oracle.bwd_dw(x, d_out, idx, E, mode)
         np.testing.assert_allclose(got["dW"], dW, rtol=1e-15, atol=1e-15)
         np.testing.assert_allclose(got["db"], db, rtol=1e-15, atol=1e-15)
+
+
+# ---------------------------------------------------------------- forward through the horizon mean
+def test_fwd_mean_collapse_with_one_horizon_token_is_the_forward():
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=7, N_H=1)
+    got, _ = oracle.fwd_mean_collapse(x, W, bias, idx, 1)
+    np.testing.assert_array_equal(got, oracle.fwd(x, W, bias, idx))
+
+
+def test_fwd_mean_collapse_is_the_horizon_mean_of_the_forward():
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=4, N_H=5)
+    got, _ = oracle.fwd_mean_collapse(x, W, bias, idx, N_H)
+    want = oracle.fwd(x, W, bias, idx).reshape(B, N_H, H).mean(axis=1)
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-14)
+
+
+def test_fwd_mean_collapse_identity_experts_average_x():
+    x, _, _, _, idx, B, N_H, E, H = _collapse_case(B=5, N_H=6)
+    W = np.broadcast_to(np.eye(H, dtype=np.float32), (E, H, H)).copy()
+    got, mag = oracle.fwd_mean_collapse(x, W, np.zeros((E, H), np.float32), idx, N_H)
+    np.testing.assert_allclose(got, x.astype(np.float64).reshape(B, N_H, H).mean(axis=1), rtol=1e-15, atol=1e-15)
+    np.testing.assert_allclose(mag, np.abs(x.astype(np.float64)).reshape(B, N_H, H).mean(axis=1), rtol=1e-15)
+
+
+def test_fwd_mean_collapse_of_zero_input_averages_the_chosen_biases():
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=6, N_H=7, E=4)
+    got, _ = oracle.fwd_mean_collapse(np.zeros_like(x), W, bias, idx, N_H)
+    want = bias.astype(np.float64)[idx.reshape(B, N_H)].mean(axis=1)
+    np.testing.assert_allclose(got, want, rtol=1e-15, atol=1e-17)
+
+
+def test_fwd_mean_collapse_does_not_depend_on_the_horizon_order():
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=4, N_H=6)
+    perm = np.random.default_rng(5).permutation(N_H)
+    xs = x.reshape(B, N_H, H)[:, perm].reshape(B * N_H, H)
+    ids = idx.reshape(B, N_H)[:, perm].reshape(-1)
+    a, ma = oracle.fwd_mean_collapse(x, W, bias, idx, N_H)
+    b, mb = oracle.fwd_mean_collapse(xs, W, bias, ids, N_H)
+    np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(ma, mb, rtol=1e-13)
+
+
+def test_fwd_mean_collapse_is_the_adjoint_of_the_pinned_backward():
+    """ctx_mean is affine in x and its linear part is adjoint to the collapsed
+    input gradient: sum_b g[b] . (ctx(x) - ctx(0)) = sum_t d_x[t] . x[t]."""
+    x, W, bias, g, idx, B, N_H, E, H = _collapse_case(B=5, N_H=3, E=4)
+    cx, _ = oracle.fwd_mean_collapse(x, W, bias, idx, N_H)
+    c0, _ = oracle.fwd_mean_collapse(np.zeros_like(x), W, bias, idx, N_H)
+    lhs = float((g.astype(np.float64) * (cx - c0)).sum())
+    d_x = oracle.bwd_mean_collapse(x, W, g, idx, N_H, E, with_dw=False)["d_x"]
+    rhs = float((d_x * x.astype(np.float64)).sum())
+    assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs)), (lhs, rhs)
+
+
+def test_fwd_mean_collapse_magnitude_bounds_the_value_and_is_exact_for_positive_terms():
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=4, N_H=5)
+    got, mag = oracle.fwd_mean_collapse(x, W, bias, idx, N_H)
+    assert np.all(np.abs(got) <= mag * (1 + 1e-14))
+    got, mag = oracle.fwd_mean_collapse(np.abs(x), np.abs(W), np.abs(bias), idx, N_H)
+    np.testing.assert_allclose(mag, got, rtol=1e-14)
