@@ -48,15 +48,19 @@ def load_peaks():
 
 def algorithmic(spec, grad: str = "token"):
     """Bytes and flops the method itself must move / compute for one step.
-    grad = "mean_collapse": the output gradient arrives as [B, H] (the gradient
-    of the horizon mean) instead of [T, H]."""
+    grad = "mean_collapse": the gate's output is averaged over the horizon axis,
+    so the forward writes ctx_mean [B, H] instead of routed [T, H], and the
+    output gradient arrives as [B, H] (the gradient of that mean)."""
     T, E, H, B = spec.T, spec.E, spec.H, spec.B
     step_flops = 6 * H * H * T
     if grad == "mean_collapse":
         g_bytes = B * H * 4
-        step_bytes = T * (4 * (4 * H + 3 * E) + 16) + g_bytes + 2 * E * H * H * 4
+        # per token: x read twice, d_x written (3 H floats); logits read twice and
+        # d_logits written (3 E floats); expert index and permutation traffic
+        step_bytes = T * (4 * (3 * H + 3 * E) + 16) + 2 * g_bytes + 2 * E * H * H * 4
         per_kernel_bytes = {
-            "fwd": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
+            # x and the expert indices read, ctx_mean written; W and bias
+            "fwd": T * (4 * H + 4) + g_bytes + E * H * H * 4 + E * H * 4,
             # grad_ctx_mean read once, d_x written, perm read; W
             "d_x": T * (4 * H + 4) + g_bytes + E * H * H * 4,
             # x and grad_ctx_mean read, perm read; dW and db written
@@ -85,8 +89,9 @@ def l2_note(spec, collapse: bool, flushed: bool) -> str:
     act = T * H * 4
     if act * 2 > L2_BYTES:
         if collapse:
-            return ("inputs larger than L2 (x, routed, d_x: 3 x %.2f GB; the [B, H] gradient, %.0f MB, stays in "
-                    "L2)%s" % (act / 1e9, B * H * 4 / 1e6, ", L2 also flushed between steps" if flushed else ", no flush"))
+            return ("inputs larger than L2 (x, d_x: 2 x %.2f GB; the [B, H] mean and its gradient, %.0f MB each, "
+                    "stay in L2)%s" % (act / 1e9, B * H * 4 / 1e6,
+                                       ", L2 also flushed between steps" if flushed else ", no flush"))
         return "inputs larger than L2 (x, d_out, routed, d_x: 4 x %.2f GB)%s" % (
             act / 1e9, ", L2 also flushed between steps" if flushed else ", no flush")
     total = 4 * act + T * E * 8 + 2 * E * H * H * 4
@@ -272,7 +277,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--grad", choices=["token", "mean_collapse"], default="token",
-                    help="output gradient per token [T, H] (default) or of the horizon mean [B, H]")
+                    help="the gate's output per token [T, H] with its gradient (default), or averaged over "
+                         "the horizon axis: the forward writes ctx_mean [B, H] and its gradient is [B, H]")
     ap.add_argument("--graph", action="store_true",
                     help="time K replays of one step captured in a CUDA graph (the per-call times then come "
                          "from a separate un-captured loop); for launch-bound small workloads")
@@ -327,7 +333,10 @@ def main():
         gate.route(logits)
         if ev:
             ev[1].record(stream)
-        gate.forward(x)
+        if collapse:
+            gate.forward_mean_collapse(x)
+        else:
+            gate.forward(x)
         if ev:
             ev[2].record(stream)
         bwd = ops.moe_top1_bwd_mean_collapse if collapse else ops.moe_top1_bwd
@@ -417,7 +426,7 @@ def main():
         d_out.copy_(h_dout, non_blocking=True)
         if collapse:
             gate.route(logits)
-            gate.forward(x)
+            gate.forward_mean_collapse(x)
             gate.backward_mean_collapse(x, d_out)
             gate.aux(logits)
             gate.update_lambda()
@@ -441,7 +450,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": spec.name + ("+mean_collapse_bwd" if collapse else ""), "B": spec.B,
+            "config": {"workload": spec.name + ("+mean_collapse" if collapse else ""), "B": spec.B,
                        "N_H": spec.N_H, "E": E, "H": H, "tokens": T, "grad": args.grad,
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": l2_note(spec, collapse, flush is not None)},

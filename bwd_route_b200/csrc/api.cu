@@ -363,6 +363,44 @@ moe_status_t moe_top1_fwd(const float* x, const float* W, const float* bias, con
     return cuda_status(launch_grouped_ffma(x, W, bias, routing->offsets, routing->perm, T, E, H, 1, 0, 1, 1.0f, routed, s));
 }
 
+moe_status_t moe_top1_fwd_mean_collapse(const float* x, const float* W, const float* bias,
+                                        const moe_routing_t* routing, int64_t B, int64_t N_H, int32_t E, int32_t H,
+                                        moe_math_t math, float* ctx_mean, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+    int64_t T = 0;
+    moe_status_t st = tokens(B, N_H, &T);
+    if (st != MOE_OK) return st;
+    if (math != MOE_MATH_TF32 && math != MOE_MATH_FFMA) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || E > 32 || !h_supported(H, math)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (B > 0 && (N_H < 1 || N_H > 32)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!routing || !W || !bias) return MOE_ERR_INVALID_ARG;
+    if (B > 0 && (!x || !ctx_mean || !routing->expert_idx)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(W, 16) || !aligned(bias, 16) || !aligned(ctx_mean, 16)) return MOE_ERR_MISALIGNED;
+    if (!aligned(routing->expert_idx, 4)) return MOE_ERR_MISALIGNED;
+    const Range outs[1] = {{ctx_mean, sizeof(float) * B * H}};
+    const Range ins[5] = {{x, sizeof(float) * T * H},
+                          {W, sizeof(float) * E * H * H},
+                          {bias, sizeof(float) * E * H},
+                          {routing->expert_idx, sizeof(int32_t) * T},
+                          {workspace, workspace ? workspace_bytes : 0}};
+    if (any_alias(outs, 1, ins, 5)) return MOE_ERR_ALIAS;
+    if (math == MOE_MATH_TF32) {
+        if (!workspace) return MOE_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
+        if (workspace_bytes < 256) return MOE_ERR_WORKSPACE;
+    }
+    if (B == 0) return MOE_OK;
+    DeviceInfo* dev = nullptr;
+    cudaError_t e = device_info(&dev);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int nh = static_cast<int>(N_H);
+    if (math == MOE_MATH_TF32)
+        return cuda_status(launch_hmean_fwd_tf32(x, W, bias, routing->expert_idx, B, nh, E, H, ctx_mean,
+                                                 static_cast<uint32_t*>(workspace), dev->num_sms, s));
+    return cuda_status(launch_hmean_fwd_ffma(x, W, bias, routing->expert_idx, B, nh, E, H, ctx_mean, s));
+}
+
 moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out, const moe_routing_t* routing,
                           int64_t B, int64_t N_H, int32_t E, int32_t H, moe_math_t math, float* d_x, float* dW,
                           float* db, uint32_t accumulate_flags, void* workspace, size_t workspace_bytes,

@@ -137,6 +137,115 @@ __global__ void __launch_bounds__(kGThreads) grouped_ffma_kernel(const float* __
     }
 }
 
+// ---------------------------------------------------------------- forward through the horizon mean (FFMA)
+// ctx_mean[b] = (1/N_H) (sum_e W[e] X_be + sum_e n_be bias[e]) with
+// X_be = sum_{h : e_bh = e} x[b,h] summed in ascending h ("Single source of
+// truth for the attention path", MHA additions). Block = 128 batch rows x 32
+// outputs; the K loop runs over (e, 32-wide k-chunk) in a fixed order.
+__global__ void __launch_bounds__(kGThreads) hmean_fwd_ffma_kernel(const float* __restrict__ x,
+                                                                  const float* __restrict__ W,
+                                                                  const float* __restrict__ bias,
+                                                                  const int32_t* __restrict__ expert_idx, int B,
+                                                                  int N_H, int E, int H, float inv_nh,
+                                                                  float* __restrict__ out) {
+    __shared__ uint32_t s_mask[kGBM][32];  // [row][e], bit h: horizon token h (N_H <= 32) chose expert e
+    __shared__ __align__(16) float sA[kGBK][kGBM + 4];    // X_be^T: [k][row]
+    __shared__ __align__(16) float sB[kGBK][kGBN + 4];    // [k][n]
+    const int tid = threadIdx.x;
+    const int b0 = blockIdx.x * kGBM;
+    const int n0 = blockIdx.y * kGBN;
+    for (int m = tid; m < kGBM; m += kGThreads) {
+        uint32_t mk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mk[e] = 0u;
+        const int b = b0 + m;
+        if (b < B) {
+            for (int h = 0; h < N_H; ++h) {
+                const int e = expert_idx[static_cast<int64_t>(b) * N_H + h];
+#pragma unroll
+                for (int f = 0; f < 32; ++f)
+                    if (f == e) mk[f] |= 1u << h;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s_mask[m][e] = mk[e];
+    }
+    __syncthreads();
+    const int tm = tid / 8, tn = tid % 8;  // rows tm*4.., cols tn*4..
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int e = 0; e < E; ++e) {
+        const float* We = W + static_cast<int64_t>(e) * H * H;
+        for (int k0 = 0; k0 < H; k0 += kGBK) {
+#pragma unroll
+            for (int q = 0; q < (kGBM * kGBK / 4) / kGThreads; ++q) {
+                const int idx = tid + q * kGThreads;
+                const int m = idx / 8, kq = idx % 8;
+                uint32_t mk = s_mask[m][e];
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (mk) {
+                    const float* xr = x + static_cast<int64_t>(b0 + m) * N_H * H + k0 + kq * 4;
+                    v = __ldg(reinterpret_cast<const float4*>(xr + static_cast<int64_t>(__ffs(mk) - 1) * H));
+                    for (mk &= mk - 1; mk; mk &= mk - 1) {
+                        const float4 u = __ldg(reinterpret_cast<const float4*>(xr + static_cast<int64_t>(__ffs(mk) - 1) * H));
+                        v.x += u.x;
+                        v.y += u.y;
+                        v.z += u.z;
+                        v.w += u.w;
+                    }
+                }
+                sA[kq * 4 + 0][m] = v.x;
+                sA[kq * 4 + 1][m] = v.y;
+                sA[kq * 4 + 2][m] = v.z;
+                sA[kq * 4 + 3][m] = v.w;
+            }
+            {  // B[k][n] = W[e][n0+n][k0+k]
+                const int n = tid / 8, kq = tid % 8;
+                const float4 v = __ldg(reinterpret_cast<const float4*>(We + static_cast<int64_t>(n0 + n) * H + k0) + kq);
+                sB[kq * 4 + 0][n] = v.x;
+                sB[kq * 4 + 1][n] = v.y;
+                sB[kq * 4 + 2][n] = v.z;
+                sB[kq * 4 + 3][n] = v.w;
+            }
+            __syncthreads();
+#pragma unroll 8
+            for (int k = 0; k < kGBK; ++k) {
+                const float4 a = *reinterpret_cast<const float4*>(&sA[k][tm * 4]);
+                const float4 b = *reinterpret_cast<const float4*>(&sB[k][tn * 4]);
+                const float av[4] = {a.x, a.y, a.z, a.w};
+                const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            }
+            __syncthreads();
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int m = tm * 4 + i;
+        const int b = b0 + m;
+        if (b >= B) continue;
+        float r[4] = {acc[i][0], acc[i][1], acc[i][2], acc[i][3]};
+        for (int e = 0; e < E; ++e) {
+            const uint32_t mk = s_mask[m][e];
+            if (!mk) continue;
+            const float n = static_cast<float>(__popc(mk));
+            const float4 bb = __ldg(reinterpret_cast<const float4*>(bias + static_cast<int64_t>(e) * H + n0 + tn * 4));
+            r[0] = fmaf(n, bb.x, r[0]);
+            r[1] = fmaf(n, bb.y, r[1]);
+            r[2] = fmaf(n, bb.z, r[2]);
+            r[3] = fmaf(n, bb.w, r[3]);
+        }
+        *reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * H + n0 + tn * 4) =
+            make_float4(r[0] * inv_nh, r[1] * inv_nh, r[2] * inv_nh, r[3] * inv_nh);
+    }
+}
+
 // ---------------------------------------------------------------- weight gradient (FFMA)
 // CTA (c, o-tile, i-tile): for every expert piece of range c, accumulate the
 // 32 x 32 block of d_out^T x over the piece's tokens (ascending sorted order),
@@ -337,6 +446,15 @@ cudaError_t launch_grouped_ffma(const float* src, const float* Wsrc, const float
     dim3 grid(static_cast<unsigned>(tiles), H / kGBN);
     grouped_ffma_kernel<<<grid, kGThreads, 0, s>>>(src, Wsrc, bias, offsets, perm, E, H, b_kmajor, accumulate,
                                                    src_div, out_scale, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_hmean_fwd_ffma(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
+                                  int64_t B, int N_H, int E, int H, float* out, cudaStream_t s) {
+    const dim3 grid(static_cast<unsigned>((B + kGBM - 1) / kGBM), static_cast<unsigned>(H / kGBN));
+    const float inv_nh = static_cast<float>(1.0 / static_cast<double>(N_H));
+    hmean_fwd_ffma_kernel<<<grid, kGThreads, 0, s>>>(x, W, bias, expert_idx, static_cast<int>(B), N_H, E, H, inv_nh,
+                                                     out);
     return cudaGetLastError();
 }
 

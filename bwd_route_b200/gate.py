@@ -42,6 +42,7 @@ class MoETop1Gate:
         self.routing = ops.Routing.empty(T, E, dev)
         self.routed = torch.empty(T, H, dtype=f32, device=dev)
         self.d_x = torch.empty(T, H, dtype=f32, device=dev)
+        self.ctx_mean = torch.empty(B, H, dtype=f32, device=dev)
         # dW and db are views of one flat buffer, so that a data-parallel step sums
         # both over the ranks with one collective (db starts E*H*H*4 bytes in: a
         # multiple of 4 KiB for every supported H)
@@ -67,6 +68,11 @@ class MoETop1Gate:
     def forward(self, x, stream=None):
         ops.moe_top1_fwd(x, self.W, self.bias, self.routing, self.B, self.N_H, self.E, self.H, self.math,
                          self.routed, self.ws, stream)
+
+    def forward_mean_collapse(self, x, stream=None):
+        """Forward followed by the horizon mean: ctx_mean [B, H] (no [T, H] output)."""
+        ops.moe_top1_fwd_mean_collapse(x, self.W, self.bias, self.routing, self.B, self.N_H, self.E, self.H, self.math,
+                                       self.ctx_mean, self.ws, stream)
 
     def backward(self, x, d_out, stream=None):
         ops.moe_top1_bwd(x, self.W, d_out, self.routing, self.B, self.N_H, self.E, self.H, self.math, self.d_x,

@@ -29,7 +29,7 @@ EXPORTED = [
     "moe_top1_workspace_bytes", "moe_top1_workspace_init", "moe_top1_route", "moe_top1_fwd",
     "moe_top1_bwd", "moe_aux_loss_fwd_bwd", "moe_lambda_eff_update", "moe_top1_device_flags",
     "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc", "moe_top1_selftest_wait_timeout",
-    "moe_usage_entropy_ema_update", "moe_top1_bwd_mean_collapse",
+    "moe_usage_entropy_ema_update", "moe_top1_bwd_mean_collapse", "moe_top1_fwd_mean_collapse",
 ]
 MOE_NOALLOC_MAX_TOKENS = 2097152
 
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.moe_top1_route.argtypes = [P, I64, I64, I32, ctypes.POINTER(RoutingC), P, SZ, P]
         L.moe_top1_fwd.restype = I32
         L.moe_top1_fwd.argtypes = [P, P, P, ctypes.POINTER(RoutingC), I64, I64, I32, I32, I32, P, P, SZ, P]
+        L.moe_top1_fwd_mean_collapse.restype = I32
+        L.moe_top1_fwd_mean_collapse.argtypes = L.moe_top1_fwd.argtypes
         L.moe_top1_bwd.restype = I32
         L.moe_top1_bwd.argtypes = [P, P, P, ctypes.POINTER(RoutingC), I64, I64, I32, I32, I32, P, P, P, U32,
                                    P, SZ, P]
@@ -182,6 +184,16 @@ def moe_top1_fwd(x, W, bias, routing: Routing, B: int, N_H: int, E: int, H: int,
     f = torch.float32
     _check("moe_top1_fwd", lib().moe_top1_fwd(_ptr(x, f), _ptr(W, f), _ptr(bias, f), ctypes.byref(rc), B, N_H, E, H,
                                               math, _ptr(routed, f), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_top1_fwd_mean_collapse(x, W, bias, routing: Routing, B: int, N_H: int, E: int, H: int, math: int, ctx_mean,
+                               ws: torch.Tensor, stream=None):
+    """ctx_mean [B, H] = the horizon mean of moe_top1_fwd's [B * N_H, H] output."""
+    rc = routing.c()
+    f = torch.float32
+    _check("moe_top1_fwd_mean_collapse",
+           lib().moe_top1_fwd_mean_collapse(_ptr(x, f), _ptr(W, f), _ptr(bias, f), ctypes.byref(rc), B, N_H, E, H,
+                                            math, _ptr(ctx_mean, f), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def moe_top1_bwd(x, W, d_out, routing: Routing, B: int, N_H: int, E: int, H: int, math: int, d_x, dW, db,

@@ -55,8 +55,9 @@ extern "C" {
 
 /* 1: routing, forward, backward, aux loss, lambda update.
  * 2: adds moe_usage_entropy_ema_update and moe_top1_bwd_mean_collapse (every
- *    version-1 call is unchanged). */
-#define MOE_TOP1_ABI_VERSION 2
+ *    version-1 call is unchanged).
+ * 3: adds moe_top1_fwd_mean_collapse (every earlier call is unchanged). */
+#define MOE_TOP1_ABI_VERSION 3
 
 typedef enum {
     MOE_OK = 0,
@@ -151,6 +152,27 @@ moe_status_t moe_top1_fwd(const float* x, const float* W, const float* bias,
                           int32_t H, moe_math_t math, float* routed, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/*
+ * Forward with the horizon mean-collapse folded in. [P5] MHA additions and the
+ * horizon_mean_collapse kernel: the MoE output [B, N_H, H] is averaged over the
+ * horizon axis into ctx_mean [B, H]:
+ *   ctx_mean[b, o] = (1/N_H) sum_h routed[b * N_H + h, o]
+ * with routed as in moe_top1_fwd, without that [T, H] array ever existing. The
+ * horizon tokens of row b that chose expert e are summed first (ascending h,
+ * fp32), so ctx_mean[b] = (1/N_H) (sum_e W[e] X_be + sum_e n_be bias[e]) is one
+ * contraction per row with K = E * H, accumulated over the experts in a fixed
+ * order (deterministic, no atomics). Reads only routing->expert_idx. ctx_mean
+ * [B, H] is overwritten and must not overlap any input. 1 <= N_H <= 32 when
+ * B > 0 (MOE_ERR_UNSUPPORTED_SHAPE otherwise). MOE_MATH_TF32 rounds the summed
+ * rows and W to TF32 inside the tensor core; MOE_MATH_FFMA multiplies in FP32.
+ * An expert index outside [0, E) contributes nothing. Same workspace rule as
+ * moe_top1_fwd (TF32: the flag word).
+ */
+moe_status_t moe_top1_fwd_mean_collapse(const float* x, const float* W, const float* bias,
+                                        const moe_routing_t* routing, int64_t B, int64_t N_H, int32_t E,
+                                        int32_t H, moe_math_t math, float* ctx_mean, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
 /* Accumulate flags of moe_top1_bwd: a set bit adds the result to the output
  * buffer instead of overwriting it ([P1] kernel list calls d_fused_ctx an
  * accumulator; [P5] zeroes the gradients at step start). */
@@ -190,9 +212,7 @@ moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out,
  * is applied once to each result (exact when N_H is a power of two; otherwise
  * within one rounding of the definition). Same arguments, outputs, flags,
  * workspace and errors as moe_top1_bwd; grad_ctx_mean must not overlap any
- * output. No counterpart of the forward half: a token's N_H horizon siblings go
- * to different experts, so a fused forward collapse would need a cross-CTA sum
- * that is not deterministic.
+ * output. The forward half is moe_top1_fwd_mean_collapse.
  */
 moe_status_t moe_top1_bwd_mean_collapse(const float* x, const float* W, const float* grad_ctx_mean,
                                         const moe_routing_t* routing, int64_t B, int64_t N_H, int32_t E,

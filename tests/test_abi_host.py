@@ -53,7 +53,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_top1_abi_version() == 2
+    assert L.moe_top1_abi_version() == 3
     for s, name in enumerate(ops._STATUS):
         assert L.moe_status_string(s).decode() == name
     assert L.moe_status_string(99).decode() == "MOE_ERR_UNKNOWN"
@@ -156,6 +156,24 @@ def test_bwd_mean_collapse_rejects_bad_arguments(L):
     assert b(*args(g=_p(A + 0x3000004))) == MISALIGNED
     # d_x overlapping the last row of grad_ctx_mean [B, H] = 8 x 128 floats
     assert b(*args(dx=_p(A + 0x3000000 + 4 * 128 * 7))) == ALIAS
+
+
+def test_fwd_mean_collapse_rejects_bad_arguments(L):
+    f = L.moe_top1_fwd_mean_collapse
+    R = ops.RoutingC(_p(A + 0x100000), _p(A + 0x200000), _p(A + 0x300000), _p(A + 0x400000))
+    x, W, b, out = _p(A + 0x1000000), _p(A + 0x2000000), _p(A + 0x3000000), _p(A + 0x4000000)
+    ws, wsb = _p(A + 0x40000000), 1 << 30
+    args = lambda **k: [x, k.get("W", W), b, ctypes.byref(R), k.get("B", 8), k.get("N_H", 5), 4, k.get("H", 128),
+                        k.get("math", 0), k.get("out", out), k.get("ws", ws), wsb, None]
+    assert f(*args(N_H=33)) == SHAPE      # one mask bit per horizon token
+    assert f(*args(N_H=0)) == SHAPE       # a mean over no tokens
+    assert f(*args(H=96)) == SHAPE
+    assert f(*args(math=7)) == INVALID
+    assert f(*args(W=None)) == INVALID
+    assert f(*args(out=_p(A + 0x4000008))) == MISALIGNED
+    assert f(*args(out=_p(A + 0x1000000 + 4 * 128 * 39))) == ALIAS   # ctx_mean on the last row of x [40, 128]
+    assert f(*args(ws=None)) == WORKSPACE
+    assert f(*args(B=0)) == OK            # nothing to compute: returns before any launch
 
 
 def test_usage_entropy_update_rejects_bad_arguments(L):

@@ -28,9 +28,11 @@ def test_algorithmic_bytes_with_the_horizon_mean_gradient():
     full, flops, per = bench.algorithmic(LARGE)
     coll, flops_c, per_c = bench.algorithmic(LARGE, "mean_collapse")
     assert flops_c == flops
-    # d_out [T, H] is read once in the plain step; the [B, H] gradient replaces it
-    assert full - coll == T * H * 4 - B * H * 4
+    # d_out [T, H] is read once and routed [T, H] written once in the plain step;
+    # the [B, H] gradient and the [B, H] mean replace them
+    assert full - coll == 2 * (T * H * 4 - B * H * 4)
     assert per["d_x"] - per_c["d_x"] == T * H * 4 - B * H * 4
+    assert per["fwd"] - per_c["fwd"] == T * H * 4 - B * H * 4
 
 
 def test_fp32_simt_ceiling_and_l2_note():

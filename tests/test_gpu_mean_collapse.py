@@ -99,3 +99,108 @@ def test_mean_collapse_accumulate_flags(math_mode):
     acc = _run(inp, g, math_mode, acc_flags=ops.MOE_ACC_DX | ops.MOE_ACC_DW | ops.MOE_ACC_DB, preset=pre)
     for k in ("d_x", "dW", "db"):
         np.testing.assert_array_equal(acc[k], (pre[k] + plain[k]).astype(np.float32), err_msg=k)
+
+
+# ---------------------------------------------------------------- forward through the horizon mean
+FWD_SPECS = [
+    wl.make_spec("mcf_b8_h5_e4_h128", 8, 5, 4, 128, 51),                # one partial tile
+    wl.make_spec("mcf_b1024_h5_e4_h128", 1024, 5, 4, 128, 52),          # eight full tiles
+    wl.make_spec("mcf_b777_h3_e8_h256", 777, 3, 8, 256, 53),            # ragged last tile, H = 256
+    wl.make_spec("mcf_b2048_h16_e8_h256", 2048, 16, 8, 256, 54),        # the throughput shape's N_H, E, H
+    wl.make_spec("mcf_b300_h32_e32_h128", 300, 32, 32, 128, 55),        # N_H and E at their maximum
+    wl.make_spec("mcf_b257_h7_e4_h128", 257, 7, 4, 128, 56, skew_expert=2, skew_value=3.0),  # > 2 tokens per (b, e)
+    wl.make_spec("mcf_b130_h5_e4_h128", 130, 5, 4, 128, 57, logits="binary"),               # frequent ties
+]
+
+
+def fwd_bound(spec, math):
+    """|got - exact| <= c * mag, mag = (1/N_H) sum_h (sum_i |W x| + |bias|) from the
+    oracle. fp32 sums: the horizon pre-sum (N_H terms), the K = E * H products and
+    the epilogue's bias, scale and store (8 more roundings), each at most one
+    unit 2^-24 of mag. TF32 adds the rounding of both operands of every product,
+    each below 2^-10 relative."""
+    c = (spec.E * spec.H + spec.N_H + 8) * 2.0 ** -24
+    if math == ops.MOE_MATH_TF32:
+        c += 2.0 ** -9
+    return c
+
+
+def _run_fwd(spec, inp, math):
+    out = Guarded(spec.B * spec.H, shape=(spec.B, spec.H))
+    r = ops.Routing.empty(spec.T, spec.E, "cuda")
+    ws = ops.new_workspace(spec.T, spec.E, spec.H, "cuda")
+    ops.moe_top1_route(dev(inp.gate_logits), spec.B, spec.N_H, spec.E, r, ws)
+    ops.moe_top1_fwd_mean_collapse(dev(inp.x), dev(inp.W), dev(inp.bias), r, spec.B, spec.N_H, spec.E, spec.H,
+                                   math, out.t, ws)
+    torch.cuda.synchronize()
+    assert ops.moe_top1_device_flags(ws) == 0
+    assert out.guards_intact()
+    return out.host(), r, ws
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+@pytest.mark.parametrize("spec", FWD_SPECS, ids=lambda s: s.name)
+def test_fwd_mean_collapse_parity(spec, math_mode):
+    inp = wl.generate(spec)
+    got, _, _ = _run_fwd(spec, inp, math_mode)
+    idx = oracle.route(inp.gate_logits)[0]
+    want, mag = oracle.fwd_mean_collapse(inp.x, inp.W, inp.bias, idx, spec.N_H)
+    err = np.abs(got.astype(np.float64) - want)
+    bound = fwd_bound(spec, math_mode) * mag
+    assert np.isfinite(got).all()
+    assert (err <= bound).all(), f"max err/bound {np.max(err / bound):.3g}"
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_fwd_mean_collapse_with_one_horizon_token_is_the_plain_forward_bitwise(math_mode):
+    """N_H = 1: every (b, e) sum is one row or zero, the other experts add exact
+    zeros, and the products run in the plain forward's k order, so the result
+    must equal moe_top1_fwd bit for bit."""
+    spec = wl.make_spec("mcf_b1000_h1_e8_h256", 1000, 1, 8, 256, 58)
+    inp = wl.generate(spec)
+    got, r, ws = _run_fwd(spec, inp, math_mode)
+    routed = torch.empty(spec.T, spec.H, device="cuda")
+    ops.moe_top1_fwd(dev(inp.x), dev(inp.W), dev(inp.bias), r, spec.B, 1, spec.E, spec.H, math_mode, routed, ws)
+    torch.cuda.synchronize()
+    assert got.tobytes() == routed.cpu().numpy().tobytes()
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_fwd_mean_collapse_is_deterministic(math_mode):
+    spec = FWD_SPECS[3]
+    inp = wl.generate(spec)
+    a, _, _ = _run_fwd(spec, inp, math_mode)
+    b, _, _ = _run_fwd(spec, inp, math_mode)
+    assert a.tobytes() == b.tobytes()
+
+
+def test_fwd_mean_collapse_empty_batch_writes_nothing():
+    spec = wl.make_spec("mcf_empty", 0, 5, 4, 128, 59)
+    out = Guarded(0)
+    r = ops.Routing.empty(0, 4, "cuda")
+    ws = ops.new_workspace(0, 4, 128, "cuda")
+    W = torch.zeros(4, 128, 128, device="cuda")
+    b = torch.zeros(4, 128, device="cuda")
+    ops.moe_top1_fwd_mean_collapse(torch.empty(0, 128, device="cuda"), W, b, r, 0, 5, 4, 128, ops.MOE_MATH_TF32,
+                                   out.t, ws)
+    torch.cuda.synchronize()
+    assert out.guards_intact()
+
+
+def test_fwd_mean_collapse_full_size_sampled_rows():
+    """The 1,048,576-token workload (B 65536, N_H 16, E 8, H 256) through the gate,
+    as the benchmark runs it; 64 sampled rows against the oracle."""
+    from bwd_route_b200.gate import MoETop1Gate
+    spec = wl.WORKLOADS[wl.THROUGHPUT_WORKLOAD]
+    inp = wl.generate(spec)
+    gate = MoETop1Gate(dev(inp.W), dev(inp.bias), spec.B, spec.N_H, ops.MOE_MATH_TF32)
+    gate.route(dev(inp.gate_logits))
+    gate.forward_mean_collapse(dev(inp.x))
+    torch.cuda.synchronize()
+    assert ops.moe_top1_device_flags(gate.ws) == 0
+    rows = np.sort(np.random.default_rng(60).choice(spec.B, 64, replace=False))
+    tok = (rows[:, None] * spec.N_H + np.arange(spec.N_H)).reshape(-1)
+    idx = oracle.route(inp.gate_logits[tok])[0]
+    want, mag = oracle.fwd_mean_collapse(inp.x[tok], inp.W, inp.bias, idx, spec.N_H)
+    got = gate.ctx_mean[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64)
+    assert (np.abs(got - want) <= fwd_bound(spec, ops.MOE_MATH_TF32) * mag).all()
