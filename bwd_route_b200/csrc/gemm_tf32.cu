@@ -401,10 +401,20 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
 //   ctx_mean[b] = (1/N_H) (sum_e W[e] X_be + sum_e n_be bias[e]),
 // one dense GEMM per tile of 128 batch rows with K = E*H, accumulated in TMEM
 // over the experts in a fixed order: no sum crosses a CTA and no [T, H] array
-// is written. Warps 8-11 build X_be (K-major, 128-byte swizzle) in a 4-deep
-// ring from the rows of x; warp 13 streams W[e] by TMA exactly as the forward
-// does; one thread of warp 12 issues the MMAs into one of two accumulators;
-// warps 0-7 add the bias terms, scale by 1/N_H and store the rows.
+// is written. Warps 8-15 build X_be (K-major, 128-byte swizzle) in a 4-deep
+// ring from the rows of x: each thread owns 4 rows and loads up to 4 tokens of
+// each before adding any, so a stage costs about one memory latency; warp 17
+// streams W[e] by TMA exactly as the forward does; one thread of warp 16
+// issues the MMAs into one of two accumulators; warps 0-7 add the bias terms,
+// scale by 1/N_H and store the rows.
+constexpr int kThreadsHmean = 576;
+constexpr int kHProducer0 = 256;   // warps 8-15
+constexpr int kHProducers = 256;
+constexpr int kHMmaWarp = 16;
+constexpr int kHBLoadWarp = 17;
+constexpr int kHMaxHorizon = 32;   // horizon tokens per row (one bit each in a 32-bit mask)
+constexpr int kHTokAhead = 4;      // tokens of a row loaded before the first add
+
 struct __align__(8) HCtl {
     uint64_t afull[kMaxStages];
     uint64_t aempty[kMaxStages];
@@ -416,8 +426,6 @@ struct __align__(8) HCtl {
     int abort;
 };
 
-constexpr int kHMaxHorizon = 32;  // horizon tokens per row (one bit each in a 32-bit mask)
-
 template <int H>
 struct HCfg {
     static constexpr int BM = 128;
@@ -428,7 +436,7 @@ struct HCfg {
     static constexpr int B_STAGES = (H == 256) ? 3 : 4;
     static constexpr int RING_BYTES = A_STAGES * A_BYTES + B_STAGES * B_BYTES;
     static constexpr int BIAS_BYTES = 32 * H * 4;             // bias of up to 32 experts
-    static constexpr int IDX_BYTES = 4 * 32 * kHMaxHorizon;   // producer warp w: experts of its 32 rows
+    static constexpr int IDX_BYTES = 8 * 16 * kHMaxHorizon;   // producer warp w: experts of its 16 rows
     static constexpr int CNT_BYTES = kGEpiWarps * 32 * 32;    // epilogue lane: tokens per expert of its row
     static constexpr int TMEM_COLS = 2 * H;
     static constexpr int SMEM_BYTES =
@@ -438,7 +446,7 @@ struct HCfg {
 };
 
 template <int H>
-__global__ void __launch_bounds__(kThreadsGrouped, 1)
+__global__ void __launch_bounds__(kThreadsHmean, 1)
 hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUtensorMap tm_b,
                       const float* __restrict__ bias, const int32_t* __restrict__ expert_idx, int B, int N_H, int E,
                       float inv_nh, float* __restrict__ out, uint32_t* __restrict__ dev_flags) {
@@ -454,8 +462,8 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::A_STAGES; ++s) {
-            mbar_init(&ctl->afull[s], 128);  // 128 producer threads
-            mbar_init(&ctl->aempty[s], 1);   // tcgen05.commit
+            mbar_init(&ctl->afull[s], kHProducers);  // every producer thread
+            mbar_init(&ctl->aempty[s], 1);           // tcgen05.commit
         }
         for (int s = 0; s < C::B_STAGES; ++s) {
             mbar_init(&ctl->bfull[s], 1);    // arrive.expect_tx + TMA bytes
@@ -470,8 +478,8 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
     }
     for (int k = threadIdx.x; k < E * H / 4; k += blockDim.x)
         reinterpret_cast<float4*>(bias_s)[k] = __ldg(reinterpret_cast<const float4*>(bias) + k);
-    if (warp == kGBLoadWarp && lane == 0) tma_prefetch_desc(&tm_b);
-    if (warp == kGMmaWarp) {
+    if (warp == kHBLoadWarp && lane == 0) tma_prefetch_desc(&tm_b);
+    if (warp == kHMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -482,32 +490,33 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
     const int ntiles = (B + C::BM - 1) / C::BM;
     volatile int* abort = &ctl->abort;
 
-    if (warp >= kGProducer0 / 32 && warp < kGProducer0 / 32 + 4) {
+    if (warp >= kHProducer0 / 32 && warp < (kHProducer0 + kHProducers) / 32) {
         // ---------------- producers: X_be for 128 rows x one 32-column k-chunk per stage.
-        // Thread (prow, pg) owns rows r = it * 16 + prow (it = 0..7) and the 16-byte
+        // Thread (prow, pg) owns rows r = it * 32 + prow (it = 0..3) and the 16-byte
         // granule pg of each; warp pw's rows are the prow values 4 pw .. 4 pw + 3, and
         // it keeps their experts in its own block of idx_s (warp-local row rl = 4 it + lane / 8).
-        const int pw = warp - kGProducer0 / 32;
-        const int ptid = threadIdx.x - kGProducer0;
+        const int pw = warp - kHProducer0 / 32;
+        const int ptid = threadIdx.x - kHProducer0;
         const int prow = ptid >> 3, pg = ptid & 7;
-        uint8_t* sidx = idx_s + pw * 32 * kHMaxHorizon;
+        uint8_t* sidx = idx_s + pw * 16 * kHMaxHorizon;
         int sa = 0;
         uint32_t pa = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
             const int b0 = tile * C::BM;
             __syncwarp();
-            for (int k = lane; k < 32 * N_H; k += 32) {
+#pragma unroll 4
+            for (int k = lane; k < 16 * N_H; k += 32) {
                 const int rl = k / N_H, h = k - rl * N_H;
-                const int b = b0 + (rl >> 2) * 16 + pw * 4 + (rl & 3);
+                const int b = b0 + (rl >> 2) * 32 + pw * 4 + (rl & 3);
                 const int e = (b < B) ? expert_idx[static_cast<int64_t>(b) * N_H + h] : -1;
                 sidx[rl * kHMaxHorizon + h] = (e >= 0 && e < E) ? static_cast<uint8_t>(e) : uint8_t{0xFF};
             }
             __syncwarp();
             for (int e = 0; e < E && ok; ++e) {
-                uint32_t mask[8];  // bit h: horizon token h of the row chose expert e
+                uint32_t mask[4];  // bit h: horizon token h of the row chose expert e
 #pragma unroll
-                for (int it = 0; it < 8; ++it) {
+                for (int it = 0; it < 4; ++it) {
                     const uint8_t* row = sidx + (it * 4 + (lane >> 3)) * kHMaxHorizon;
                     uint32_t m = 0;
                     for (int h = 0; h < N_H; ++h) m |= static_cast<uint32_t>(row[h] == e) << h;
@@ -517,44 +526,46 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
                     ok = mbar_wait(&ctl->aempty[sa], pa ^ 1, abort, dev_flags);
                     if (!(ok = __all_sync(0xffffffffu, ok))) break;
                     const float* xk = x + kc * 32 + pg * 4;
-                    // the first two tokens of every row are loaded before any is added, so
-                    // that 16 loads per thread are in flight; later tokens (rare) follow
-                    float4 v0[8], v1[8];
-                    uint32_t rest[8];
+                    float4 v[4][kHTokAhead];
 #pragma unroll
-                    for (int it = 0; it < 8; ++it) {
-                        const int64_t t0 = static_cast<int64_t>(b0 + it * 16 + prow) * N_H;
+                    for (int it = 0; it < 4; ++it) {
+                        const int64_t t0 = static_cast<int64_t>(b0 + it * 32 + prow) * N_H;
                         uint32_t m = mask[it];
-                        v0[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        v1[it] = v0[it];
-                        if (m) {
-                            v0[it] = __ldcs(reinterpret_cast<const float4*>(xk + (t0 + __ffs(m) - 1) * H));
-                            m &= m - 1;
+#pragma unroll
+                        for (int j = 0; j < kHTokAhead; ++j) {
+                            v[it][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (m) {
+                                v[it][j] = __ldcs(reinterpret_cast<const float4*>(xk + (t0 + __ffs(m) - 1) * H));
+                                m &= m - 1;
+                            }
                         }
-                        if (m) {
-                            v1[it] = __ldcs(reinterpret_cast<const float4*>(xk + (t0 + __ffs(m) - 1) * H));
-                            m &= m - 1;
-                        }
-                        rest[it] = m;
                     }
                     const uint32_t a_u32 = smem_u32(aring + sa * C::A_BYTES);
 #pragma unroll
-                    for (int it = 0; it < 8; ++it) {
-                        const int r = it * 16 + prow;
-                        float4 acc = v0[it];
-                        if (mask[it] & (mask[it] - 1)) {  // a second token
-                            acc.x += v1[it].x;
-                            acc.y += v1[it].y;
-                            acc.z += v1[it].z;
-                            acc.w += v1[it].w;
+                    for (int it = 0; it < 4; ++it) {
+                        const int r = it * 32 + prow;
+                        const int n = __popc(mask[it]);
+                        float4 acc = v[it][0];
+#pragma unroll
+                        for (int j = 1; j < kHTokAhead; ++j) {
+                            if (j < n) {
+                                acc.x += v[it][j].x;
+                                acc.y += v[it][j].y;
+                                acc.z += v[it][j].z;
+                                acc.w += v[it][j].w;
+                            }
                         }
-                        const int64_t t0 = static_cast<int64_t>(b0 + r) * N_H;
-                        for (uint32_t m = rest[it]; m; m &= m - 1) {
-                            const float4 u = __ldcs(reinterpret_cast<const float4*>(xk + (t0 + __ffs(m) - 1) * H));
-                            acc.x += u.x;
-                            acc.y += u.y;
-                            acc.z += u.z;
-                            acc.w += u.w;
+                        if (n > kHTokAhead) {  // rare: more tokens of this expert than were loaded ahead
+                            uint32_t m = mask[it];
+                            for (int j = 0; j < kHTokAhead; ++j) m &= m - 1;
+                            const int64_t t0 = static_cast<int64_t>(b0 + r) * N_H;
+                            for (; m; m &= m - 1) {
+                                const float4 u = __ldcs(reinterpret_cast<const float4*>(xk + (t0 + __ffs(m) - 1) * H));
+                                acc.x += u.x;
+                                acc.y += u.y;
+                                acc.z += u.z;
+                                acc.w += u.w;
+                            }
                         }
                         st_shared_v4(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), acc.x, acc.y, acc.z, acc.w);
                     }
@@ -567,7 +578,7 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
                 }
             }
         }
-    } else if (warp == kGBLoadWarp) {
+    } else if (warp == kHBLoadWarp) {
         // ---------------- W[e] k-chunks by TMA, in the producers' (e, kc) order
         if (lane == 0) {
             int sb = 0;
@@ -588,7 +599,7 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
             }
         }
         __syncwarp();
-    } else if (warp == kGMmaWarp) {
+    } else if (warp == kHMmaWarp) {
         // ---------------- MMA issuer (one thread): D = sum over (e, kc) of X_be W[e]^T
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_tf32(128, H, 0, 0);
@@ -649,6 +660,7 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
 #pragma unroll
             for (int k = 0; k < 8; ++k) reinterpret_cast<uint32_t*>(cnt)[k] = 0u;
             if (b < B) {
+#pragma unroll 4
                 for (int h = 0; h < N_H; ++h) {
                     const int e = expert_idx[static_cast<int64_t>(b) * N_H + h];
                     if (e >= 0 && e < E) cnt[e] += 1;
@@ -658,16 +670,16 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < HALF / 64; ++cc) {
-                float v[64];
-                tmem_ld_32x32b_x64(tmem + (static_cast<uint32_t>(32 * q) << 16) +
-                                       static_cast<uint32_t>(acc * H + c0 + cc * 64), v);
+            for (int cc = 0; cc < HALF / 32; ++cc) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) +
+                                       static_cast<uint32_t>(acc * H + c0 + cc * 32), v);
                 for (int e = 0; e < E; ++e) {
                     const float n = static_cast<float>(cnt[e]);
                     if (!__any_sync(0xffffffffu, n != 0.0f)) continue;
-                    const float4* bs = reinterpret_cast<const float4*>(bias_s + e * H + c0 + cc * 64);
+                    const float4* bs = reinterpret_cast<const float4*>(bias_s + e * H + c0 + cc * 32);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
+                    for (int j = 0; j < 8; ++j) {
                         const float4 bb = bs[j];
                         v[4 * j] = fmaf(n, bb.x, v[4 * j]);
                         v[4 * j + 1] = fmaf(n, bb.y, v[4 * j + 1]);
@@ -676,9 +688,9 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
                     }
                 }
                 if (b < B) {
-                    float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * H + c0 + cc * 64);
+                    float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * H + c0 + cc * 32);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
+                    for (int j = 0; j < 8; ++j)
                         __stcs(dst + j, make_float4(v[4 * j] * inv_nh, v[4 * j + 1] * inv_nh, v[4 * j + 2] * inv_nh,
                                                     v[4 * j + 3] * inv_nh));
                 }
@@ -692,7 +704,7 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kGMmaWarp) {
+    if (warp == kHMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -988,10 +1000,10 @@ cudaError_t launch_hmean_fwd_tf32(const float* x, const float* W, const float* b
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     const float inv_nh = static_cast<float>(1.0 / static_cast<double>(N_H));
     if (H == 256)
-        hmean_fwd_tf32_kernel<256><<<grid, kThreadsGrouped, HCfg<256>::SMEM_BYTES, s>>>(
+        hmean_fwd_tf32_kernel<256><<<grid, kThreadsHmean, HCfg<256>::SMEM_BYTES, s>>>(
             x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
     else
-        hmean_fwd_tf32_kernel<128><<<grid, kThreadsGrouped, HCfg<128>::SMEM_BYTES, s>>>(
+        hmean_fwd_tf32_kernel<128><<<grid, kThreadsHmean, HCfg<128>::SMEM_BYTES, s>>>(
             x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
     return cudaGetLastError();
 }
