@@ -522,6 +522,17 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
                     for (int h = 0; h < N_H; ++h) m |= static_cast<uint32_t>(row[h] == e) << h;
                     mask[it] = m;
                 }
+                // the k-chunks of a token row are consumed one stage apart: fetch each
+                // matching row whole into L2 now (the row's 8 granule threads take one
+                // 128-byte chunk each), so that stages kc >= 1 read it from L2
+                if (pg < C::KCH) {
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int64_t t0 = static_cast<int64_t>(b0 + it * 32 + prow) * N_H;
+                        for (uint32_t m = mask[it]; m; m &= m - 1)
+                            prefetch_l2(x + (t0 + __ffs(m) - 1) * H + pg * 32);
+                    }
+                }
                 for (int kc = 0; kc < C::KCH; ++kc) {
                     ok = mbar_wait(&ctl->aempty[sa], pa ^ 1, abort, dev_flags);
                     if (!(ok = __all_sync(0xffffffffu, ok))) break;
