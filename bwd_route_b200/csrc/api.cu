@@ -6,6 +6,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "hmean.h"
 #include "internal.h"
 #include "moe_top1.h"
 
@@ -42,6 +43,7 @@ cudaError_t device_info(DeviceInfo** out) {
         e = aux_set_smem_limits();
         if (e == cudaSuccess) e = route_set_smem_limits();
         if (e == cudaSuccess) e = tf32_set_smem_limits();
+        if (e == cudaSuccess) e = hmean_set_smem_limits();
         if (e != cudaSuccess) return e;
         d.aux_ready = true;
     }

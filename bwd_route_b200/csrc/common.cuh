@@ -113,11 +113,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Hint: bring the 128-byte line at p into L2 (no data returned, no fault
-// semantics relied on: p always points into a live buffer here).
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
 // Orders shared-memory data observed by this thread (written through the
 // generic proxy, e.g. by cp.async) before its later tensor-core reads.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -15,6 +15,7 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "hmean.h"
 #include "internal.h"
 
 namespace moe {

@@ -1,0 +1,381 @@
+// gemm_tf32_hmean.cu -- the forward through the horizon mean on tcgen05 TF32
+// tensor cores ("Single source of truth for the attention path", MHA
+// additions: the gate's output [B, N_H, H] is averaged over the horizon axis
+// into ctx_mean [B, H]), in a translation unit of its own.
+#include <cstdint>
+
+#include "common.cuh"
+#include "hmean.h"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxStages = 8;
+constexpr int kGEpiWarps = 8;  // epilogue warps 0-7: warp w drains TMEM lane quadrant w % 4
+
+// Hint: bring the 128-byte line at p into L2 (p always points into a live
+// buffer here; no data is returned).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// ------------------------------------------------------------------ forward through the horizon mean
+// ctx_mean[b] = (1/N_H) sum_h (W[e_bh] x[b,h] + bias[e_bh]) ("Single source of
+// truth for the attention path", MHA additions: the gate's output is averaged
+// over the horizon axis). The horizon tokens of row b that chose expert e are
+// summed first, X_be = sum_{h : e_bh = e} x[b,h] (ascending h, fp32), so
+//   ctx_mean[b] = (1/N_H) (sum_e W[e] X_be + sum_e n_be bias[e]),
+// one dense GEMM per tile of 128 batch rows with K = E*H, accumulated in TMEM
+// over the experts in a fixed order: no sum crosses a CTA and no [T, H] array
+// is written. Warps 8-15 build X_be (K-major, 128-byte swizzle) in a 4-deep
+// ring from the rows of x: each thread owns 4 rows and loads up to 4 tokens of
+// each before adding any, so a stage costs about one memory latency; warp 17
+// streams W[e] by TMA exactly as the forward does; one thread of warp 16
+// issues the MMAs into one of two accumulators; warps 0-7 add the bias terms,
+// scale by 1/N_H and store the rows.
+constexpr int kThreadsHmean = 576;
+constexpr int kHProducer0 = 256;   // warps 8-15
+constexpr int kHProducers = 256;
+constexpr int kHMmaWarp = 16;
+constexpr int kHBLoadWarp = 17;
+constexpr int kHMaxHorizon = 32;   // horizon tokens per row (one bit each in a 32-bit mask)
+constexpr int kHTokAhead = 4;      // tokens of a row loaded before the first add
+
+struct __align__(8) HCtl {
+    uint64_t afull[kMaxStages];
+    uint64_t aempty[kMaxStages];
+    uint64_t bfull[kMaxStages];
+    uint64_t bempty[kMaxStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int H>
+struct HCfg {
+    static constexpr int BM = 128;
+    static constexpr int KCH = H / 32;
+    static constexpr int A_BYTES = BM * 128;                  // 16 KiB
+    static constexpr int B_BYTES = H * 128;                   // 16 / 32 KiB
+    static constexpr int A_STAGES = 4;
+    static constexpr int B_STAGES = (H == 256) ? 3 : 4;
+    static constexpr int RING_BYTES = A_STAGES * A_BYTES + B_STAGES * B_BYTES;
+    static constexpr int BIAS_BYTES = 32 * H * 4;             // bias of up to 32 experts
+    static constexpr int IDX_BYTES = 8 * 16 * kHMaxHorizon;   // producer warp w: experts of its 16 rows
+    static constexpr int CNT_BYTES = kGEpiWarps * 32 * 32;    // epilogue lane: tokens per expert of its row
+    static constexpr int TMEM_COLS = 2 * H;
+    static constexpr int SMEM_BYTES =
+        1024 + RING_BYTES + BIAS_BYTES + IDX_BYTES + CNT_BYTES + static_cast<int>(sizeof(HCtl));
+    static_assert(A_STAGES <= kMaxStages && B_STAGES <= kMaxStages, "stages");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <int H>
+__global__ void __launch_bounds__(kThreadsHmean, 1)
+hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUtensorMap tm_b,
+                      const float* __restrict__ bias, const int32_t* __restrict__ expert_idx, int B, int N_H, int E,
+                      float inv_nh, float* __restrict__ out, uint32_t* __restrict__ dev_flags) {
+    using C = HCfg<H>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* aring = smem;
+    uint8_t* bring = smem + C::A_STAGES * C::A_BYTES;
+    float* bias_s = reinterpret_cast<float*>(smem + C::RING_BYTES);
+    uint8_t* idx_s = smem + C::RING_BYTES + C::BIAS_BYTES;
+    uint8_t* cnt_s = idx_s + C::IDX_BYTES;
+    HCtl* ctl = reinterpret_cast<HCtl*>(cnt_s + C::CNT_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::A_STAGES; ++s) {
+            mbar_init(&ctl->afull[s], kHProducers);  // every producer thread
+            mbar_init(&ctl->aempty[s], 1);           // tcgen05.commit
+        }
+        for (int s = 0; s < C::B_STAGES; ++s) {
+            mbar_init(&ctl->bfull[s], 1);    // arrive.expect_tx + TMA bytes
+            mbar_init(&ctl->bempty[s], 1);   // tcgen05.commit
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], kGEpiWarps);
+        }
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    for (int k = threadIdx.x; k < E * H / 4; k += blockDim.x)
+        reinterpret_cast<float4*>(bias_s)[k] = __ldg(reinterpret_cast<const float4*>(bias) + k);
+    if (warp == kHBLoadWarp && lane == 0) tma_prefetch_desc(&tm_b);
+    if (warp == kHMmaWarp) {
+        tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    const int ntiles = (B + C::BM - 1) / C::BM;
+    volatile int* abort = &ctl->abort;
+
+    if (warp >= kHProducer0 / 32 && warp < (kHProducer0 + kHProducers) / 32) {
+        // ---------------- producers: X_be for 128 rows x one 32-column k-chunk per stage.
+        // Thread (prow, pg) owns rows r = it * 32 + prow (it = 0..3) and the 16-byte
+        // granule pg of each; warp pw's rows are the prow values 4 pw .. 4 pw + 3, and
+        // it keeps their experts in its own block of idx_s (warp-local row rl = 4 it + lane / 8).
+        const int pw = warp - kHProducer0 / 32;
+        const int ptid = threadIdx.x - kHProducer0;
+        const int prow = ptid >> 3, pg = ptid & 7;
+        uint8_t* sidx = idx_s + pw * 16 * kHMaxHorizon;
+        int sa = 0;
+        uint32_t pa = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            const int b0 = tile * C::BM;
+            __syncwarp();
+#pragma unroll 4
+            for (int k = lane; k < 16 * N_H; k += 32) {
+                const int rl = k / N_H, h = k - rl * N_H;
+                const int b = b0 + (rl >> 2) * 32 + pw * 4 + (rl & 3);
+                const int e = (b < B) ? expert_idx[static_cast<int64_t>(b) * N_H + h] : -1;
+                sidx[rl * kHMaxHorizon + h] = (e >= 0 && e < E) ? static_cast<uint8_t>(e) : uint8_t{0xFF};
+            }
+            __syncwarp();
+            for (int e = 0; e < E && ok; ++e) {
+                uint32_t mask[4];  // bit h: horizon token h of the row chose expert e
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const uint8_t* row = sidx + (it * 4 + (lane >> 3)) * kHMaxHorizon;
+                    uint32_t m = 0;
+                    for (int h = 0; h < N_H; ++h) m |= static_cast<uint32_t>(row[h] == e) << h;
+                    mask[it] = m;
+                }
+                // the k-chunks of a token row are consumed one stage apart: fetch each
+                // matching row whole into L2 now (the row's 8 granule threads take one
+                // 128-byte chunk each), so that stages kc >= 1 read it from L2
+                if (pg < C::KCH) {
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int64_t t0 = static_cast<int64_t>(b0 + it * 32 + prow) * N_H;
+                        for (uint32_t m = mask[it]; m; m &= m - 1)
+                            prefetch_l2(x + (t0 + __ffs(m) - 1) * H + pg * 32);
+                    }
+                }
+                for (int kc = 0; kc < C::KCH; ++kc) {
+                    ok = mbar_wait(&ctl->aempty[sa], pa ^ 1, abort, dev_flags);
+                    if (!(ok = __all_sync(0xffffffffu, ok))) break;
+                    const float* xk = x + kc * 32 + pg * 4;
+                    float4 v[4][kHTokAhead];
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int64_t t0 = static_cast<int64_t>(b0 + it * 32 + prow) * N_H;
+                        uint32_t m = mask[it];
+#pragma unroll
+                        for (int j = 0; j < kHTokAhead; ++j) {
+                            v[it][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (m) {
+                                v[it][j] = __ldcs(reinterpret_cast<const float4*>(xk + (t0 + __ffs(m) - 1) * H));
+                                m &= m - 1;
+                            }
+                        }
+                    }
+                    const uint32_t a_u32 = smem_u32(aring + sa * C::A_BYTES);
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int r = it * 32 + prow;
+                        const int n = __popc(mask[it]);
+                        float4 acc = v[it][0];
+#pragma unroll
+                        for (int j = 1; j < kHTokAhead; ++j) {
+                            if (j < n) {
+                                acc.x += v[it][j].x;
+                                acc.y += v[it][j].y;
+                                acc.z += v[it][j].z;
+                                acc.w += v[it][j].w;
+                            }
+                        }
+                        if (n > kHTokAhead) {  // rare: more tokens of this expert than were loaded ahead
+                            uint32_t m = mask[it];
+                            for (int j = 0; j < kHTokAhead; ++j) m &= m - 1;
+                            const int64_t t0 = static_cast<int64_t>(b0 + r) * N_H;
+                            for (; m; m &= m - 1) {
+                                const float4 u = __ldcs(reinterpret_cast<const float4*>(xk + (t0 + __ffs(m) - 1) * H));
+                                acc.x += u.x;
+                                acc.y += u.y;
+                                acc.z += u.z;
+                                acc.w += u.w;
+                            }
+                        }
+                        st_shared_v4(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), acc.x, acc.y, acc.z, acc.w);
+                    }
+                    fence_proxy_async_smem();  // the MMA reads these stores through the async proxy
+                    mbar_arrive(&ctl->afull[sa]);
+                    if (++sa == C::A_STAGES) {
+                        sa = 0;
+                        pa ^= 1;
+                    }
+                }
+            }
+        }
+    } else if (warp == kHBLoadWarp) {
+        // ---------------- W[e] k-chunks by TMA, in the producers' (e, kc) order
+        if (lane == 0) {
+            int sb = 0;
+            uint32_t pb = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                for (int e = 0; e < E && ok; ++e) {
+                    for (int kc = 0; kc < C::KCH; ++kc) {
+                        if (!(ok = mbar_wait(&ctl->bempty[sb], pb ^ 1, abort, dev_flags))) break;
+                        mbar_arrive_expect_tx(&ctl->bfull[sb], C::B_BYTES);
+                        tma_load_2d(bring + sb * C::B_BYTES, &tm_b, kc * 32, e * H, &ctl->bfull[sb]);
+                        if (++sb == C::B_STAGES) {
+                            sb = 0;
+                            pb ^= 1;
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kHMmaWarp) {
+        // ---------------- MMA issuer (one thread): D = sum over (e, kc) of X_be W[e]^T
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_tf32(128, H, 0, 0);
+            int sa = 0, sb = 0;
+            uint32_t pa = 0, pb = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                if (!(ok = mbar_wait(&ctl->tempty[acc], acc_phase ^ 1, abort, dev_flags))) break;
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(acc * H);
+                uint32_t accumulate = 0;
+                for (int e = 0; e < E && ok; ++e) {
+                    for (int kc = 0; kc < C::KCH; ++kc) {
+                        if (!(ok = mbar_wait(&ctl->afull[sa], pa, abort, dev_flags))) break;
+                        if (!(ok = mbar_wait(&ctl->bfull[sb], pb, abort, dev_flags))) break;
+                        fence_proxy_async_smem();
+                        tc_fence_after();
+                        const uint32_t a_addr = smem_u32(aring + sa * C::A_BYTES);
+                        const uint32_t b_addr = smem_u32(bring + sb * C::B_BYTES);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            mma_tf32(d, sw128_desc(a_addr + ks * 32, 16, 1024), sw128_desc(b_addr + ks * 32, 16, 1024),
+                                     idesc, accumulate);
+                            accumulate = 1u;
+                        }
+                        mma_commit(&ctl->aempty[sa]);
+                        mma_commit(&ctl->bempty[sb]);
+                        if (++sa == C::A_STAGES) {
+                            sa = 0;
+                            pa ^= 1;
+                        }
+                        if (++sb == C::B_STAGES) {
+                            sb = 0;
+                            pb ^= 1;
+                        }
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+        }
+        __syncwarp();
+    } else if (warp < kGEpiWarps) {
+        // ---------------- epilogue: row b = lane of TMEM quadrant q; column half c0.
+        // (acc + sum_e n_be bias[e]) / N_H, n_be counted from the row's experts.
+        constexpr int HALF = H / 2;
+        const int q = warp & 3;
+        const int c0 = (warp >> 2) * HALF;
+        uint8_t* cnt = cnt_s + (warp * 32 + lane) * 32;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int b = tile * C::BM + 32 * q + lane;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) reinterpret_cast<uint32_t*>(cnt)[k] = 0u;
+            if (b < B) {
+#pragma unroll 4
+                for (int h = 0; h < N_H; ++h) {
+                    const int e = expert_idx[static_cast<int64_t>(b) * N_H + h];
+                    if (e >= 0 && e < E) cnt[e] += 1;
+                }
+            }
+            bool ok = mbar_wait(&ctl->tfull[acc], acc_phase, abort, dev_flags);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < HALF / 32; ++cc) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) +
+                                       static_cast<uint32_t>(acc * H + c0 + cc * 32), v);
+                for (int e = 0; e < E; ++e) {
+                    const float n = static_cast<float>(cnt[e]);
+                    if (!__any_sync(0xffffffffu, n != 0.0f)) continue;
+                    const float4* bs = reinterpret_cast<const float4*>(bias_s + e * H + c0 + cc * 32);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 bb = bs[j];
+                        v[4 * j] = fmaf(n, bb.x, v[4 * j]);
+                        v[4 * j + 1] = fmaf(n, bb.y, v[4 * j + 1]);
+                        v[4 * j + 2] = fmaf(n, bb.z, v[4 * j + 2]);
+                        v[4 * j + 3] = fmaf(n, bb.w, v[4 * j + 3]);
+                    }
+                }
+                if (b < B) {
+                    float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * H + c0 + cc * 32);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        __stcs(dst + j, make_float4(v[4 * j] * inv_nh, v[4 * j + 1] * inv_nh, v[4 * j + 2] * inv_nh,
+                                                    v[4 * j + 3] * inv_nh));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kHMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+cudaError_t launch_hmean_fwd_tf32(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
+                                  int64_t B, int N_H, int E, int H, float* out, uint32_t* dev_flags, int num_sms,
+                                  cudaStream_t s) {
+    CUtensorMap tm_b;
+    if (!make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, H)) return cudaErrorInvalidValue;
+    const int64_t tiles = (B + 127) / 128;
+    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    const float inv_nh = static_cast<float>(1.0 / static_cast<double>(N_H));
+    if (H == 256)
+        hmean_fwd_tf32_kernel<256><<<grid, kThreadsHmean, HCfg<256>::SMEM_BYTES, s>>>(
+            x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
+    else
+        hmean_fwd_tf32_kernel<128><<<grid, kThreadsHmean, HCfg<128>::SMEM_BYTES, s>>>(
+            x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
+    return cudaGetLastError();
+}
+
+cudaError_t hmean_set_smem_limits() {
+    cudaError_t e = set_smem(hmean_fwd_tf32_kernel<256>, HCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(hmean_fwd_tf32_kernel<128>, HCfg<128>::SMEM_BYTES);
+    return e;
+}
+
+}  // namespace moe

@@ -108,13 +108,6 @@ cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t*
                               cudaStream_t s);
 // Fixed-order pairwise sum of the slots of each expert, times scale, into dW / db
 // (either may be null).
-// Forward through the horizon mean: ctx_mean [B, H] from x [B * N_H, H] and the
-// routing's expert_idx (N_H <= 32).
-cudaError_t launch_hmean_fwd_tf32(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
-                                  int64_t B, int N_H, int E, int H, float* out, uint32_t* dev_flags, int num_sms,
-                                  cudaStream_t s);
-cudaError_t launch_hmean_fwd_ffma(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
-                                  int64_t B, int N_H, int E, int H, float* out, cudaStream_t s);
 cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const int32_t* offsets, int64_t T,
                                 int E, int H, float scale, float* dW, float* db, int acc_dw, int acc_db,
                                 cudaStream_t s);
