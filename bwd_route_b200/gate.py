@@ -11,6 +11,11 @@ source of truth for the attention path", PerceptionTrainer integration):
 forward through the MoE dispatch, backward through it, then the load-balance
 loss, whose weight lambda_eff is read from device memory and updated by the
 controller of foxhunt commit 2d0e6b6bdc at the end of the step.
+
+Beside step(): forward_mean_collapse / backward_mean_collapse when the gate's
+output is averaged over the horizon axis (ctx_mean [B, H]); update_controller,
+which produces ent_ema from the step's expert usage and recomputes lambda_eff;
+and, for data-parallel jobs, enable_data_parallel / allreduce_gradients.
 """
 from __future__ import annotations
 

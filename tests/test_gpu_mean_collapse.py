@@ -1,5 +1,6 @@
-"""GPU parity of the backward with the horizon mean folded in
-(moe_top1_bwd_mean_collapse) against the oracle, in both math modes."""
+"""GPU parity of the horizon mean [B, N_H, H] -> [B, H] folded into the gate,
+against the oracle in both math modes: the backward (moe_top1_bwd_mean_collapse)
+and the forward (moe_top1_fwd_mean_collapse)."""
 import numpy as np
 import pytest
 import torch
