@@ -10,14 +10,11 @@
 // nothing but its inputs and outputs. The routing kernels are the same ones
 // moe_top1_route launches.
 #include <cstdint>
-#include <mutex>
 
 #include "internal.h"
 #include "moe_top1.h"
 
 namespace moe {
-
-cudaError_t route_set_smem_limits();  // route.cu
 
 namespace {
 
@@ -29,30 +26,21 @@ static_assert(MOE_NOALLOC_MAX_TOKENS % kRouteTokPerBlk == 0, "whole routing bloc
 // int32 = 512 KiB. Every GPU that loads the library holds this until the
 // process exits. Host code must not use the array's name as a device address
 // (on the host it is only a stand-in); it uses the address that
-// cudaGetSymbolAddress returns for the current device.
+// cudaGetSymbolAddress returns in the current context.
 static __device__ __align__(256) int32_t g_route_scratch[2 * kNoAllocMaxBlocks * kNoAllocMaxExperts];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-int32_t* g_scratch[kMaxDevices] = {};
-
-// First call on a device: look up the scratch address and set the routing
-// kernels' shared-memory limits, with that device current.
-cudaError_t scratch_of_current_device(int32_t** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+// The array's device address in the CUDA context current on the calling thread.
+// A module-scope __device__ variable has one copy per context that loads the
+// library's module, and that copy's address belongs to the context: a context
+// created after a cudaDeviceReset, or a non-primary context a host made current
+// on the same device, has its own copy at its own address. So the address is
+// looked up on every call (a host-side table lookup that allocates nothing and
+// enqueues no work) instead of being cached per device number.
+cudaError_t scratch_of_current_context(int32_t** out) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_route_scratch);
-        if (e != cudaSuccess) return e;
-        e = route_set_smem_limits();
-        if (e != cudaSuccess) return e;
-        g_scratch[dev] = static_cast<int32_t*>(p);
-    }
-    *out = g_scratch[dev];
+    *out = static_cast<int32_t*>(p);
     return cudaSuccess;
 }
 
@@ -95,7 +83,7 @@ extern "C" moe_status_t moe_top1_route_noalloc(const float* gate_logits, int64_t
         return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
     int32_t* scratch = nullptr;
-    if (scratch_of_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    if (scratch_of_current_context(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
     // The count kernel writes every per-block count the scan reads, and the scan
     // writes every base the scatter reads: nothing in the scratch has to start at 0.
     const int64_t nblk = (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk;

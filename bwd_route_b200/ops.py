@@ -20,6 +20,7 @@ MOE_MATH_TF32 = 0
 MOE_MATH_FFMA = 1
 MOE_ACC_DX, MOE_ACC_DW, MOE_ACC_DB = 0x1, 0x2, 0x4
 MOE_FLAG_WAIT_TIMEOUT = 0x1
+MOE_FLAG_BAD_ROUTING = 0x2
 
 _STATUS = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED_SHAPE", "MOE_ERR_MISALIGNED",
            "MOE_ERR_ALIAS", "MOE_ERR_WORKSPACE", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_CHECK"]
@@ -30,6 +31,7 @@ EXPORTED = [
     "moe_top1_bwd", "moe_aux_loss_fwd_bwd", "moe_lambda_eff_update", "moe_top1_device_flags",
     "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc", "moe_top1_selftest_wait_timeout",
     "moe_usage_entropy_ema_update", "moe_top1_bwd_mean_collapse", "moe_top1_fwd_mean_collapse",
+    "moe_top1_check_routing",
 ]
 MOE_NOALLOC_MAX_TOKENS = 2097152
 
@@ -91,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.moe_top1_selftest_wait_timeout.argtypes = [P, SZ, I64, P]
         L.moe_usage_entropy_ema_update.restype = I32
         L.moe_usage_entropy_ema_update.argtypes = [P, I64, I32, ctypes.c_float, I32, P, P, P, P]
+        L.moe_top1_check_routing.restype = I32
+        L.moe_top1_check_routing.argtypes = [ctypes.POINTER(RoutingC), I64, I32, P, SZ, P]
         L.moe_top1_route_noalloc.restype = I32
         L.moe_top1_route_noalloc.argtypes = [P, I64, I64, I32, ctypes.POINTER(RoutingC), P]
         _lib = L
@@ -176,6 +180,14 @@ def moe_top1_route_noalloc(gate_logits: torch.Tensor, B: int, N_H: int, E: int, 
     rc = routing.c()
     _check("moe_top1_route_noalloc", lib().moe_top1_route_noalloc(_ptr(gate_logits, torch.float32), B, N_H, E,
                                                                   ctypes.byref(rc), _stream(stream)))
+
+
+def moe_top1_check_routing(routing: Routing, T: int, E: int, ws: torch.Tensor, stream=None):
+    """Enqueues the check of a routing not produced by moe_top1_route; a malformed
+    one sets MOE_FLAG_BAD_ROUTING in the workspace flag word (moe_top1_device_flags)."""
+    rc = routing.c()
+    _check("moe_top1_check_routing", lib().moe_top1_check_routing(ctypes.byref(rc), T, E, _ptr(ws), ws.numel(),
+                                                                  _stream(stream)))
 
 
 def moe_top1_fwd(x, W, bias, routing: Routing, B: int, N_H: int, E: int, H: int, math: int, routed,

@@ -56,8 +56,10 @@ extern "C" {
 /* 1: routing, forward, backward, aux loss, lambda update.
  * 2: adds moe_usage_entropy_ema_update and moe_top1_bwd_mean_collapse (every
  *    version-1 call is unchanged).
- * 3: adds moe_top1_fwd_mean_collapse (every earlier call is unchanged). */
-#define MOE_TOP1_ABI_VERSION 3
+ * 3: adds moe_top1_fwd_mean_collapse (every earlier call is unchanged).
+ * 4: adds moe_top1_check_routing and MOE_FLAG_BAD_ROUTING (every earlier call is
+ *    unchanged). */
+#define MOE_TOP1_ABI_VERSION 4
 
 typedef enum {
     MOE_OK = 0,
@@ -77,6 +79,7 @@ typedef enum {
 
 /* Bits of the device flag word. */
 #define MOE_FLAG_WAIT_TIMEOUT 0x1u  /* a pipeline wait ran past its bound */
+#define MOE_FLAG_BAD_ROUTING  0x2u  /* moe_top1_check_routing found a malformed routing */
 
 /* Routing result: caller-owned device buffers. The forward, backward and aux
  * entry points take a routing as an input and trust it: it must be what
@@ -84,7 +87,8 @@ typedef enum {
  * contraction kernels index activations with offsets and perm without checking
  * them again (a check per token costs about 5 % of their time), so a routing
  * from anywhere else -- an uninitialised buffer, another batch -- can make them
- * read and write outside the arrays. */
+ * read and write outside the arrays. A caller that builds or receives a routing
+ * some other way checks it first with moe_top1_check_routing. */
 typedef struct {
     int32_t* expert_idx; /* [T]     selected expert of each token */
     int32_t* counts;     /* [E]     tokens routed to each expert */
@@ -124,9 +128,12 @@ moe_status_t moe_top1_route(const float* gate_logits, int64_t B, int64_t N_H, in
  * 512 KiB on every GPU that loads the library, held until the process exits.
  * Limits: T = B * N_H <= MOE_NOALLOC_MAX_TOKENS and E <= 32; a larger call
  * returns MOE_ERR_UNSUPPORTED_SHAPE and launches nothing.
- * The first call on a device looks up the array's device address and sets
- * kernel attributes, with that device current; make that first call before
- * any stream capture.
+ * Every call looks up the array's address in the CUDA context current on the
+ * calling thread (cudaGetSymbolAddress: a host-side lookup that allocates
+ * nothing) and uses that context's copy of the array, so a context created
+ * after a cudaDeviceReset, or a non-primary context a host makes current, gets
+ * its own copy. The first call in a context may make the runtime load the
+ * library's device code into it; make that first call before any stream capture.
  * All calls share the one array: calls that can run on the GPU at the same time
  * (other streams, other host threads) race on it, so the caller must order them.
  * The array keeps the last call's contents; the kernels overwrite every entry
@@ -136,6 +143,32 @@ moe_status_t moe_top1_route(const float* gate_logits, int64_t B, int64_t N_H, in
 #define MOE_NOALLOC_MAX_TOKENS 2097152
 moe_status_t moe_top1_route_noalloc(const float* gate_logits, int64_t B, int64_t N_H, int32_t E,
                                     const moe_routing_t* out, void* stream);
+
+/*
+ * Validation of a routing that did not come from moe_top1_route. [P5] BUG
+ * CAUGHT DURING WIRING records a scratch sized for the wrong count that only
+ * showed up as wrong memory traffic; the contraction kernels here trust offsets
+ * and perm the same way, so a caller holding a routing from anywhere else (its
+ * own sort, a file, another process) checks it once before the first
+ * contraction uses it. One kernel reads the four arrays of `routing` (device
+ * pointers, none NULL when T > 0; counts and offsets always), within their
+ * declared sizes only, and sets MOE_FLAG_BAD_ROUTING in the workspace flag word
+ * unless all of these hold:
+ *   offsets[0] = 0, offsets[E] = T, offsets non-decreasing;
+ *   counts[e] = offsets[e + 1] - offsets[e];
+ *   every perm entry lies in [0, T), entries of one expert's segment
+ *   [offsets[e], offsets[e + 1]) strictly ascend, and expert_idx[perm[k]] = e
+ *   for every position k of segment e.
+ * These make perm a permutation of 0..T-1 grouping the tokens by expert in
+ * ascending t, with every expert index in [0, E): exactly what moe_top1_route
+ * writes (whose routings always pass). The result is read with
+ * moe_top1_device_flags (MOE_ERR_DEVICE_CHECK, bit MOE_FLAG_BAD_ROUTING), which
+ * synchronises; the check itself is enqueued on `stream` and touches no
+ * activation. Needs 256 bytes of workspace (the flag word), 256-byte aligned.
+ * 0 <= T < 2^31 - 256, 1 <= E <= 32.
+ */
+moe_status_t moe_top1_check_routing(const moe_routing_t* routing, int64_t T, int32_t E, void* workspace,
+                                    size_t workspace_bytes, void* stream);
 
 /*
  * Forward. [P1] kernel list (the chosen expert's [H, H] linear is applied to

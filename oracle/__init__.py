@@ -48,6 +48,7 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_bwd_db.argtypes = [P, P, i64, i32, i32, P, P]
     lib.oracle_bwd_dw_entries.argtypes = [P, P, P, i64, i32, i32, i64, P, P, P, P, P]
     lib.oracle_fwd_mean_collapse.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P]
+    lib.oracle_fwd_mean_collapse_presum.argtypes = [P, P, P, P, i64, i32, i32, i32, i32, P]
     lib.oracle_aux.argtypes = [P, P, i64, i32, ctypes.c_float, P, P, P, P, P]
     lib.oracle_lambda_eff.restype = ctypes.c_double
     lib.oracle_lambda_eff.argtypes = [ctypes.c_double] * 4
@@ -148,6 +149,23 @@ def fwd_mean_collapse(x, W, bias, expert_idx, N_H: int):
     mag = np.empty((B, H), np.float64)
     _load().oracle_fwd_mean_collapse(_p(x), _p(W), _p(bias), _p(idx), B, N_H, E, H, _p(out), _p(mag))
     return out, mag
+
+
+def fwd_mean_collapse_presum(x, W, bias, expert_idx, N_H: int, tf32_mode: int = TF32_NONE):
+    """The horizon mean of the forward computed as one contraction per batch row
+    over the per-(row, expert) sums of the horizon tokens' inputs, X_be, formed in
+    fp32 in ascending h; tf32_mode rounds X_be and W (the operands a TF32 tensor
+    core is given). -> ctx_mean [B, H] float64."""
+    x, W, bias, idx = _f32(x), _f32(W), _f32(bias), _i32(expert_idx)
+    T, H = x.shape
+    E = W.shape[0]
+    N_H = int(N_H)
+    if N_H < 1 or T % N_H:
+        raise ValueError("T must be a multiple of N_H >= 1")
+    B = T // N_H
+    out = np.empty((B, H), np.float64)
+    _load().oracle_fwd_mean_collapse_presum(_p(x), _p(W), _p(bias), _p(idx), B, N_H, E, H, int(tf32_mode), _p(out))
+    return out
 
 
 def bwd_mean_collapse(x, W, grad_ctx_mean, expert_idx, N_H: int, E: int, tf32_mode: int = TF32_NONE,

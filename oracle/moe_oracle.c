@@ -150,6 +150,49 @@ void oracle_fwd_mean_collapse(const float* x, const float* W, const float* bias,
 }
 
 /* ------------------------------------------------------------------------- */
+/* The same horizon mean, written as a contraction over summed inputs, with  */
+/* the contraction's operands rounded like a TF32 tensor core rounds them.   */
+/* The forward is linear in x, so the horizon tokens of row b that chose     */
+/* expert e can be summed before the expert's matrix is applied:              */
+/*   ctx_mean[b, o] = (1/N_H) sum_e (sum_i W[e, o, i] X_be[i] + n_be bias[e, o])*/
+/*   X_be = sum_{h : e*(b*N_H + h) = e} x[b*N_H + h],  n_be = that count.     */
+/* Reading for the TF32 mode: X_be is formed in fp32, adding the horizon      */
+/* tokens in ascending h, and then X_be and W are the operands that           */
+/* tf32_mode rounds (bias and the counts are not rounded). Products are      */
+/* exact in double and every other sum is in double. An expert index outside */
+/* [0, E) contributes nothing.                                                */
+/* ------------------------------------------------------------------------- */
+void oracle_fwd_mean_collapse_presum(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
+                                     int64_t B, int32_t N_H, int32_t E, int32_t H, int32_t tf32_mode,
+                                     double* ctx_mean)
+{
+    float* X = (float*)malloc(sizeof(float) * (size_t)H);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)H);
+    for (int64_t b = 0; b < B; ++b) {
+        for (int32_t o = 0; o < H; ++o) acc[o] = 0.0;
+        for (int32_t e = 0; e < E; ++e) {
+            int32_t n_be = 0;
+            for (int32_t h = 0; h < N_H; ++h) {
+                const int64_t t = b * N_H + h;
+                if (expert_idx[t] != e) continue;
+                for (int32_t i = 0; i < H; ++i) X[i] = (n_be == 0) ? x[t * H + i] : X[i] + x[t * H + i];
+                ++n_be;
+            }
+            if (n_be == 0) continue;
+            for (int32_t o = 0; o < H; ++o) {
+                const float* w_row = W + ((int64_t)e * H + o) * H;
+                double dot = 0.0;
+                for (int32_t i = 0; i < H; ++i) dot += tf(w_row[i], tf32_mode) * tf(X[i], tf32_mode);
+                acc[o] += dot + (double)n_be * (double)bias[(int64_t)e * H + o];
+            }
+        }
+        for (int32_t o = 0; o < H; ++o) ctx_mean[b * H + o] = acc[o] / (double)N_H;
+    }
+    free(X);
+    free(acc);
+}
+
+/* ------------------------------------------------------------------------- */
 /* Backward, input gradient. [P1] kernel list and PERFORMANCE: the chain rule */
 /* runs through the selected expert only, and the weight column lines up     */
 /* with the input index:  d_x[t, i] = sum_o W[e*, o, i] * d_out[t, o].        */

@@ -53,7 +53,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_top1_abi_version() == 3
+    assert L.moe_top1_abi_version() == 4
     for s, name in enumerate(ops._STATUS):
         assert L.moe_status_string(s).decode() == name
     assert L.moe_status_string(99).decode() == "MOE_ERR_UNKNOWN"
@@ -197,3 +197,21 @@ def test_python_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         ops._ptr(torch.zeros(4))
+
+
+def test_check_routing_rejects_bad_arguments(L):
+    r = ops.RoutingC(_p(A), _p(A + 0x100000), _p(A + 0x200000), _p(A + 0x300000))
+    ws = _p(A + 0x400000)
+    f = L.moe_top1_check_routing
+    assert f(None, 10, 4, ws, 256, None) == INVALID
+    assert f(ctypes.byref(r), -1, 4, ws, 256, None) == INVALID
+    assert f(ctypes.byref(r), 10, 0, ws, 256, None) == SHAPE
+    assert f(ctypes.byref(r), 10, 33, ws, 256, None) == SHAPE
+    assert f(ctypes.byref(r), 2 ** 31, 4, ws, 256, None) == SHAPE
+    assert f(ctypes.byref(r), 10, 4, None, 256, None) == WORKSPACE
+    assert f(ctypes.byref(r), 10, 4, ws, 255, None) == WORKSPACE
+    assert f(ctypes.byref(r), 10, 4, _p(A + 0x400010), 256, None) == MISALIGNED
+    bad = ops.RoutingC(_p(A + 2), _p(A + 0x100000), _p(A + 0x200000), _p(A + 0x300000))
+    assert f(ctypes.byref(bad), 10, 4, ws, 256, None) == MISALIGNED
+    nul = ops.RoutingC(None, _p(A + 0x100000), _p(A + 0x200000), None)
+    assert f(ctypes.byref(nul), 10, 4, ws, 256, None) == INVALID

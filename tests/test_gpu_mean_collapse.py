@@ -63,6 +63,15 @@ def test_mean_collapse_backward_parity(spec, math_mode):
     assert_close("db", got["db"], want["db"], atol, rtol, scale=want["db_scale"])
 
 
+# FFMA also serves the widths TF32 does not (H a multiple of 32 up to 256).
+FFMA_WIDTH_SPECS = [wl.make_spec(f"mc_ffma_b203_h5_e6_h{H}", 203, 5, 6, H, 400 + H) for H in (32, 96, 160, 224)]
+
+
+@pytest.mark.parametrize("spec", FFMA_WIDTH_SPECS, ids=lambda s: s.name)
+def test_mean_collapse_backward_parity_ffma_other_widths(spec):
+    test_mean_collapse_backward_parity(spec, ops.MOE_MATH_FFMA)
+
+
 @pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
 def test_mean_collapse_matches_plain_backward_bitwise_for_power_of_two_horizons(math_mode):
     """With N_H = 16, g / N_H is exact, so the two entry points must agree bit for
@@ -115,15 +124,34 @@ FWD_SPECS = [
 
 
 def fwd_bound(spec, math):
-    """|got - exact| <= c * mag, mag = (1/N_H) sum_h (sum_i |W x| + |bias|) from the
-    oracle. fp32 sums: the horizon pre-sum (N_H terms), the K = E * H products and
-    the epilogue's bias, scale and store (8 more roundings), each at most one
-    unit 2^-24 of mag. TF32 adds the rounding of both operands of every product,
-    each below 2^-10 relative."""
+    """A worst-case bound against the exact definition: |got - exact| <= c * mag,
+    mag = (1/N_H) sum_h (sum_i |W x| + |bias|) from the oracle. fp32 sums: the
+    horizon pre-sum (N_H terms), the K = E * H products and the epilogue's bias,
+    scale and store (8 more roundings), each at most one unit 2^-24 of mag. TF32
+    adds the rounding of both operands of every product, each below 2^-10
+    relative."""
     c = (spec.E * spec.H + spec.N_H + 8) * 2.0 ** -24
     if math == ops.MOE_MATH_TF32:
         c += 2.0 ** -9
     return c
+
+
+def fwd_reference(inp, idx, N_H, math):
+    """The oracle the kernel is held to at the gate's own tolerances: FFMA against
+    the exact definition (|g - o| <= 1e-5 + 1e-5 |o|); TF32 against the oracle's
+    TF32 mode of the same mean, whose contraction operands are the per-(row,
+    expert) horizon sums X_be (formed in fp32, ascending h) and W, rounded the way
+    the tensor core rounds them (|g - o| <= 1e-4 + 2e-3 |o|)."""
+    if math == ops.MOE_MATH_TF32:
+        return oracle.fwd_mean_collapse_presum(inp.x, inp.W, inp.bias, idx, N_H, tf32_mode(math))
+    return oracle.fwd_mean_collapse(inp.x, inp.W, inp.bias, idx, N_H)[0]
+
+
+def fwd_outside(got, want, math):
+    """Number of elements outside the tolerance of the math mode."""
+    atol, rtol = TOL[math]
+    err = np.abs(got.astype(np.float64) - want)
+    return int((~(err <= atol + rtol * np.abs(want))).sum())
 
 
 def _run_fwd(spec, inp, math):
@@ -145,11 +173,42 @@ def test_fwd_mean_collapse_parity(spec, math_mode):
     inp = wl.generate(spec)
     got, _, _ = _run_fwd(spec, inp, math_mode)
     idx = oracle.route(inp.gate_logits)[0]
+    assert np.isfinite(got).all()
+    assert_close("ctx_mean", got, fwd_reference(inp, idx, spec.N_H, math_mode), *TOL[math_mode])
+    # and the worst-case bound against the exact definition in both modes
     want, mag = oracle.fwd_mean_collapse(inp.x, inp.W, inp.bias, idx, spec.N_H)
     err = np.abs(got.astype(np.float64) - want)
     bound = fwd_bound(spec, math_mode) * mag
-    assert np.isfinite(got).all()
     assert (err <= bound).all(), f"max err/bound {np.max(err / bound):.3g}"
+
+
+@pytest.mark.parametrize("spec", FFMA_WIDTH_SPECS, ids=lambda s: s.name)
+def test_fwd_mean_collapse_parity_ffma_other_widths(spec):
+    test_fwd_mean_collapse_parity(spec, ops.MOE_MATH_FFMA)
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_fwd_mean_collapse_check_catches_one_token_on_the_wrong_expert(math_mode):
+    """The parity check must be tight enough to see one horizon token of one row
+    sent to another expert (its W and bias change): the kernel is handed a
+    routing with that one index changed, and the result is compared with the
+    oracle on the true routing."""
+    spec = wl.make_spec("mcf_sens_b256_h16_e8_h256", 256, 16, 8, 256, 61)
+    inp = wl.generate(spec)
+    idx = oracle.route(inp.gate_logits)[0]
+    want = fwd_reference(inp, idx, spec.N_H, math_mode)
+    got, r, ws = _run_fwd(spec, inp, math_mode)
+    assert fwd_outside(got, want, math_mode) == 0
+    t = 5 * spec.N_H + 3  # row 5, horizon token 3
+    r.expert_idx[t] = (int(idx[t]) + 1) % spec.E
+    out = torch.empty(spec.B, spec.H, device="cuda")
+    ops.moe_top1_fwd_mean_collapse(dev(inp.x), dev(inp.W), dev(inp.bias), r, spec.B, spec.N_H, spec.E, spec.H,
+                                   math_mode, out, ws)
+    torch.cuda.synchronize()
+    bad = out.cpu().numpy()
+    n_bad = fwd_outside(bad, want, math_mode)
+    assert n_bad > spec.H // 2, n_bad   # row 5 is off almost everywhere
+    assert fwd_outside(np.delete(bad, 5, axis=0), np.delete(want, 5, axis=0), math_mode) == 0  # other rows intact
 
 
 @pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
@@ -202,6 +261,6 @@ def test_fwd_mean_collapse_full_size_sampled_rows():
     rows = np.sort(np.random.default_rng(60).choice(spec.B, 64, replace=False))
     tok = (rows[:, None] * spec.N_H + np.arange(spec.N_H)).reshape(-1)
     idx = oracle.route(inp.gate_logits[tok])[0]
-    want, mag = oracle.fwd_mean_collapse(inp.x[tok], inp.W, inp.bias, idx, spec.N_H)
-    got = gate.ctx_mean[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64)
-    assert (np.abs(got - want) <= fwd_bound(spec, ops.MOE_MATH_TF32) * mag).all()
+    got = gate.ctx_mean[torch.from_numpy(rows).cuda()].cpu().numpy()
+    want = oracle.fwd_mean_collapse_presum(inp.x[tok], inp.W, inp.bias, idx, spec.N_H, tf32_mode(ops.MOE_MATH_TF32))
+    assert_close("ctx_mean (sampled rows)", got, want, *TOL[ops.MOE_MATH_TF32])

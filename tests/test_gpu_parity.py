@@ -14,7 +14,7 @@ import torch
 import oracle
 from bwd_route_b200 import ops
 from bwd_route_b200 import workloads as wl
-from gpu_harness import TOL, assert_close, run_gpu, tf32_mode
+from gpu_harness import TOL, assert_close, dev, run_gpu, tf32_mode
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +40,13 @@ EDGE = [
     wl.make_spec("h256_b4096_e8_h256", 4096, 8, 8, 256, 18),
     wl.make_spec("h256_max_experts_b4000_e32_h256", 4000, 5, 32, 256, 19),
 ]
+
+
+# FFMA accepts every H that is a multiple of 32 up to 256 (TF32 only 128 and
+# 256): ragged token counts with 5 and with 32 experts at each of the other widths.
+FFMA_WIDTHS = [32, 64, 96, 160, 192, 224]
+FFMA_SHAPES = ([wl.make_spec(f"ffma_b311_e5_h{H}", 311, 3, 5, H, 100 + H) for H in FFMA_WIDTHS] +
+               [wl.make_spec(f"ffma_b700_e32_h{H}", 700, 3, 32, H, 300 + H) for H in FFMA_WIDTHS])
 
 
 def lam_of(inp):
@@ -102,6 +109,59 @@ def test_full_parity(name, math_mode):
 @pytest.mark.parametrize("spec", EDGE, ids=lambda s: s.name)
 def test_edge_parity(spec, math_mode):
     check_all(wl.generate(spec), math_mode)
+
+
+@pytest.mark.parametrize("spec", FFMA_SHAPES, ids=lambda s: s.name)
+def test_ffma_parity_at_every_supported_width(spec):
+    check_all(wl.generate(spec), ops.MOE_MATH_FFMA)
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_straight_through_expert_path_gives_the_logits_no_gradient(math_mode):
+    """STE: the top-1 choice is piecewise constant in the logits, so the expert
+    path contributes nothing to their gradient. (1) The aux loss's logit
+    gradient is bitwise the same before and after a backward of the expert path
+    on the same tokens: the backward writes no logit gradient. (2) Changing the
+    logits without changing any argmax (scaling by 2, exact in fp32) leaves the
+    routing and every expert-path output bitwise unchanged, while the aux
+    gradient does change."""
+    spec = wl.make_spec("ste_b900_e8_h256", 900, 3, 8, 256, 71)
+    inp = wl.generate(spec)
+    B, N_H, E, H, T = spec.B, spec.N_H, spec.E, spec.H, spec.T
+    logits, x, d_out = dev(inp.gate_logits), dev(inp.x), dev(inp.d_out)
+    W, bias = dev(inp.W), dev(inp.bias)
+    lam = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    ws = ops.new_workspace(T, E, H, "cuda")
+
+    def aux_grad(lg, r):
+        d = torch.empty(T, E, device="cuda")
+        ops.moe_aux_loss_fwd_bwd(lg, r.counts, B, N_H, E, lam, d, torch.empty(2, device="cuda"),
+                                 torch.empty(E, device="cuda"), None, ws)
+        return d
+
+    def expert_path(lg):
+        r = ops.Routing.empty(T, E, "cuda")
+        ops.moe_top1_route(lg, B, N_H, E, r, ws)
+        out = [torch.empty(T, H, device="cuda"), torch.empty(T, H, device="cuda"),
+               torch.empty(E, H, H, device="cuda"), torch.empty(E, H, device="cuda")]
+        ops.moe_top1_fwd(x, W, bias, r, B, N_H, E, H, math_mode, out[0], ws)
+        ops.moe_top1_bwd(x, W, d_out, r, B, N_H, E, H, math_mode, out[1], out[2], out[3], 0, ws)
+        return r, out
+
+    r = ops.Routing.empty(T, E, "cuda")
+    ops.moe_top1_route(logits, B, N_H, E, r, ws)
+    before = aux_grad(logits, r).cpu().numpy()
+    _, path = expert_path(logits)
+    after = aux_grad(logits, r).cpu().numpy()
+    torch.cuda.synchronize()
+    assert ops.moe_top1_device_flags(ws) == 0
+    assert before.tobytes() == after.tobytes()
+    r2, path2 = expert_path(logits * 2.0)
+    for name in ("expert_idx", "counts", "offsets", "perm"):
+        assert torch.equal(getattr(r2, name), getattr(r, name)), name
+    for a, b in zip(path, path2):
+        assert torch.equal(a, b)
+    assert not np.array_equal(aux_grad(logits * 2.0, r2).cpu().numpy(), before)
 
 
 def test_identity_experts_bit_exact():

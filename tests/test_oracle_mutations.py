@@ -60,6 +60,14 @@ MUTATIONS = [
     ("horizon mean reads token 0's input", "(double)w_row[i] * (double)x[t * H + i];",
      "(double)w_row[i] * (double)x[b * N_H * H + i];"),
     ("horizon mean magnitude keeps signs", "acc_abs += fabs(term);", "acc_abs += term;"),
+    ("summed horizon mean adds each bias once per row", "acc[o] += dot + (double)n_be * (double)bias[(int64_t)e * H + o];",
+     "acc[o] += dot + (double)bias[(int64_t)e * H + o];"),
+    ("summed horizon mean leaves X_be unrounded", "dot += tf(w_row[i], tf32_mode) * tf(X[i], tf32_mode);",
+     "dot += tf(w_row[i], tf32_mode) * (double)X[i];"),
+    ("summed horizon mean keeps only the last token", "X[i] = (n_be == 0) ? x[t * H + i] : X[i] + x[t * H + i];",
+     "X[i] = x[t * H + i];"),
+    ("summed horizon mean not divided by N_H", "ctx_mean[b * H + o] = acc[o] / (double)N_H;",
+     "ctx_mean[b * H + o] = acc[o];"),
 ]
 
 

@@ -617,3 +617,79 @@ def test_fwd_mean_collapse_magnitude_bounds_the_value_and_is_exact_for_positive_
     assert np.all(np.abs(got) <= mag * (1 + 1e-14))
     got, mag = oracle.fwd_mean_collapse(np.abs(x), np.abs(W), np.abs(bias), idx, N_H)
     np.testing.assert_allclose(mag, got, rtol=1e-14)
+
+
+# ---------------------------------------------------------------- the same mean as a contraction over summed inputs
+def _small_integer_case(B=5, N_H=6, E=4, H=32, seed=21):
+    """Inputs whose fp32 horizon sums are exact (small integers), so the pre-summed
+    form must agree with the definition to double rounding."""
+    rng = np.random.default_rng(seed)
+    x = rng.integers(-8, 9, size=(B * N_H, H)).astype(np.float32)
+    W = (rng.integers(-4, 5, size=(E, H, H)) / 16.0).astype(np.float32)
+    bias = (rng.integers(-4, 5, size=(E, H)) / 8.0).astype(np.float32)
+    idx = oracle.route(rng.standard_normal((B * N_H, E)).astype(np.float32))[0]
+    return x, W, bias, idx, B, N_H, E, H
+
+
+def test_presum_horizon_mean_equals_the_definition_when_the_sums_are_exact():
+    x, W, bias, idx, B, N_H, E, H = _small_integer_case()
+    want, _ = oracle.fwd_mean_collapse(x, W, bias, idx, N_H)
+    for mode in (oracle.TF32_NONE, oracle.TF32_RZ):  # integers and multiples of 1/16 are TF32 values
+        got = oracle.fwd_mean_collapse_presum(x, W, bias, idx, N_H, mode)
+        np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-14)
+
+
+def test_presum_horizon_mean_with_one_horizon_token_is_the_tf32_forward():
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=9, N_H=1, E=4)
+    for mode in (oracle.TF32_NONE, oracle.TF32_RZ, oracle.TF32_RNE):
+        got = oracle.fwd_mean_collapse_presum(x, W, bias, idx, 1, mode)
+        np.testing.assert_allclose(got, oracle.fwd(x, W, bias, idx, mode), rtol=1e-14, atol=1e-15)
+
+
+def test_presum_horizon_mean_counts_each_expert_bias_once_per_token():
+    # zero input: only the biases remain, n_be of expert e's bias per row
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=6, N_H=7, E=4)
+    got = oracle.fwd_mean_collapse_presum(np.zeros_like(x), W, bias, idx, N_H, oracle.TF32_RZ)
+    want = bias.astype(np.float64)[idx.reshape(B, N_H)].mean(axis=1)
+    np.testing.assert_allclose(got, want, rtol=1e-15, atol=1e-17)
+    # an expert index outside [0, E) contributes nothing (zero input, bias only)
+    bad = idx.copy()
+    bad[0] = E
+    got = oracle.fwd_mean_collapse_presum(np.zeros_like(x), W, bias, bad, N_H, oracle.TF32_NONE)
+    keep = idx.reshape(B, N_H).copy()
+    want = bias.astype(np.float64)[keep]
+    want[0, 0] = 0.0
+    np.testing.assert_allclose(got, want.sum(axis=1) / N_H, rtol=1e-15, atol=1e-17)
+
+
+def test_presum_horizon_mean_tf32_error_within_the_operand_rounding_bound():
+    """Cutting X_be and W to 10 mantissa bits changes each product by less than
+    2 * 2^-10 of its size; the fp32 horizon sums add at most N_H roundings of
+    2^-24 each. So |tf32 - exact| <= (2^-9 + N_H 2^-24) * mag, and truncation
+    (RZ) of positive operands can only lower the result."""
+    x, W, bias, _, idx, B, N_H, E, H = _collapse_case(B=6, N_H=5, E=3, H=64)
+    exact, mag = oracle.fwd_mean_collapse(x, W, bias, idx, N_H)
+    got = oracle.fwd_mean_collapse_presum(x, W, bias, idx, N_H, oracle.TF32_RZ)
+    assert np.all(np.abs(got - exact) <= (2.0 ** -9 + N_H * 2.0 ** -23) * mag)
+    assert np.any(got != exact)  # the rounding does act
+    xp, Wp, bp = np.abs(x), np.abs(W), np.abs(bias)
+    exact, _ = oracle.fwd_mean_collapse(xp, Wp, bp, idx, N_H)
+    none = oracle.fwd_mean_collapse_presum(xp, Wp, bp, idx, N_H, oracle.TF32_NONE)
+    rz = oracle.fwd_mean_collapse_presum(xp, Wp, bp, idx, N_H, oracle.TF32_RZ)
+    assert np.all(rz <= none)
+    np.testing.assert_allclose(none, exact, rtol=N_H * 2.0 ** -23)
+
+
+def test_presum_horizon_mean_sums_the_horizon_in_fp32_ascending():
+    # one row, two horizon tokens on one expert: X = fl32(x0 + x1); with x0 = 1,
+    # x1 = 2^-24 the fp32 sum rounds to 1 (the definition keeps 1 + 2^-24)
+    H, E, N_H = 32, 1, 2
+    x = np.zeros((N_H, H), np.float32)
+    x[0, 0], x[1, 0] = 1.0, 2.0 ** -24
+    W = np.zeros((E, H, H), np.float32)
+    W[0, 0, 0] = 1.0
+    idx = np.zeros(N_H, np.int32)
+    got = oracle.fwd_mean_collapse_presum(x, W, np.zeros((E, H), np.float32), idx, N_H, oracle.TF32_NONE)
+    assert got[0, 0] == 0.5
+    exact, _ = oracle.fwd_mean_collapse(x, W, np.zeros((E, H), np.float32), idx, N_H)
+    assert exact[0, 0] == (1.0 + 2.0 ** -24) / 2

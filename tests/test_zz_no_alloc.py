@@ -62,3 +62,35 @@ def test_noalloc_route_rejects_more_tokens_than_its_scratch_holds():
     ops.moe_top1_route_noalloc(logits, T, 1, E, r)
     torch.cuda.synchronize()
     assert r.counts.cpu().tolist() == [T, 0, 0, 0]
+
+
+def test_noalloc_route_fills_the_whole_array_at_the_limit_with_32_experts():
+    # T = MOE_NOALLOC_MAX_TOKENS and E = 32 use every entry of the fixed array
+    # (2048 routing blocks x 32 experts, counts and bases): the result must still
+    # be exactly moe_top1_route's
+    E = 32
+    T = ops.MOE_NOALLOC_MAX_TOKENS
+    g = torch.Generator(device="cuda").manual_seed(7)
+    logits = torch.randint(0, 4, (T, E), generator=g, device="cuda").to(torch.float32)  # many ties
+    ref = ops.Routing.empty(T, E, "cuda")
+    ws = ops.new_workspace(T, E, 0, "cuda")
+    ops.moe_top1_route(logits, T, 1, E, ref, ws)
+    got = ops.Routing.empty(T, E, "cuda")
+    for t in (got.expert_idx, got.counts, got.offsets, got.perm):
+        t.fill_(-7)
+    ops.moe_top1_route_noalloc(logits, T, 1, E, got)
+    torch.cuda.synchronize()
+    for name in ("expert_idx", "counts", "offsets", "perm"):
+        assert torch.equal(getattr(got, name), getattr(ref, name)), name
+
+
+def test_noalloc_route_with_no_tokens_zeroes_counts_and_offsets():
+    E = 6
+    r = ops.Routing(torch.empty(0, dtype=torch.int32, device="cuda"),
+                    torch.full((E,), 9, dtype=torch.int32, device="cuda"),
+                    torch.full((E + 1,), 9, dtype=torch.int32, device="cuda"),
+                    torch.empty(0, dtype=torch.int32, device="cuda"))
+    ops.moe_top1_route_noalloc(torch.empty(0, E, device="cuda"), 0, 4, E, r)
+    torch.cuda.synchronize()
+    assert r.counts.cpu().tolist() == [0] * E
+    assert r.offsets.cpu().tolist() == [0] * (E + 1)
