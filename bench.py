@@ -61,20 +61,18 @@ def algorithmic(spec, grad: str = "token"):
         per_kernel_bytes = {
             # x and the expert indices read, ctx_mean written; W and bias
             "fwd": T * (4 * H + 4) + g_bytes + E * H * H * 4 + E * H * 4,
-            # grad_ctx_mean read once, d_x written, perm read; W
-            "d_x": T * (4 * H + 4) + g_bytes + E * H * H * 4,
-            # x and grad_ctx_mean read, perm read; dW and db written
-            "wgrad": T * (4 * H + 4) + g_bytes + E * H * H * 4 + E * H * 4,
+            # the whole backward call: x read, d_x written, perm read, grad_ctx_mean
+            # read once; W read, dW and db written
+            "bwd": T * (8 * H + 4) + g_bytes + 2 * E * H * H * 4 + E * H * 4,
         }
         return step_bytes, step_flops, per_kernel_bytes
     step_bytes = T * (4 * (5 * H + 3 * E) + 16) + 2 * E * H * H * 4
     per_kernel_bytes = {
         # x read, routed written, perm read; W and bias
         "fwd": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
-        # d_out read, d_x written, perm read; W
-        "d_x": T * (8 * H + 4) + E * H * H * 4,
-        # x and d_out read, perm read; dW and db written
-        "wgrad": T * (8 * H + 4) + E * H * H * 4 + E * H * 4,
+        # the whole backward call: x and d_out read once, d_x written, perm read;
+        # W read, dW and db written
+        "bwd": T * (12 * H + 4) + 2 * E * H * H * 4 + E * H * 4,
     }
     return step_bytes, step_flops, per_kernel_bytes
 
@@ -126,6 +124,13 @@ def host_cpu() -> dict:
 
 TRAFFIC_RECORD = os.path.join(HERE, "profiles", "launch_list_large_b65536_e8_h256.md")
 
+# The library kernels each timed call launches, per (call, fused TF32 H = 256 backward).
+CALL_KERNELS = {
+    ("fwd", True): ["grouped_tf32_kernel"], ("fwd", False): ["grouped_tf32_kernel or grouped_ffma_kernel"],
+    ("bwd", True): ["bwd_fused_tf32_kernel", "wgrad_reduce_kernel"],
+    ("bwd", False): ["grouped d_x kernel", "weight-gradient kernel", "wgrad_reduce_kernel"],
+}
+
 
 def code_sha1(paths) -> str:
     """sha1 of the code of the given source files with comments and blank space
@@ -164,7 +169,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
                0x10: "sync_boost", 0x1: "gpu_idle"}
 
-    def __init__(self, index: int, period: float = 0.02):
+    def __init__(self, index: int, period: float = 0.001):
         self.index, self.period = index, period
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -236,6 +241,37 @@ def cpu_oracle_tokens_per_s(inp, n_tokens: int):
     oracle.step(sample)
     dt = time.perf_counter() - t0
     return sample.spec.T / dt, dt, sample.spec.T
+
+
+def _oracle_shard(args):
+    """One worker of the all-cores CPU baseline: the oracle, unchanged, on one
+    token shard; returns its dW and db (the sums the shards share)."""
+    inp, lo, hi = args
+    import oracle
+    shard = wl.token_sample(wl.dataclasses.replace(inp, gate_logits=inp.gate_logits[lo:hi], x=inp.x[lo:hi],
+                                                   d_out=inp.d_out[lo:hi]), hi - lo)
+    out = oracle.step(shard)
+    return out["dW"], out["db"]
+
+
+def cpu_oracle_all_cores(inp, tokens_per_core: int, cores: int):
+    """The oracle, as it stands, on `cores` token shards in `cores` processes
+    (spawned, so no process inherits a CUDA context), with dW and db of the
+    shards added in shard order. Returns (tokens/s, seconds, tokens)."""
+    import multiprocessing as mp
+    n = min(inp.spec.T, tokens_per_core * cores)
+    bounds = [(n * k // cores, n * (k + 1) // cores) for k in range(cores)]
+    small = wl.token_sample(inp, n)
+    with mp.get_context("spawn").Pool(cores) as pool:
+        pool.map(_oracle_shard, [(wl.token_sample(small, 64), 0, 64)] * cores)  # start-up and oracle build
+        t0 = time.perf_counter()
+        parts = pool.map(_oracle_shard, [(small, lo, hi) for lo, hi in bounds])
+        dW, db = parts[0]
+        for pw, pb in parts[1:]:
+            dW = dW + pw
+            db = db + pb
+        dt = time.perf_counter() - t0
+    return n / dt, dt, n
 
 
 def run_reference(args, spec):
@@ -326,8 +362,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
-        # the backward is issued as two calls (d_x; dW and db) so that each
-        # contraction kernel can be timed on its own
+        # the calls of one training step, with an event between consecutive calls
         if ev:
             ev[0].record(stream)
         gate.route(logits)
@@ -339,19 +374,16 @@ def main():
             gate.forward(x)
         if ev:
             ev[2].record(stream)
-        bwd = ops.moe_top1_bwd_mean_collapse if collapse else ops.moe_top1_bwd
-        bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, gate.d_x, None, None, 0,
-                         gate.ws)
+        if collapse:
+            gate.backward_mean_collapse(x, d_out)
+        else:
+            gate.backward(x, d_out)
         if ev:
             ev[3].record(stream)
-        bwd(x, W, d_out, gate.routing, spec.B, spec.N_H, E, H, math_mode, None, gate.dW, gate.db, 0,
-                         gate.ws)
-        if ev:
-            ev[4].record(stream)
         gate.aux(logits)
         gate.update_lambda()
         if ev:
-            ev[5].record(stream)
+            ev[4].record(stream)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -367,7 +399,7 @@ def main():
 
     # timed region: K whole steps, events on the launching stream
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
-    per_call = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    per_call = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     graph = None
     if args.graph:
@@ -387,12 +419,12 @@ def main():
             if graph is not None:
                 per_call[k][0].record(stream)
                 graph.replay()
-                per_call[k][5].record(stream)
+                per_call[k][4].record(stream)
             else:
                 step(per_call[k])
         end.record(stream)
         barrier()
-    step_ms = sorted(per_call[k][0].elapsed_time(per_call[k][5]) for k in range(args.steps))
+    step_ms = sorted(per_call[k][0].elapsed_time(per_call[k][4]) for k in range(args.steps))
     if flush is not None:  # the flushes sit between the steps' own events
         ms = sum(step_ms)
     else:
@@ -400,10 +432,10 @@ def main():
     ms = max_over_ranks(ms, dev)
     ms_per_step = ms / args.steps
     pct = lambda f: step_ms[min(len(step_ms) - 1, int(f * len(step_ms)))]  # noqa: E731
-    names = ["route", "fwd", "d_x", "wgrad", "aux+lambda"]
+    names = ["route", "fwd", "bwd", "aux+lambda"]
     if graph is not None:
         # per-call times from a separate un-captured loop
-        per_call = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(min(args.steps, 20))]
+        per_call = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(min(args.steps, 20))]
         for ev in per_call:
             step(ev)
         torch.cuda.synchronize(dev)
@@ -444,7 +476,8 @@ def main():
         tf32_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * TF32_OVER_BF16
         t_roof = max(step_bytes / (hbm * 1e9), step_flops / (tf32_sus * 1e12))
         value = job_throughput(world, T, ms_per_step)
-        dominant = max(["fwd", "d_x", "wgrad"], key=lambda n: call_ms[n])
+        dominant = max(["fwd", "bwd"], key=lambda n: call_ms[n])
+        fused = math_mode == ops.MOE_MATH_TF32 and H == 256
         achieved = kbytes[dominant] / (call_ms[dominant] * 1e-3) / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -454,7 +487,8 @@ def main():
                        "N_H": spec.N_H, "E": E, "H": H, "tokens": T, "grad": args.grad,
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": l2_note(spec, collapse, flush is not None)},
-            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "roofline": {"bound": "hbm", "kernel": dominant, "launches_in_call": CALL_KERNELS[(dominant, fused)],
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm,
                          "traffic": None if collapse else recorded_traffic(dominant, spec.name, args.math),
                          "algorithmic_bytes": kbytes[dominant], "peak_source": f"{peak_kind} hbm_gbs"},
@@ -469,7 +503,7 @@ def main():
                       + ("; 256 MB written between steps, outside their events" if flush is not None else ""),
             "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
                     "h2d_bytes_per_step": (T * (E + H) + g_host.shape[0] * H) * 4, "d2h_bytes_per_step": 8},
-            "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode),
+            "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode, H, T, E),
             "clocks": clocks.summary(),
             "device_flags": flags,
         }
@@ -479,6 +513,15 @@ def main():
                                     "sample": f"first {n} tokens of {spec.name}: route, forward, d_x, dW/db and "
                                               f"aux in plain single-threaded C (fp64 accumulation), {dt:.1f} s",
                                     **host_cpu()}
+            cores = host_cpu()["cores_available"] or 1
+            if cores > 1:
+                v, dt, n = cpu_oracle_all_cores(inp, CPU_SAMPLE_TOKENS, cores)
+                line["cpu_baseline_all_cores"] = {
+                    "value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                    "sample": f"first {n} tokens of {spec.name} in {cores} equal shards, one process per core, "
+                              f"each running the unchanged single-threaded oracle (route, forward, d_x, dW/db, aux "
+                              f"of its shard); dW and db of the shards added in shard order; {dt:.1f} s",
+                    **host_cpu()}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

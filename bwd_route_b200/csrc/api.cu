@@ -23,6 +23,7 @@ constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
     int num_sms = 0;
+    int fused_pairs = 0;  // CTA pairs of the fused backward that run at once
     bool aux_ready = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -44,7 +45,14 @@ cudaError_t device_info(DeviceInfo** out) {
         if (e == cudaSuccess) e = route_set_smem_limits();
         if (e == cudaSuccess) e = tf32_set_smem_limits();
         if (e == cudaSuccess) e = hmean_set_smem_limits();
+        if (e == cudaSuccess) e = bwd_fused_set_smem_limits();
         if (e != cudaSuccess) return e;
+        // pairs of the fused backward that fit at once; a failed query only
+        // disables that call (it then returns MOE_ERR_CUDA), not the others
+        if (bwd_fused_max_pairs(&d.fused_pairs) != cudaSuccess) {
+            d.fused_pairs = 0;
+            (void)cudaGetLastError();
+        }
         d.aux_ready = true;
     }
     *out = &d;
@@ -115,11 +123,11 @@ struct MapKey {
     const float* base;
     uint64_t rows, cols;
     uint32_t box_cols, box_rows;
-    bool atom32;
+    int layout;
     int dev;
     bool operator==(const MapKey& o) const {
         return base == o.base && rows == o.rows && cols == o.cols && box_cols == o.box_cols &&
-               box_rows == o.box_rows && atom32 == o.atom32 && dev == o.dev;
+               box_rows == o.box_rows && layout == o.layout && dev == o.dev;
     }
 };
 constexpr int kMapCache = 16;
@@ -131,10 +139,10 @@ std::mutex g_map_mu;
 }  // namespace
 
 bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                 uint32_t box_rows, bool atom32) {
+                 uint32_t box_rows, int layout) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    const MapKey key{base, rows, cols, box_cols, box_rows, atom32, dev};
+    const MapKey key{base, rows, cols, box_cols, box_rows, layout, dev};
     {
         std::lock_guard<std::mutex> lock(g_map_mu);
         for (int i = 0; i < g_map_n; ++i)
@@ -143,7 +151,7 @@ bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t co
                 return true;
             }
     }
-    if (!encode_map_2d(map, base, rows, cols, box_cols, box_rows, atom32)) return false;
+    if (!encode_map_2d(map, base, rows, cols, box_cols, box_rows, layout)) return false;
     std::lock_guard<std::mutex> lock(g_map_mu);
     const int slot = g_map_n < kMapCache ? g_map_n++ : (g_map_next++ % kMapCache);
     g_map_key[slot] = key;
@@ -152,17 +160,19 @@ bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t co
 }
 
 bool encode_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                   uint32_t box_rows, bool atom32) {
+                   uint32_t box_rows, int layout) {
     EncodeTiledFn enc = get_encode_tiled();
     if (!enc) return false;
+    const CUtensorMapSwizzle swz = layout == kMapSw128Atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                   : layout == kMapSw64      ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : layout == kMapPlain     ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                                             : CU_TENSOR_MAP_SWIZZLE_128B;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * sizeof(float)};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -220,6 +230,18 @@ moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
+    if (math == MOE_MATH_TF32 && H == 256 && d_x && (dW || db)) {
+        // one pass over d_out: d_x, and the dW / db partial sums, then the slot reduction
+        float* part = reinterpret_cast<float*>(ws + L.wg_part);
+        float* part_db = reinterpret_cast<float*>(ws + L.wg_part_db);
+        if (dev->fused_pairs < 1) return MOE_ERR_CUDA;
+        const int P = bwd_fused_pairs(T, dev->fused_pairs);
+        e = launch_bwd_fused_tf32(x, W, d_out, routing->offsets, routing->perm, T, E, P, g_div, g_scale, acc_dx, d_x,
+                                  part, part_db, flags, s);
+        if (e == cudaSuccess)
+            e = launch_wgrad_reduce(part, part_db, routing->offsets, T, E, H, P, g_scale, dW, db, acc_dw, acc_db, s);
+        return cuda_status(e);
+    }
     if (d_x) {
         if (math == MOE_MATH_TF32) {
             e = launch_grouped_tf32(d_out, W, nullptr, routing->offsets, routing->perm, T, E, H, 1, acc_dx, g_div,
@@ -238,7 +260,8 @@ moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_
         else
             e = launch_wgrad_ffma(x, d_out, routing->offsets, routing->perm, T, E, H, g_div, part, part_db, s);
         if (e == cudaSuccess)
-            e = launch_wgrad_reduce(part, part_db, routing->offsets, T, E, H, g_scale, dW, db, acc_dw, acc_db, s);
+            e = launch_wgrad_reduce(part, part_db, routing->offsets, T, E, H, wgrad_splits(T), g_scale, dW, db, acc_dw,
+                                    acc_db, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
     return MOE_OK;
@@ -459,7 +482,8 @@ moe_status_t moe_aux_loss_fwd_bwd(const float* gate_logits, const int32_t* count
     if (device_info(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     return cuda_status(launch_aux(gate_logits, counts, T, E, lambda_eff, d_logits, loss_out, mean_p, stats,
-                                  reinterpret_cast<float*>(ws + L.aux_psum), static_cast<cudaStream_t>(stream)));
+                                  reinterpret_cast<float*>(ws + L.aux_psum),
+                                  reinterpret_cast<uint32_t*>(ws + kWsTicketOffset), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_lambda_eff_update(const float* ent_ema, float lambda_floor, float lambda_max_extra,

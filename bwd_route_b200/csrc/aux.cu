@@ -14,8 +14,8 @@
 // The logit gradient of token t needs only its own softmax row and the global
 // frac, so one streaming pass reads the logits once, writes d_logits and leaves
 // per-block sums of p (warps work on 32-token chunks staged in their own shared
-// buffers); a one-block kernel then sums those in a fixed order (mean_p, aux,
-// loss, stats). No atomics: every bit is reproducible.
+// buffers); the last block to finish then sums those in a fixed order (mean_p,
+// aux, loss, stats). No floating-point atomics: every bit is reproducible.
 #include <cstdint>
 
 #include "common.cuh"
@@ -40,6 +40,11 @@ __device__ __forceinline__ int row_slot(int t, int q) {
     return t * Q + (q ^ ((t >> SH) & (Q - 1)));
 }
 
+__device__ void aux_finalize_block(const float* blk_psum, int64_t nblk,
+                                   const int32_t* __restrict__ counts, int64_t T, int E,
+                                   const float* __restrict__ lambda_eff, float* __restrict__ loss_out,
+                                   float* __restrict__ mean_p, float* __restrict__ stats);
+
 // One block per 1024 consecutive tokens; warp w handles chunks w, w + 8, w + 16,
 // w + 24 of 32 tokens. The warp stages all four chunks' logits in its own
 // shared buffer (128-bit loads, every load in flight before the first use, no
@@ -50,7 +55,9 @@ template <int EMAX>
 __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__ logits,
                                                       const int32_t* __restrict__ counts, int64_t T, int E,
                                                       const float* __restrict__ lambda_eff,
-                                                      float* __restrict__ d_logits, float* __restrict__ blk_psum) {
+                                                      float* __restrict__ d_logits, float* __restrict__ blk_psum,
+                                                      uint32_t* __restrict__ ticket, float* __restrict__ loss_out,
+                                                      float* __restrict__ mean_p, float* __restrict__ stats) {
     constexpr int Q = EMAX / 4;          // float4s per staged row
     constexpr int BUF4 = kChunk * Q;     // float4s per chunk buffer
     extern __shared__ float4 s_dyn4[];   // kWarps x kChunksPerWarp chunk buffers
@@ -179,54 +186,63 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
         float acc = s_part[0][threadIdx.x];
         for (int w = 1; w < kWarps; ++w) acc += s_part[w][threadIdx.x];
         blk_psum[static_cast<int64_t>(blockIdx.x) * E + threadIdx.x] = acc;
+        __threadfence();  // this block's partials are visible before its ticket is taken
+    }
+    // The block that takes the last ticket (an integer counter in the workspace)
+    // finalizes: every other block's partials are in memory by then. The order of
+    // the sums does not depend on which block is last. The counter is reset for
+    // the next call.
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1) ? 1 : 0;
+    __syncthreads();
+    if (s_last) {
+        __threadfence();
+        aux_finalize_block(blk_psum, gridDim.x, counts, T, E, lambda_eff, loss_out, mean_p, stats);
+        if (threadIdx.x == 0) *ticket = 0u;
     }
 }
 
 // One block: mean_p from the per-block sums (double, fixed order), then aux,
-// loss, stats. Expert e's partial sums are split over the warps of group e
-// (32 / E warps; block b of the expert goes to thread b mod the group's
-// threads), summed per thread in block order, by an xor butterfly per warp and
-// across the group's warps in order.
-__global__ void __launch_bounds__(1024) aux_finalize_kernel(const float* __restrict__ blk_psum, int64_t nblk,
-                                                           const int32_t* __restrict__ counts, int64_t T, int E,
-                                                           const float* __restrict__ lambda_eff,
-                                                           float* __restrict__ loss_out, float* __restrict__ mean_p,
-                                                           float* __restrict__ stats) {
-    __shared__ double s_wsum[32];
+// loss, stats. Warp w takes experts w, w + nwarps, ...; lane l of it sums the
+// expert's per-block partials l, l + 32, l + 64, ... in block order (eight
+// loads in flight), then an xor butterfly combines the lanes.
+__device__ void aux_finalize_block(const float* blk_psum, int64_t nblk,
+                                   const int32_t* __restrict__ counts, int64_t T, int E,
+                                   const float* __restrict__ lambda_eff, float* __restrict__ loss_out,
+                                   float* __restrict__ mean_p, float* __restrict__ stats) {
+    __shared__ double s_sum[32];
     __shared__ float s_mean[32];
     __shared__ double s_hf[32], s_hm[32];
     __shared__ int s_cnt[32];
     __shared__ float s_lam;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wpe = 32 / E;                 // warps per expert
-    const int e = warp / wpe;               // expert of this warp (e >= E: idle)
-    const int g = (warp % wpe) * 32 + lane; // thread index inside the expert's group
-    const int G = wpe * 32;
+    const int nwarps = blockDim.x >> 5;
     if (threadIdx.x == 0) s_lam = *lambda_eff;
     if (threadIdx.x < E) s_cnt[threadIdx.x] = counts[threadIdx.x];
-    double acc = 0.0;
-    if (e < E) {
-        for (int64_t b0 = g; b0 < nblk; b0 += 8 * static_cast<int64_t>(G)) {
+    for (int e = warp; e < E; e += nwarps) {
+        double acc = 0.0;
+        for (int64_t b0 = lane; b0 < nblk; b0 += 8 * 32) {
             float v[8];  // eight independent loads, then added in block order
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t b = b0 + static_cast<int64_t>(u) * G;
-                v[u] = (b < nblk) ? blk_psum[b * E + e] : 0.0f;
+                const int64_t b = b0 + static_cast<int64_t>(u) * 32;
+                // written by other blocks of the same launch: read through L2 (coherent), not the
+                // non-coherent read-only path
+                v[u] = (b < nblk) ? __ldcg(blk_psum + b * E + e) : 0.0f;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                if (b0 + static_cast<int64_t>(u) * G < nblk) acc += static_cast<double>(v[u]);
+                if (b0 + static_cast<int64_t>(u) * 32 < nblk) acc += static_cast<double>(v[u]);
         }
-    }
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) s_wsum[warp] = acc;
+        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) s_sum[e] = acc;
+    }
     __syncthreads();
     if (threadIdx.x < E) {
         const int x = threadIdx.x;
-        double tot = 0.0;
-        for (int w = 0; w < wpe; ++w) tot += s_wsum[x * wpe + w];
-        const float m = T > 0 ? static_cast<float>(tot / static_cast<double>(T)) : 0.0f;
+        const float m = T > 0 ? static_cast<float>(s_sum[x] / static_cast<double>(T)) : 0.0f;
         s_mean[x] = m;
         // entropy terms of expert x (0 ln 0 = 0)
         const double f = T > 0 ? static_cast<double>(s_cnt[x]) / static_cast<double>(T) : 0.0;
@@ -258,6 +274,14 @@ __global__ void __launch_bounds__(1024) aux_finalize_kernel(const float* __restr
             stats[3 * E + 3] = static_cast<float>(hm);
         }
     }
+}
+
+// The empty batch: only the finalize (zeros, and lambda in the stats).
+__global__ void __launch_bounds__(kThreads) aux_finalize_kernel(const int32_t* __restrict__ counts, int E,
+                                                               const float* __restrict__ lambda_eff,
+                                                               float* __restrict__ loss_out, float* __restrict__ mean_p,
+                                                               float* __restrict__ stats) {
+    aux_finalize_block(nullptr, 0, counts, 0, E, lambda_eff, loss_out, mean_p, stats);
 }
 
 __global__ void lambda_eff_kernel(const float* __restrict__ ent_ema, float lambda_floor, float lambda_max_extra,
@@ -302,22 +326,25 @@ cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, fl
 
 cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, int E, const float* lambda_eff,
                        float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,
-                       cudaStream_t s) {
-    const int64_t nblk = T > 0 ? (T + kAuxTokPerBlk - 1) / kAuxTokPerBlk : 0;
-    if (T > 0) {
-        const size_t smem = sizeof(float) * kWarps * kChunksPerWarp * kChunk * (E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32);
-        if (E <= 4)
-            aux_kernel<4><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum);
-        else if (E <= 8)
-            aux_kernel<8><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum);
-        else if (E <= 16)
-            aux_kernel<16><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum);
-        else
-            aux_kernel<32><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum);
-        const cudaError_t err = cudaGetLastError();
-        if (err != cudaSuccess) return err;
+                       uint32_t* ticket, cudaStream_t s) {
+    if (T == 0) {
+        aux_finalize_kernel<<<1, kThreads, 0, s>>>(counts, E, lambda_eff, loss_out, mean_p, stats);
+        return cudaGetLastError();
     }
-    aux_finalize_kernel<<<1, 1024, 0, s>>>(blk_psum, nblk, counts, T, E, lambda_eff, loss_out, mean_p, stats);
+    const int64_t nblk = (T + kAuxTokPerBlk - 1) / kAuxTokPerBlk;
+    const size_t smem = sizeof(float) * kWarps * kChunksPerWarp * kChunk * (E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32);
+    if (E <= 4)
+        aux_kernel<4><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
+                                                            ticket, loss_out, mean_p, stats);
+    else if (E <= 8)
+        aux_kernel<8><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
+                                                            ticket, loss_out, mean_p, stats);
+    else if (E <= 16)
+        aux_kernel<16><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
+                                                             ticket, loss_out, mean_p, stats);
+    else
+        aux_kernel<32><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
+                                                             ticket, loss_out, mean_p, stats);
     return cudaGetLastError();
 }
 

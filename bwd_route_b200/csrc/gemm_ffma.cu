@@ -468,9 +468,8 @@ cudaError_t launch_wgrad_ffma(const float* x, const float* d_out, const int32_t*
 }
 
 cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const int32_t* offsets, int64_t T,
-                                int E, int H, float scale, float* dW, float* db, int acc_dw, int acc_db,
+                                int E, int H, int P, float scale, float* dW, float* db, int acc_dw, int acc_db,
                                 cudaStream_t s) {
-    const int P = wgrad_splits(T);
     const int64_t HH = static_cast<int64_t>(H) * H;
     const int nb_w = static_cast<int>((HH / 4 + 255) / 256);
     dim3 grid(nb_w + 1, E);

@@ -642,7 +642,7 @@ cudaError_t launch_grouped_tf32(const float* src, const float* W, const float* b
                                 int src_div, float out_scale, float* out, uint32_t* dev_flags, int num_sms,
                                 cudaStream_t s) {
     CUtensorMap tm_b;
-    const bool ok = w_transposed ? make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, 32, true)
+    const bool ok = w_transposed ? make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, 32, kMapSw128Atom32)
                                  : make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, H);
     if (!ok) return cudaErrorInvalidValue;
     const int64_t tiles = (T + 127) / 128 + E;

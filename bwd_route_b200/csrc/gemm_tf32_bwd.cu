@@ -1,0 +1,543 @@
+// gemm_tf32_bwd.cu -- the whole backward of the expert path (d_x, dW and db) in
+// one pass over d_out and x, on pairs of CTAs that share one tcgen05 MMA
+// (cta_group::2), for H = 256.
+//
+// foxhunt commit 11b96dac6a ("Top-1 Mixture-of-Experts gate per Switch
+// Transformer"), kernel list: one backward kernel produces the input gradient
+// (d_fused_ctx) and the expert weight and bias gradients together:
+//   d_x[t, i]   = sum_o W[e*, o, i] d_out[t, o]
+//   dW[e, o, i] = sum_{t in e} d_out[t, o] x[t, i],   db[e, o] = sum_{t in e} d_out[t, o].
+// Both contractions read the same d_out rows, so doing them in one kernel reads
+// d_out from memory once instead of twice.
+//
+// Tensor memory decides the shape. At H = 256 one expert's dW is 256 x 256 fp32
+// = all 512 columns of one SM's tensor memory, leaving nothing for d_x. A pair
+// of CTAs (a cluster of 2 on two SMs) shares every MMA: the accumulator's rows
+// are split between the two CTAs' tensor memories, so each CTA holds half of
+// dW's rows (256 columns) and the d_x rows of its own 128 tokens (256 columns).
+//
+// Work split. The expert-sorted token list is cut into P equal ranges (cut
+// again at expert boundaries), one per pair; range c of expert e gives the
+// partial-sum slot c + e, which the fixed-order slot reduction adds up (no
+// atomics: foxhunt commit b23f8f2efa, Discipline). A pair walks its range in
+// pair-tiles of 256 tokens of one expert; CTA v owns tokens 128 v .. 128 v +
+// 127 of each pair-tile. Per pair-tile the even CTA's MMA thread issues
+//   d_x: M = 256 tokens x N = 256 i x K = 256 o (8 stages of 32 o), A = the
+//        d_out rows of each CTA's tokens (K-major), B = W[e] read MN-major, CTA
+//        v holding the columns i in [128 v, 128 v + 128);
+//   dW:  M = 256 o x N = 256 i x K = the 256 tokens (8 stages of 32 tokens),
+//        A = d_out with CTA v holding the rows o in [128 v, +128), B = x with
+//        CTA v holding the columns i in [128 v, +128) (both MN-major).
+// d_out rows therefore reach shared memory twice (one copy per operand layout:
+// the tensor core takes TF32 K-major operands only with the 16-byte-granule
+// swizzle and MN-major ones only with the 32-byte-granule swizzle), but from
+// HBM once: the second read, by the same or the peer CTA, hits L2.
+//
+// Warp roles (each CTA): 0-7 drain the d_x accumulator (TMEM -> transpose in
+// shared memory -> token rows); 8-11 gather token rows with cp.async; 12: the
+// MMA issuer (even CTA) or the relay (odd CTA: once its stage has landed, it
+// makes it visible to the tensor core and arrives on the even CTA's barrier);
+// 13 loads the W[e] slab by TMA; 14-17 sum d_out over the staged tokens for db
+// and drain dW into the slot at the end of an expert's run.
+//
+// Every wait is bounded (common.cuh); a CTA that gives up records
+// MOE_FLAG_WAIT_TIMEOUT, waits for its own TMA loads in flight and leaves
+// through the pair's final cluster barrier, after the MMAs it issued are done.
+#include <cstdint>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kH = 256;
+constexpr int kHalf = 128;
+constexpr int kThreads = 576;
+constexpr int kEpiWarps = 8;     // warps 0-7
+constexpr int kProducer0 = 256;  // warps 8-11
+constexpr int kMmaWarp = 12;
+constexpr int kWLoadWarp = 13;
+constexpr int kDbWarp0 = 14;     // warps 14-17
+constexpr int kXStages = 3;
+constexpr int kWStages = 3;
+constexpr int kStageBytes = 32768;  // region 0 (A) and region 1 (B), 16 KiB each
+constexpr int kRegion = 16384;
+constexpr int kGroupBytes = 4096;   // MN-major: 32 rows x 128 bytes per 32-wide column group
+constexpr int kStgBytes = kEpiWarps * 32 * 128;
+constexpr int kTmemCols = 512;      // [0, 256) d_x, [256, 512) dW
+constexpr int kTileTok = 256;       // tokens per pair-tile
+
+struct __align__(8) Ctl {
+    uint64_t xfull[kXStages];   // even CTA: its 128 gather threads + the odd CTA's relay
+    uint64_t xready[kXStages];  // odd CTA: its 128 gather threads
+    uint64_t xtma[kXStages];    // each CTA: its own W-slab TMA (arrival + bytes)
+    uint64_t xempty[kXStages];  // each CTA: the pair's MMA commit
+    uint64_t wfull[kWStages];   // even CTA: 128 gather threads + relay
+    uint64_t wready[kWStages];  // odd CTA: 128 gather threads
+    uint64_t wempty[kWStages];  // each CTA: MMA commit + its 4 db warps
+    uint64_t dx_full;           // each CTA: MMA commit
+    uint64_t dx_empty;          // even CTA: the 8 d_x drain warps of both CTAs
+    uint64_t dw_full;           // each CTA: MMA commit
+    uint64_t dw_empty;          // even CTA: the 4 db / dW warps of both CTAs
+    uint64_t done;              // even CTA: the last commit
+    uint32_t tmem_base;
+    int abort;
+    int off[33];
+};
+
+constexpr int kSmemBytes = 1024 + (kXStages + kWStages) * kStageBytes + kStgBytes + static_cast<int>(sizeof(Ctl));
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+
+// The pair-tiles of range [lo, hi) of the sorted token list, in order: expert
+// e's run is [max(lo, off[e]), min(hi, off[e + 1])), cut into 256-token tiles.
+struct TileIter {
+    int e, p0, s, t;
+    __device__ void first(const int* off, int E, int lo, int hi) {
+        e = -1;
+        t = 0;
+        p0 = 0;
+        next_run(off, E, lo, hi);
+    }
+    __device__ void next_run(const int* off, int E, int lo, int hi) {
+        for (++e; e < E; ++e) {
+            s = max(lo, off[e]);
+            t = min(hi, off[e + 1]);
+            if (s < t) {
+                p0 = s;
+                return;
+            }
+        }
+    }
+    __device__ void next(const int* off, int E, int lo, int hi) {
+        p0 += kTileTok;
+        if (p0 >= t) next_run(off, E, lo, hi);
+    }
+    __device__ bool valid(int E) const { return e < E; }
+    __device__ int ntok() const { return min(kTileTok, t - p0); }
+    __device__ bool first_in_run() const { return p0 == s; }
+    __device__ bool last_in_run() const { return p0 + kTileTok >= t; }
+};
+
+__device__ __forceinline__ void advance(int& stage, uint32_t& phase, int n) {
+    if (++stage == n) {
+        stage = 0;
+        phase ^= 1;
+    }
+}
+
+// g_src: d_out, or the [B, H] gradient of the horizon mean (COLLAPSE: token t
+// reads row t / g_div and every result is scaled by out_scale).
+template <bool COLLAPSE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_src, const __grid_constant__ CUtensorMap tm_w,
+                      const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int T, int E, int P,
+                      int g_div, float out_scale, int acc_dx, float* __restrict__ d_x, float* __restrict__ part,
+                      float* __restrict__ part_db, uint32_t* __restrict__ dev_flags) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* xring = smem;
+    uint8_t* wring = smem + kXStages * kStageBytes;
+    float* stg = reinterpret_cast<float*>(smem + (kXStages + kWStages) * kStageBytes);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + (kXStages + kWStages) * kStageBytes + kStgBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t v = cluster_ctarank();  // 0: the even CTA, which issues the MMAs
+    const bool leader = (v == 0);
+    const int c = static_cast<int>(cluster_id_x());
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kXStages; ++s) {
+            mbar_init(&ctl->xfull[s], 128 + 1);
+            mbar_init(&ctl->xready[s], 128);
+            mbar_init(&ctl->xtma[s], 1);
+            mbar_init(&ctl->xempty[s], 1);
+        }
+        for (int s = 0; s < kWStages; ++s) {
+            mbar_init(&ctl->wfull[s], 128 + 1);
+            mbar_init(&ctl->wready[s], 128);
+            mbar_init(&ctl->wempty[s], 1 + 4);
+        }
+        mbar_init(&ctl->dx_full, 1);
+        mbar_init(&ctl->dx_empty, 2 * kEpiWarps);
+        mbar_init(&ctl->dw_full, 1);
+        mbar_init(&ctl->dw_empty, 2 * 4);
+        mbar_init(&ctl->done, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
+    if (warp == kWLoadWarp && lane == 0) tma_prefetch_desc(&tm_w);
+    if (warp == kMmaWarp) {
+        tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers initialised in both CTAs before any remote arrival
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+    const int lo = static_cast<int>(split_lo(c, T, P)), hi = static_cast<int>(split_lo(c + 1, T, P));
+    const int* off = ctl->off;
+
+    if (warp >= kProducer0 / 32 && warp < kProducer0 / 32 + 4) {
+        // ---------------- producers: cp.async gathers of the stages' token rows
+        const int ptid = threadIdx.x - kProducer0;  // 0..127
+        const int prow = ptid >> 3, pg = ptid & 7;  // X stages: row within a 16-row block, 16-byte granule
+        const int q16 = ptid & 7, gq = (ptid >> 3) & 3, rsub = ptid >> 5;  // W stages
+        int sx = 0, sw = 0;
+        uint32_t px = 0, pw = 0;
+        bool ok = true;
+        TileIter it;
+        it.first(off, E, lo, hi);
+        while (ok && it.valid(E)) {
+            const int n = it.ntok();
+            // this CTA's tokens for the X stages (rows r = j * 16 + prow) and the
+            // pair-tile's tokens for the W stages (lane l: token 32 tc + l)
+            int tx[8], tw[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = kHalf * static_cast<int>(v) + j * 16 + prow;
+                tx[j] = (r < n) ? perm[it.p0 + r] : -1;
+                const int q = j * 32 + lane;
+                tw[j] = (q < n) ? perm[it.p0 + q] : -1;
+            }
+            // X stages: A = d_out rows of this CTA's tokens, 32 o per stage, K-major
+            for (int kc = 0; kc < kH / 32 && ok; ++kc) {
+                if (!(ok = mbar_wait(&ctl->xempty[sx], px ^ 1, abort, dev_flags))) break;
+                const uint32_t a_u32 = smem_u32(xring + sx * kStageBytes);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = j * 16 + prow;
+                    const int tk = tx[j];
+                    const int gr = (COLLAPSE && tk >= 0) ? tk / g_div : tk;
+                    const float* src = g_src + static_cast<int64_t>(gr < 0 ? 0 : gr) * kH + kc * 32 + pg * 4;
+                    cp_async_16_l2_256(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), src, tk < 0 ? 0u : 16u);
+                }
+                cp_async_arrive_noinc(leader ? &ctl->xfull[sx] : &ctl->xready[sx]);
+                advance(sx, px, kXStages);
+            }
+            // W stages: 32 tokens each; A = d_out[., o-half v], B = x[., i-half v], MN-major
+            const int ntc = (n + 31) / 32;
+            for (int tc = 0; tc < ntc && ok; ++tc) {
+                if (!(ok = mbar_wait(&ctl->wempty[sw], pw ^ 1, abort, dev_flags))) break;
+                const uint32_t a_u32 = smem_u32(wring + sw * kStageBytes);
+                int tok_l = tw[0];
+#pragma unroll
+                for (int j = 1; j < 8; ++j)
+                    if (j == tc) tok_l = tw[j];
+                const int gtok_l = (COLLAPSE && tok_l >= 0) ? tok_l / g_div : tok_l;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = j * 4 + rsub;
+                    const int tk = __shfl_sync(0xffffffffu, tok_l, r);
+                    const int gtk = __shfl_sync(0xffffffffu, gtok_l, r);
+                    const uint32_t o = gq * kGroupBytes + r * 128 + ((((q16 >> 1) ^ (r & 3)) << 5) | ((q16 & 1) << 4));
+                    const int64_t col = kHalf * static_cast<int64_t>(v) + gq * 32 + q16 * 4;
+                    const uint32_t nb = tk < 0 ? 0u : 16u;
+                    cp_async_16(a_u32 + o, g_src + static_cast<int64_t>(tk < 0 ? 0 : gtk) * kH + col, nb);
+                    cp_async_16(a_u32 + kRegion + o, x + static_cast<int64_t>(tk < 0 ? 0 : tk) * kH + col, nb);
+                }
+                cp_async_arrive_noinc(leader ? &ctl->wfull[sw] : &ctl->wready[sw]);
+                advance(sw, pw, kWStages);
+            }
+            it.next(off, E, lo, hi);
+        }
+    } else if (warp == kWLoadWarp) {
+        // ---------------- W[e] slab (columns i of this CTA's half) for the X stages, by TMA
+        if (lane == 0) {
+            int sx = 0;
+            uint32_t px = 0;
+            int issued[kXStages] = {0, 0, 0};  // the parity + 1 of this stage's last load (0: none)
+            bool ok = true;
+            TileIter it;
+            it.first(off, E, lo, hi);
+            while (ok && it.valid(E)) {
+                for (int kc = 0; kc < kH / 32 && ok; ++kc) {
+                    if (!(ok = mbar_wait(&ctl->xempty[sx], px ^ 1, abort, dev_flags))) break;
+                    mbar_arrive_expect_tx(&ctl->xtma[sx], kRegion);
+                    uint8_t* dst = xring + sx * kStageBytes + kRegion;
+#pragma unroll
+                    for (int g = 0; g < kHalf / 32; ++g)
+                        tma_load_2d(dst + g * kGroupBytes, &tm_w, kHalf * static_cast<int>(v) + g * 32,
+                                    it.e * kH + kc * 32, &ctl->xtma[sx]);
+                    issued[sx] = static_cast<int>(px) + 1;
+                    advance(sx, px, kXStages);
+                }
+                it.next(off, E, lo, hi);
+            }
+            // let this CTA's loads land before it can leave (already so unless a wait gave up)
+            for (int s = 0; s < kXStages; ++s)
+                if (issued[s]) mbar_wait_drain(&ctl->xtma[s], static_cast<uint32_t>(issued[s] - 1), kWaitLimitCycles);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (leader && lane == 0) {
+            // ---------------- MMA issuer: one thread of the even CTA, for both CTAs
+            constexpr uint32_t idesc_dx = idesc_tf32(256, 256, 0, 1);  // A K-major, B MN-major
+            constexpr uint32_t idesc_dw = idesc_tf32(256, 256, 1, 1);  // both MN-major
+            const uint32_t tmem_dx = tmem, tmem_dw = tmem + kH;
+            int sx = 0, sw = 0;
+            uint32_t px = 0, pw = 0, dx_phase = 0, dw_phase = 0;
+            bool ok = true;
+            TileIter it;
+            it.first(off, E, lo, hi);
+            while (ok && it.valid(E)) {
+                // d_x of this pair-tile: the accumulator must have been drained by both CTAs
+                if (!(ok = mbar_wait_cl(&ctl->dx_empty, dx_phase ^ 1, abort, dev_flags))) break;
+                tc_fence_after();
+                for (int kc = 0; kc < kH / 32; ++kc) {
+                    if (!(ok = mbar_wait_cl(&ctl->xfull[sx], px, abort, dev_flags))) break;
+                    if (!(ok = mbar_wait(&ctl->xtma[sx], px, abort, dev_flags))) break;
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(xring + sx * kStageBytes);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_tf32_pair(tmem_dx, sw128_desc(a_addr + ks * 32, 16, 1024),
+                                      sw128_32b_mn_desc(a_addr + kRegion + ks * 1024, kGroupBytes, 512), idesc_dx,
+                                      (kc | ks) != 0 ? 1u : 0u);
+                    mma_commit_pair_mc(&ctl->xempty[sx], 0x3);
+                    advance(sx, px, kXStages);
+                }
+                if (!ok) break;
+                mma_commit_pair_mc(&ctl->dx_full, 0x3);
+                dx_phase ^= 1;
+                // dW of this pair-tile, accumulated over the expert's run
+                if (it.first_in_run()) {
+                    if (!(ok = mbar_wait_cl(&ctl->dw_empty, dw_phase ^ 1, abort, dev_flags))) break;
+                    tc_fence_after();
+                }
+                const int ntc = (it.ntok() + 31) / 32;
+                for (int tc = 0; tc < ntc; ++tc) {
+                    if (!(ok = mbar_wait_cl(&ctl->wfull[sw], pw, abort, dev_flags))) break;
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(wring + sw * kStageBytes);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_tf32_pair(tmem_dw, sw128_32b_mn_desc(a_addr + ks * 1024, kGroupBytes, 512),
+                                      sw128_32b_mn_desc(a_addr + kRegion + ks * 1024, kGroupBytes, 512), idesc_dw,
+                                      (it.first_in_run() && tc == 0 && ks == 0) ? 0u : 1u);
+                    mma_commit_pair_mc(&ctl->wempty[sw], 0x3);
+                    advance(sw, pw, kWStages);
+                }
+                if (!ok) break;
+                if (it.last_in_run()) {
+                    mma_commit_pair_mc(&ctl->dw_full, 0x3);
+                    dw_phase ^= 1;
+                }
+                it.next(off, E, lo, hi);
+            }
+            // every MMA issued (and every commit arrival on the odd CTA) is done before the pair may leave
+            mma_commit_pair(&ctl->done);
+            mbar_wait_drain(&ctl->done, 0, kWaitLimitCycles);
+        } else if (!leader && lane == 0) {
+            // ---------------- relay (odd CTA): this CTA's stage has landed -> the even CTA's barrier
+            const uint32_t xfull0 = mapa_shared(smem_u32(&ctl->xfull[0]), 0);
+            const uint32_t wfull0 = mapa_shared(smem_u32(&ctl->wfull[0]), 0);
+            int sx = 0, sw = 0;
+            uint32_t px = 0, pw = 0;
+            bool ok = true;
+            TileIter it;
+            it.first(off, E, lo, hi);
+            while (ok && it.valid(E)) {
+                for (int kc = 0; kc < kH / 32; ++kc) {
+                    if (!(ok = mbar_wait(&ctl->xready[sx], px, abort, dev_flags))) break;
+                    if (!(ok = mbar_wait(&ctl->xtma[sx], px, abort, dev_flags))) break;
+                    fence_proxy_async_smem();
+                    mbar_arrive_cluster(xfull0 + sx * 8);
+                    advance(sx, px, kXStages);
+                }
+                if (!ok) break;
+                const int ntc = (it.ntok() + 31) / 32;
+                for (int tc = 0; tc < ntc; ++tc) {
+                    if (!(ok = mbar_wait(&ctl->wready[sw], pw, abort, dev_flags))) break;
+                    fence_proxy_async_smem();
+                    mbar_arrive_cluster(wfull0 + sw * 8);
+                    advance(sw, pw, kWStages);
+                }
+                it.next(off, E, lo, hi);
+            }
+        }
+        __syncwarp();
+    } else if (warp < kEpiWarps) {
+        // ---------------- d_x drain: TMEM -> registers -> shared-memory transpose -> token rows.
+        // Warp w reads TMEM lanes 32 (w % 4) .. +31 (this CTA's tile rows) and the column half w / 4.
+        const int q = warp & 3;
+        const int c0 = (warp >> 2) * kHalf;
+        const uint32_t my_u32 = smem_u32(stg + warp * 32 * 32);
+        const int j = lane & 7;
+        const int myrow = kHalf * static_cast<int>(v) + 32 * q + lane;  // position within the pair-tile
+        const uint32_t dx_empty0 = mapa_shared(smem_u32(&ctl->dx_empty), 0);
+        uint32_t dx_phase = 0;
+        TileIter it;
+        it.first(off, E, lo, hi);
+        int tok_next = it.valid(E) ? ((myrow < it.ntok()) ? perm[it.p0 + myrow] : -1) : -1;
+        while (it.valid(E)) {
+            const int tok_mine = tok_next;
+            TileIter nx = it;
+            nx.next(off, E, lo, hi);
+            tok_next = nx.valid(E) ? ((myrow < nx.ntok()) ? perm[nx.p0 + myrow] : -1) : -1;
+            if (!mbar_wait_cl(&ctl->dx_full, dx_phase, abort, dev_flags)) break;
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < kHalf / 32; ++cc) {
+                float vals[32];
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0 + cc * 32),
+                                   vals);
+                if (COLLAPSE) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) vals[i] *= out_scale;
+                }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    st_shared_v4(my_u32 + 4 * (lane * 32 + ((jj ^ (lane & 7)) * 4)), vals[4 * jj], vals[4 * jj + 1],
+                                 vals[4 * jj + 2], vals[4 * jj + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int r8 = 0; r8 < 8; ++r8) {
+                    const int R = r8 * 4 + (lane >> 3);
+                    float4 val = ld_shared_v4(my_u32 + 4 * (R * 32 + ((j ^ (R & 7)) * 4)));
+                    const int tok = __shfl_sync(0xffffffffu, tok_mine, R);
+                    float* dst = d_x + static_cast<int64_t>(tok < 0 ? 0 : tok) * kH + c0 + cc * 32 + j * 4;
+                    if (acc_dx) {
+                        if (tok >= 0) {
+                            const float4 o = *reinterpret_cast<const float4*>(dst);
+                            val.x += o.x;
+                            val.y += o.y;
+                            val.z += o.z;
+                            val.w += o.w;
+                            *reinterpret_cast<float4*>(dst) = val;
+                        }
+                    } else {
+                        st_global_cs_v4_pred(dst, val, tok >= 0);
+                    }
+                }
+                __syncwarp();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(dx_empty0);
+            dx_phase ^= 1;
+            it = nx;
+        }
+    } else if (warp >= kDbWarp0 && warp < kDbWarp0 + 4) {
+        // ---------------- db over the staged d_out rows (column o = 128 v + tdb), and
+        // the dW drain of TMEM lane quadrant warp % 4 at the end of each expert run
+        const int tdb = threadIdx.x - kDbWarp0 * 32;  // 0..127
+        const int dq = warp & 3;
+        const int g = tdb >> 5, jo = tdb & 31;
+        const uint32_t dw_empty0 = mapa_shared(smem_u32(&ctl->dw_empty), 0);
+        int sw = 0;
+        uint32_t pw = 0, dw_phase = 0;
+        float db_run = 0.0f;
+        bool ok = true;
+        TileIter it;
+        it.first(off, E, lo, hi);
+        while (ok && it.valid(E)) {
+            const int ntc = (it.ntok() + 31) / 32;
+            for (int tc = 0; tc < ntc; ++tc) {
+                ok = leader ? mbar_wait_cl(&ctl->wfull[sw], pw, abort, dev_flags)
+                            : mbar_wait(&ctl->wready[sw], pw, abort, dev_flags);
+                if (!ok) break;
+                const uint8_t* colbase = wring + sw * kStageBytes + g * kGroupBytes + (jo & 7) * 4;
+                float acc = 0.0f;
+#pragma unroll 8
+                for (int rr = 0; rr < 32; ++rr)
+                    acc += *reinterpret_cast<const float*>(colbase + rr * 128 + (((jo >> 3) ^ (rr & 3)) << 5));
+                db_run += acc;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->wempty[sw]);
+                advance(sw, pw, kWStages);
+            }
+            if (!ok) break;
+            if (it.last_in_run()) {
+                if (!(ok = mbar_wait_cl(&ctl->dw_full, dw_phase, abort, dev_flags))) break;
+                __syncwarp();
+                tc_fence_after();
+                const int64_t slot = static_cast<int64_t>(c) + it.e;
+                const int o = kHalf * static_cast<int>(v) + 32 * dq + lane;  // dW row of this TMEM lane
+                float* prow = part + (slot * kH + o) * kH;
+#pragma unroll 1
+                for (int cc = 0; cc < kH / 32; ++cc) {
+                    float vals[32];
+                    tmem_ld_32x32b_x32(tmem + kH + (static_cast<uint32_t>(32 * dq) << 16) + static_cast<uint32_t>(cc * 32),
+                                       vals);
+#pragma unroll
+                    for (int k4 = 0; k4 < 8; ++k4)
+                        *reinterpret_cast<float4*>(prow + cc * 32 + 4 * k4) =
+                            make_float4(vals[4 * k4], vals[4 * k4 + 1], vals[4 * k4 + 2], vals[4 * k4 + 3]);
+                }
+                part_db[slot * kH + kHalf * static_cast<int>(v) + tdb] = db_run;
+                db_run = 0.0f;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(dw_empty0);
+                dw_phase ^= 1;
+            }
+            it.next(off, E, lo, hi);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while the peer may still arrive on its barriers
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+// Pairs (clusters of 2) that fit on the device at once, at most kFusedMaxPairs.
+cudaError_t bwd_fused_max_pairs(int* out) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * kFusedMaxPairs, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, bwd_fused_tf32_kernel<false>, &cfg);
+    if (e != cudaSuccess) return e;
+    *out = n < 1 ? 1 : (n > kFusedMaxPairs ? kFusedMaxPairs : n);
+    return cudaSuccess;
+}
+
+int bwd_fused_pairs(int64_t T, int max_pairs) {
+    int64_t p = (T + 2 * kTileTok - 1) / (2 * kTileTok);
+    if (p < 1) p = 1;
+    if (p > max_pairs) p = max_pairs;
+    return static_cast<int>(p);
+}
+
+cudaError_t launch_bwd_fused_tf32(const float* x, const float* W, const float* g_src, const int32_t* offsets,
+                                  const int32_t* perm, int64_t T, int E, int P, int g_div, float out_scale, int acc_dx,
+                                  float* d_x, float* part, float* part_db, uint32_t* dev_flags, cudaStream_t s) {
+    CUtensorMap tm_w;
+    if (!make_map_2d(&tm_w, W, static_cast<uint64_t>(E) * kH, kH, 32, 32, kMapSw128Atom32)) return cudaErrorInvalidValue;
+    if (g_div != 1 || out_scale != 1.0f)
+        bwd_fused_tf32_kernel<true><<<2 * P, kThreads, kSmemBytes, s>>>(
+            x, g_src, tm_w, offsets, perm, static_cast<int>(T), E, P, g_div, out_scale, acc_dx, d_x, part, part_db,
+            dev_flags);
+    else
+        bwd_fused_tf32_kernel<false><<<2 * P, kThreads, kSmemBytes, s>>>(
+            x, g_src, tm_w, offsets, perm, static_cast<int>(T), E, P, 1, 1.0f, acc_dx, d_x, part, part_db, dev_flags);
+    return cudaGetLastError();
+}
+
+cudaError_t bwd_fused_set_smem_limits() {
+    cudaError_t e = cudaFuncSetAttribute(bwd_fused_tf32_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(bwd_fused_tf32_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    return e;
+}
+
+}  // namespace moe

@@ -348,6 +348,384 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
     }
 }
 
+// ------------------------------------------------------------------ the same mean, raw rows staged by TMA (E <= 8)
+// Same result definition and the same arithmetic as hmean_fwd_tf32_kernel (X_be
+// summed in fp32 in ascending h; the MMA products of (e, k) added into TMEM;
+// then sum_e n_be bias[e] and the 1/N_H scale), organised so that memory
+// latency is never exposed: x is streamed into shared memory by TMA in raw
+// stages of 8 batch rows x N_H tokens x 16 columns (the tile's rows are one
+// contiguous block of x), and reducer warps build X_be for all experts of one
+// 16-column k-chunk from them. Every CTA owns a contiguous range of batch rows
+// (B / grid each), walked in tiles of 128 rows, so no wave of tiles is left
+// half-empty.
+//   warps 0-3   epilogue: TMEM lane quadrant = warp, all H columns
+//   warps 4-11  reducers: raw stage (k-chunk kc, row group g) goes to warp g % 8
+//   warp 12     MMA issuer: per k-chunk, for each expert, 2 MMAs of K = 8 on
+//               X_be (64-byte swizzle, K-major) and the W[e] k-chunk
+//   warp 13     raw x stages by TMA (no swizzle: rows of 16 floats)
+//   warp 14     W[e] k-chunks by TMA (64-byte swizzle)
+constexpr int kSThreads = 480;
+constexpr int kSEpiWarps = 4;
+constexpr int kSRed0 = 4;
+constexpr int kSReducers = 8;
+constexpr int kSMmaWarp = 12;
+constexpr int kSRawWarp = 13;
+constexpr int kSWWarp = 14;
+constexpr int kSMaxE = 8;
+constexpr int kSRowsPerStage = 8;
+constexpr int kSGroups = 16;  // row groups per 128-row tile
+constexpr int kSRawMaxStages = 16;
+constexpr int kSBStages = 3;
+
+struct __align__(8) SCtl {
+    uint64_t raw_full[kSRawMaxStages];
+    uint64_t raw_empty[kSRawMaxStages];
+    uint64_t a_full, a_empty;
+    uint64_t b_full[kSBStages];
+    uint64_t b_empty[kSBStages];
+    uint64_t t_full[2];
+    uint64_t t_empty[2];
+    uint64_t order_full, order_empty;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int H>
+struct SCfg {
+    static constexpr int BM = 128;
+    static constexpr int KC = H / 16;                           // 16-column k-chunks
+    static constexpr int A_BYTES = BM * 64;                     // X_be of one expert and k-chunk: 8 KiB
+    static constexpr int A_REGION = kSMaxE * A_BYTES;           // 64 KiB
+    static constexpr int B_BYTES = H * 64;                      // W[e] k-chunk
+    static constexpr int RAW_BUDGET = 96 * 1024;
+    static constexpr int ORDER_BYTES = BM * kHMaxHorizon * 2;   // uint16 (h | e << 8) per row and slot
+    static constexpr int BIAS_BYTES = kSMaxE * H * 4;
+    static constexpr int TMEM_COLS = 2 * H;
+    static constexpr int SMEM_BYTES = 1024 + A_REGION + kSBStages * B_BYTES + RAW_BUDGET + ORDER_BYTES + BIAS_BYTES +
+                                      static_cast<int>(sizeof(SCtl));
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ void advance_stage(int& s, uint32_t& ph, int n) {
+    if (++s == n) {
+        s = 0;
+        ph ^= 1;
+    }
+}
+
+template <int H>
+__global__ void __launch_bounds__(kSThreads, 1)
+hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                          const float* __restrict__ bias, const int32_t* __restrict__ expert_idx, int B, int N_H,
+                          int E, float inv_nh, int raw_stages, float* __restrict__ out,
+                          uint32_t* __restrict__ dev_flags) {
+    using C = SCfg<H>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* aregion = smem;
+    uint8_t* bring = aregion + C::A_REGION;
+    uint8_t* rawring = bring + kSBStages * C::B_BYTES;
+    uint16_t* order = reinterpret_cast<uint16_t*>(rawring + C::RAW_BUDGET);
+    float* bias_s = reinterpret_cast<float*>(rawring + C::RAW_BUDGET + C::ORDER_BYTES);
+    SCtl* ctl = reinterpret_cast<SCtl*>(rawring + C::RAW_BUDGET + C::ORDER_BYTES + C::BIAS_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int raw_bytes = kSRowsPerStage * N_H * 64;
+    const int64_t b_lo = static_cast<int64_t>(B) * blockIdx.x / gridDim.x;
+    const int64_t b_hi = static_cast<int64_t>(B) * (blockIdx.x + 1) / gridDim.x;
+    const int ntiles = static_cast<int>((b_hi - b_lo + C::BM - 1) / C::BM);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < raw_stages; ++s) {
+            mbar_init(&ctl->raw_full[s], 1);   // arrive.expect_tx + TMA bytes
+            mbar_init(&ctl->raw_empty[s], 1);  // the reducer warp that read it
+        }
+        mbar_init(&ctl->a_full, kSGroups);     // one arrival per row group of the k-chunk
+        mbar_init(&ctl->a_empty, 1);           // tcgen05.commit
+        for (int s = 0; s < kSBStages; ++s) {
+            mbar_init(&ctl->b_full[s], 1);
+            mbar_init(&ctl->b_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->t_full[b], 1);
+            mbar_init(&ctl->t_empty[b], kSEpiWarps);
+        }
+        mbar_init(&ctl->order_full, kSReducers);
+        mbar_init(&ctl->order_empty, kSReducers);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    for (int k = threadIdx.x; k < E * H / 4; k += blockDim.x)
+        reinterpret_cast<float4*>(bias_s)[k] = __ldg(reinterpret_cast<const float4*>(bias) + k);
+    if (warp == kSRawWarp && lane == 0) tma_prefetch_desc(&tm_x);
+    if (warp == kSWWarp && lane == 0) tma_prefetch_desc(&tm_w);
+    if (warp == kSMmaWarp) {
+        tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+
+    if (warp == kSRawWarp) {
+        // ---------------- raw stages: rows (b0 + 8 g) * N_H .. + 8 N_H - 1 of x, columns 16 kc .. + 15
+        if (lane == 0) {
+            int slot = 0;
+            uint32_t ph = 0;
+            int issued[kSRawMaxStages];
+            for (int s = 0; s < kSRawMaxStages; ++s) issued[s] = 0;
+            bool ok = true;
+            for (int tile = 0; tile < ntiles && ok; ++tile) {
+                const int64_t b0 = b_lo + static_cast<int64_t>(tile) * C::BM;
+                const int nrows = static_cast<int>(b_hi - b0 < C::BM ? b_hi - b0 : C::BM);
+                const int ngroups = (nrows + kSRowsPerStage - 1) / kSRowsPerStage;
+                for (int kc = 0; kc < C::KC && ok; ++kc) {
+                    for (int g = 0; g < ngroups; ++g) {
+                        if (!(ok = mbar_wait(&ctl->raw_empty[slot], ph ^ 1, abort, dev_flags))) break;
+                        mbar_arrive_expect_tx(&ctl->raw_full[slot], raw_bytes);
+                        tma_load_2d(rawring + slot * raw_bytes, &tm_x, kc * 16,
+                                    static_cast<int32_t>((b0 + kSRowsPerStage * g) * N_H), &ctl->raw_full[slot]);
+                        issued[slot] = static_cast<int>(ph) + 1;
+                        advance_stage(slot, ph, raw_stages);
+                    }
+                }
+            }
+            for (int s = 0; s < raw_stages; ++s)
+                if (issued[s]) mbar_wait_drain(&ctl->raw_full[s], static_cast<uint32_t>(issued[s] - 1), kWaitLimitCycles);
+        }
+        __syncwarp();
+    } else if (warp == kSWWarp) {
+        // ---------------- W[e] k-chunks, in the MMA's (kc, e) order
+        if (lane == 0) {
+            int sb = 0;
+            uint32_t pb = 0;
+            int issued[kSBStages] = {0, 0, 0};
+            bool ok = true;
+            for (int tile = 0; tile < ntiles && ok; ++tile) {
+                for (int kc = 0; kc < C::KC && ok; ++kc) {
+                    for (int e = 0; e < E; ++e) {
+                        if (!(ok = mbar_wait(&ctl->b_empty[sb], pb ^ 1, abort, dev_flags))) break;
+                        mbar_arrive_expect_tx(&ctl->b_full[sb], C::B_BYTES);
+                        tma_load_2d(bring + sb * C::B_BYTES, &tm_w, kc * 16, e * H, &ctl->b_full[sb]);
+                        issued[sb] = static_cast<int>(pb) + 1;
+                        advance_stage(sb, pb, kSBStages);
+                    }
+                }
+            }
+            for (int s = 0; s < kSBStages; ++s)
+                if (issued[s]) mbar_wait_drain(&ctl->b_full[s], static_cast<uint32_t>(issued[s] - 1), kWaitLimitCycles);
+        }
+        __syncwarp();
+    } else if (warp >= kSRed0 && warp < kSRed0 + kSReducers) {
+        // ---------------- reducers
+        const int rw = warp - kSRed0;
+        const int r = lane >> 2, q4 = lane & 3;
+        const uint32_t a_u32 = smem_u32(aregion);
+        const uint32_t raw_u32 = smem_u32(rawring);
+        int64_t qtile = 0;  // raw stages issued before this tile
+        uint32_t pa = 0;
+        bool ok = true;
+        for (int tile = 0; tile < ntiles && ok; ++tile) {
+            const int64_t b0 = b_lo + static_cast<int64_t>(tile) * C::BM;
+            const int nrows = static_cast<int>(b_hi - b0 < C::BM ? b_hi - b0 : C::BM);
+            const int ngroups = (nrows + kSRowsPerStage - 1) / kSRowsPerStage;
+            // the tile's tokens of each row, grouped by expert in ascending h: this
+            // warp builds rows 16 rw .. 16 rw + 15 once every warp is done with the
+            // previous tile's list
+            if (!(ok = mbar_wait(&ctl->order_empty, (tile & 1) ^ 1, abort, dev_flags))) break;
+            if (lane < 16) {
+                const int m = rw * 16 + lane;
+                uint16_t* ord = order + m * kHMaxHorizon;
+                int cnt[kSMaxE + 1];
+#pragma unroll
+                for (int e = 0; e <= kSMaxE; ++e) cnt[e] = 0;
+                const bool valid = m < nrows;
+                const int32_t* idx = expert_idx + (b0 + m) * N_H;
+                for (int h = 0; h < N_H; ++h) {
+                    const int e = valid ? idx[h] : -1;
+                    const int k = (e >= 0 && e < E) ? e : kSMaxE;
+#pragma unroll
+                    for (int f = 0; f <= kSMaxE; ++f) cnt[f] += (f == k) ? 1 : 0;
+                }
+                int pos[kSMaxE + 1];
+                int acc = 0;
+#pragma unroll
+                for (int f = 0; f <= kSMaxE; ++f) {
+                    pos[f] = acc;
+                    acc += cnt[f];
+                }
+                for (int h = 0; h < N_H; ++h) {
+                    const int e = valid ? idx[h] : -1;
+                    const int k = (e >= 0 && e < E) ? e : kSMaxE;
+                    int p = 0;
+#pragma unroll
+                    for (int f = 0; f <= kSMaxE; ++f)
+                        if (f == k) p = pos[f]++;
+                    ord[p] = static_cast<uint16_t>(h | ((k == kSMaxE ? 0xFF : k) << 8));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->order_full);
+            if (!(ok = mbar_wait(&ctl->order_full, tile & 1, abort, dev_flags))) break;
+            for (int kc = 0; kc < C::KC && ok; ++kc) {
+                // the MMAs of the previous k-chunk have read the X_be region
+                if (!(ok = mbar_wait(&ctl->a_empty, pa ^ 1, abort, dev_flags))) break;
+#pragma unroll 1
+                for (int g = rw; g < kSGroups; g += kSReducers) {
+                    if (g < ngroups) {
+                        const int64_t q = qtile + static_cast<int64_t>(kc) * ngroups + g;
+                        const int slot = static_cast<int>(q % raw_stages);
+                        if (!(ok = mbar_wait(&ctl->raw_full[slot], static_cast<uint32_t>((q / raw_stages) & 1), abort,
+                                             dev_flags)))
+                            break;
+                        const int m = g * kSRowsPerStage + r;
+                        const uint16_t* ord = order + m * kHMaxHorizon;
+                        const uint32_t rb = raw_u32 + slot * raw_bytes + r * N_H * 64 + q4 * 16;
+                        const uint32_t arow = a_u32 + m * 64 + ((q4 ^ ((m >> 1) & 3)) << 4);
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        int cur = -1;
+                        uint32_t present = 0;
+                        for (int j = 0; j < N_H; ++j) {
+                            const uint32_t o = ord[j];
+                            const int e = static_cast<int>(o >> 8);
+                            if (e >= E) break;  // out-of-range experts sort last and add nothing
+                            const float4 v = ld_shared_v4(rb + (o & 0xFFu) * 64);
+                            if (e != cur) {
+                                if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
+                                acc = v;
+                                cur = e;
+                                present |= 1u << e;
+                            } else {
+                                acc.x += v.x;
+                                acc.y += v.y;
+                                acc.z += v.z;
+                                acc.w += v.w;
+                            }
+                        }
+                        if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
+                        for (int e = 0; e < E; ++e)
+                            if (!((present >> e) & 1u)) st_shared_v4(arow + e * C::A_BYTES, 0.f, 0.f, 0.f, 0.f);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ctl->raw_empty[slot]);
+                    }
+                    fence_proxy_async_smem();  // the MMA reads these stores through the async proxy
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->a_full);
+                }
+                pa ^= 1;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->order_empty);
+            qtile += static_cast<int64_t>(C::KC) * ngroups;
+        }
+    } else if (warp == kSMmaWarp) {
+        // ---------------- MMA issuer (one thread)
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_tf32(128, H, 0, 0);
+            const uint32_t a_u32 = smem_u32(aregion);
+            int sb = 0;
+            uint32_t pb = 0, pa = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = 0; tile < ntiles && ok; ++tile) {
+                if (!(ok = mbar_wait(&ctl->t_empty[acc], acc_phase ^ 1, abort, dev_flags))) break;
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(acc * H);
+                uint32_t accumulate = 0;
+                for (int kc = 0; kc < C::KC && ok; ++kc) {
+                    if (!(ok = mbar_wait(&ctl->a_full, pa, abort, dev_flags))) break;
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    for (int e = 0; e < E; ++e) {
+                        if (!(ok = mbar_wait(&ctl->b_full[sb], pb, abort, dev_flags))) break;
+                        tc_fence_after();
+                        const uint32_t b_addr = smem_u32(bring + sb * C::B_BYTES);
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            mma_tf32(d, sw64_desc(a_u32 + e * C::A_BYTES + ks * 32, 512), sw64_desc(b_addr + ks * 32, 512),
+                                     idesc, accumulate);
+                            accumulate = 1u;
+                        }
+                        mma_commit(&ctl->b_empty[sb]);
+                        advance_stage(sb, pb, kSBStages);
+                    }
+                    if (!ok) break;
+                    mma_commit(&ctl->a_empty);
+                    pa ^= 1;
+                }
+                if (!ok) break;
+                mma_commit(&ctl->t_full[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+        }
+        __syncwarp();
+    } else if (warp < kSEpiWarps) {
+        // ---------------- epilogue: row m = 32 q + lane of the tile, all H columns;
+        // (acc + sum_e n_be bias[e]) / N_H with n_be counted from the row's experts
+        const int q = warp;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = 0; tile < ntiles; ++tile) {
+            const int64_t b = b_lo + static_cast<int64_t>(tile) * C::BM + 32 * q + lane;
+            const bool valid = b < b_hi;
+            int cnt[kSMaxE];
+#pragma unroll
+            for (int e = 0; e < kSMaxE; ++e) cnt[e] = 0;
+            if (valid) {
+                for (int h = 0; h < N_H; ++h) {
+                    const int e = expert_idx[b * N_H + h];
+#pragma unroll
+                    for (int f = 0; f < kSMaxE; ++f) cnt[f] += (f == e) ? 1 : 0;
+                }
+            }
+            const bool ok = mbar_wait(&ctl->t_full[acc], acc_phase, abort, dev_flags);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < H / 32; ++cc) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * H + cc * 32),
+                                   v);
+#pragma unroll
+                for (int e = 0; e < kSMaxE; ++e) {
+                    if (e >= E) break;
+                    const float n = static_cast<float>(cnt[e]);
+                    if (!__any_sync(0xffffffffu, n != 0.0f)) continue;
+                    const float4* bs = reinterpret_cast<const float4*>(bias_s + e * H + cc * 32);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 bb = bs[j];
+                        v[4 * j] = fmaf(n, bb.x, v[4 * j]);
+                        v[4 * j + 1] = fmaf(n, bb.y, v[4 * j + 1]);
+                        v[4 * j + 2] = fmaf(n, bb.z, v[4 * j + 2]);
+                        v[4 * j + 3] = fmaf(n, bb.w, v[4 * j + 3]);
+                    }
+                }
+                if (valid) {
+                    float4* dst = reinterpret_cast<float4*>(out + b * H + cc * 32);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        __stcs(dst + j, make_float4(v[4 * j] * inv_nh, v[4 * j + 1] * inv_nh, v[4 * j + 2] * inv_nh,
+                                                    v[4 * j + 3] * inv_nh));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->t_empty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kSMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -358,6 +736,26 @@ cudaError_t set_smem(K kernel, int bytes) {
 cudaError_t launch_hmean_fwd_tf32(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
                                   int64_t B, int N_H, int E, int H, float* out, uint32_t* dev_flags, int num_sms,
                                   cudaStream_t s) {
+    if (E <= kSMaxE) {
+        // raw rows staged by TMA; every CTA owns B / grid batch rows
+        CUtensorMap tm_x, tm_w;
+        const uint64_t T = static_cast<uint64_t>(B) * N_H;
+        if (!make_map_2d(&tm_x, x, T, H, 16, static_cast<uint32_t>(kSRowsPerStage * N_H), kMapPlain) ||
+            !make_map_2d(&tm_w, W, static_cast<uint64_t>(E) * H, H, 16, H, kMapSw64))
+            return cudaErrorInvalidValue;
+        const int raw_bytes = kSRowsPerStage * N_H * 64;
+        int raw_stages = SCfg<256>::RAW_BUDGET / raw_bytes;
+        if (raw_stages > kSRawMaxStages) raw_stages = kSRawMaxStages;
+        const int grid = static_cast<int>(B < num_sms ? B : num_sms);
+        const float inv_nh = static_cast<float>(1.0 / static_cast<double>(N_H));
+        if (H == 256)
+            hmean_fwd_tf32_sum_kernel<256><<<grid, kSThreads, SCfg<256>::SMEM_BYTES, s>>>(
+                tm_x, tm_w, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, raw_stages, out, dev_flags);
+        else
+            hmean_fwd_tf32_sum_kernel<128><<<grid, kSThreads, SCfg<128>::SMEM_BYTES, s>>>(
+                tm_x, tm_w, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, raw_stages, out, dev_flags);
+        return cudaGetLastError();
+    }
     CUtensorMap tm_b;
     if (!make_map_2d(&tm_b, W, static_cast<uint64_t>(E) * H, H, 32, H)) return cudaErrorInvalidValue;
     const int64_t tiles = (B + 127) / 128;
@@ -375,6 +773,8 @@ cudaError_t launch_hmean_fwd_tf32(const float* x, const float* W, const float* b
 cudaError_t hmean_set_smem_limits() {
     cudaError_t e = set_smem(hmean_fwd_tf32_kernel<256>, HCfg<256>::SMEM_BYTES);
     if (e == cudaSuccess) e = set_smem(hmean_fwd_tf32_kernel<128>, HCfg<128>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(hmean_fwd_tf32_sum_kernel<256>, SCfg<256>::SMEM_BYTES);
+    if (e == cudaSuccess) e = set_smem(hmean_fwd_tf32_sum_kernel<128>, SCfg<128>::SMEM_BYTES);
     return e;
 }
 

@@ -28,6 +28,10 @@ inline int wgrad_splits(int64_t T) {
 // First sorted position of split c (floor(c * T / P)); ranges are [lo(c), lo(c+1)).
 __host__ __device__ inline int64_t split_lo(int c, int64_t T, int P) { return (static_cast<int64_t>(c) * T) / P; }
 
+// Byte offset, inside the workspace's 256-byte head, of the aux kernel's ticket
+// counter (the flag word is at 0).
+constexpr size_t kWsTicketOffset = 64;
+
 struct WsLayout {
     size_t flags = 0;        // uint32 flag word (256 B reserved)
     size_t route_counts = 0; // int32 [nblk_route][E]
@@ -72,9 +76,11 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
                          int32_t* offsets, int32_t* perm, int32_t* blk_counts, int32_t* blk_base,
                          cudaStream_t s);
 
+// ticket: a uint32 of the workspace's reserved head (zeroed by
+// moe_top1_workspace_init); the aux kernel's last block resets it after use.
 cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, int E, const float* lambda_eff,
                        float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,
-                       cudaStream_t s);
+                       uint32_t* ticket, cudaStream_t s);
 
 cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, float alpha, int reset,
                                      float* usage_ema, float* ent_ema, float* ent_step, cudaStream_t s);
@@ -107,10 +113,27 @@ cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t*
                               int64_t T, int E, int H, int g_div, float* part, float* part_db, uint32_t* dev_flags,
                               cudaStream_t s);
 // Fixed-order pairwise sum of the slots of each expert, times scale, into dW / db
-// (either may be null).
+// (either may be null). P: the number of ranges the partial sums were cut into
+// (wgrad_splits(T) for the weight-gradient kernels, the pair count for the
+// fused backward).
 cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const int32_t* offsets, int64_t T,
-                                int E, int H, float scale, float* dW, float* db, int acc_dw, int acc_db,
+                                int E, int H, int P, float scale, float* dW, float* db, int acc_dw, int acc_db,
                                 cudaStream_t s);
+
+// The fused TF32 backward at H = 256 (d_x, and dW / db partial sums into the
+// slots, in one pass over d_out and x) on P pairs of CTAs; range c of expert e
+// gives slot c + e. Token t's gradient row is g_src[t / g_div]; d_x is scaled by
+// out_scale (the slot reduction applies it to dW and db).
+constexpr int kFusedMaxPairs = 74;
+cudaError_t launch_bwd_fused_tf32(const float* x, const float* W, const float* g_src, const int32_t* offsets,
+                                  const int32_t* perm, int64_t T, int E, int P, int g_div, float out_scale, int acc_dx,
+                                  float* d_x, float* part, float* part_db, uint32_t* dev_flags, cudaStream_t s);
+// Pairs that run at once on the current device (at most kFusedMaxPairs).
+cudaError_t bwd_fused_max_pairs(int* out);
+// Pairs used for T tokens: one per 512 tokens, at most max_pairs (<= wgrad_splits(T),
+// so the slots fit the workspace).
+int bwd_fused_pairs(int64_t T, int max_pairs);
+cudaError_t bwd_fused_set_smem_limits();
 
 // Driver entry point for tensor-map encoding (resolved at run time, so the
 // library does not link libcuda).
@@ -119,13 +142,19 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn get_encode_tiled();
 
-// 2D fp32 tensor [rows][cols] with a 128-byte-swizzled box of box_cols x box_rows
-// (16-byte granules, or 32-byte granules when atom32 is set). make_map_2d returns
-// a cached copy when the same map was encoded before on this device;
-// encode_map_2d always encodes.
+// Shared-memory layouts a 2D tensor map writes its boxes in.
+enum MapLayout : int {
+    kMapSw128 = 0,        // 128-byte swizzle, 16-byte granules (box_cols = 32 floats)
+    kMapSw128Atom32 = 1,  // 128-byte swizzle, 32-byte granules (box_cols = 32 floats)
+    kMapSw64 = 2,         // 64-byte swizzle, 16-byte granules (box_cols = 16 floats)
+    kMapPlain = 3         // no swizzle: rows of box_cols floats, back to back
+};
+// 2D fp32 tensor [rows][cols] with a box of box_cols x box_rows in the given
+// layout. make_map_2d returns a cached copy when the same map was encoded before
+// on this device; encode_map_2d always encodes.
 bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                 uint32_t box_rows, bool atom32 = false);
+                 uint32_t box_rows, int layout = kMapSw128);
 bool encode_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                   uint32_t box_rows, bool atom32);
+                   uint32_t box_rows, int layout);
 
 }  // namespace moe

@@ -10,7 +10,8 @@
 // scan's result (equal values, -0 / +0 included, keep the lower index; NaN
 // entries are never chosen; a NaN at e = 0 pins the result to 0).
 //
-// Three launches, all integer-exact and deterministic:
+// Three launches (two while nblk x E <= 32768: the scan then runs inside every
+// scatter block), all integer-exact and deterministic:
 //   1. route_count   : E a multiple of 4: one thread per token scans its row
 //                      (128-bit loads); other E: each warp loads its 128
 //                      tokens' logits (a lane group of LPT lanes per token, 16
@@ -285,6 +286,105 @@ __global__ void __launch_bounds__(kThreads) route_scatter_kernel(const int32_t* 
     }
 }
 
+// The scan folded into the scatter: every block reads the per-block counts of
+// all blocks (nblk x E integers, L2-resident) and computes, with exact integer
+// sums, the expert totals and its own base in each expert's segment:
+//   base[b][e] = offsets[e] + sum_{b' < b} blk_counts[b'][e],
+//   offsets[e] = sum_{e' < e} counts[e'],   counts[e] = sum_{b'} blk_counts[b'][e];
+// block 0 also writes counts and offsets. Thread i reads expert e = i % EP
+// (EP = E rounded up to a power of two, so a thread always sees the same expert)
+// of blocks i / EP, i / EP + 256 / EP, ...; lanes of one expert combine with xor
+// shuffles, warps through shared-memory integer adds. Then the tokens are
+// scattered exactly as route_scatter_kernel does. Used while nblk x E is small
+// enough that reading it in every block is cheaper than a separate scan launch.
+constexpr int64_t kPrefixMaxEntries = 32768;
+
+__global__ void __launch_bounds__(kThreads) route_scatter_prefix_kernel(const int32_t* __restrict__ expert_idx,
+                                                                       int64_t T, int E, int EP, int64_t nblk,
+                                                                       const int32_t* __restrict__ blk_counts,
+                                                                       int32_t* __restrict__ counts,
+                                                                       int32_t* __restrict__ offsets,
+                                                                       int32_t* __restrict__ perm) {
+    __shared__ int s_before[32], s_total[32], s_base[32];
+    __shared__ int s_pos[kWarps][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < 32) {
+        s_before[threadIdx.x] = 0;
+        s_total[threadIdx.x] = 0;
+    }
+    __syncthreads();
+    {
+        const int e = threadIdx.x % EP;
+        const int step = kThreads / EP;
+        int before = 0, total = 0;
+        if (e < E) {
+            for (int64_t b = threadIdx.x / EP; b < nblk; b += step) {
+                const int v = blk_counts[b * E + e];
+                total += v;
+                if (b < static_cast<int64_t>(blockIdx.x)) before += v;
+            }
+        }
+        // lanes e, e + EP, e + 2 EP, ... of this warp hold expert e (EP <= 32)
+        for (int off = 16; off >= EP; off >>= 1) {
+            before += __shfl_xor_sync(0xffffffffu, before, off);
+            total += __shfl_xor_sync(0xffffffffu, total, off);
+        }
+        if (lane < EP && e < E) {
+            atomicAdd(&s_before[e], before);
+            atomicAdd(&s_total[e], total);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int e = 0; e < E; ++e) {
+            if (blockIdx.x == 0) {
+                offsets[e] = acc;
+                counts[e] = s_total[e];
+            }
+            s_base[e] = acc + s_before[e];
+            acc += s_total[e];
+        }
+        if (blockIdx.x == 0) offsets[E] = acc;
+    }
+    s_pos[warp][lane] = 0;
+    __syncthreads();
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokPerBlk + warp * kTokPerWarp;
+    constexpr int IT = kTokPerWarp / 32;
+    const unsigned lt = (1u << lane) - 1u;
+    int k[IT];
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+        const int64_t t = t0 + it * 32 + lane;
+        k[it] = (t < T) ? expert_idx[t] : -1;
+    }
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+        const unsigned same = __match_any_sync(0xffffffffu, k[it]);
+        if (k[it] >= 0 && (same & lt) == 0) s_pos[warp][k[it]] += __popc(same);
+        __syncwarp();
+    }
+    __syncthreads();
+    int run = 0;
+    if (lane < E) {
+        run = s_base[lane];
+        for (int w = 0; w < warp; ++w) run += s_pos[w][lane];
+    }
+    __syncthreads();
+    if (lane < E) s_pos[warp][lane] = run;
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+        const int kk = k[it];
+        const unsigned same = __match_any_sync(0xffffffffu, kk);
+        const int base = kk >= 0 ? s_pos[warp][kk] : 0;
+        if (kk >= 0) perm[base + __popc(same & lt)] = static_cast<int32_t>(t0 + it * 32 + lane);
+        __syncwarp();
+        if (kk >= 0 && (same & lt) == 0) s_pos[warp][kk] = base + __popc(same);
+        __syncwarp();
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_idx, int32_t* counts,
@@ -307,6 +407,13 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
         route_count_kernel<16><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
     else
         route_count_kernel<32><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+    if (nblk * E <= kPrefixMaxEntries) {
+        int ep = 1;
+        while (ep < E) ep <<= 1;
+        route_scatter_prefix_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(expert_idx, T, E, ep, nblk, blk_counts, counts,
+                                                                        offsets, perm);
+        return cudaGetLastError();
+    }
     route_scan_kernel<<<1, 1024, 0, s>>>(blk_counts, nblk, E, counts, offsets, blk_base);
     route_scatter_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(expert_idx, T, E, blk_base, perm);
     return cudaGetLastError();

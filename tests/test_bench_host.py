@@ -18,7 +18,13 @@ def test_algorithmic_bytes_and_flops_of_the_throughput_workload():
     assert step_bytes == T * (4 * (5 * H + 3 * E) + 16) + 2 * E * H * H * 4
     assert abs(step_bytes - 5.49e9) < 0.01e9
     assert step_flops == 6 * H * H * T
-    assert per["fwd"] == per["d_x"] + E * H * 4 == T * (8 * H + 4) + E * H * H * 4 + E * H * 4
+    assert per["fwd"] == T * (8 * H + 4) + E * H * H * 4 + E * H * 4
+    # the backward call reads x and d_out once and writes d_x: 12 H bytes per token
+    assert per["bwd"] == T * (12 * H + 4) + 2 * E * H * H * 4 + E * H * 4
+    # the step's bytes are the two calls' plus the routing and aux traffic (logits read
+    # twice, d_logits written, expert_idx written, perm written), less what the calls
+    # count and the step does not (W read by both calls but counted once, bias and db)
+    assert step_bytes - (per["fwd"] + per["bwd"]) == T * (4 * 3 * E + 8) - E * H * H * 4 - 2 * E * H * 4
     # the step roofline quoted in the docs: HBM-bound at the measured 6541 GB/s
     assert abs(step_bytes / 6541e9 * 1e6 - 839) < 1
 
@@ -31,7 +37,7 @@ def test_algorithmic_bytes_with_the_horizon_mean_gradient():
     # d_out [T, H] is read once and routed [T, H] written once in the plain step;
     # the [B, H] gradient and the [B, H] mean replace them
     assert full - coll == 2 * (T * H * 4 - B * H * 4)
-    assert per["d_x"] - per_c["d_x"] == T * H * 4 - B * H * 4
+    assert per["bwd"] - per_c["bwd"] == T * H * 4 - B * H * 4
     assert per["fwd"] - per_c["fwd"] == T * H * 4 - B * H * 4
 
 

@@ -164,6 +164,64 @@ def test_straight_through_expert_path_gives_the_logits_no_gradient(math_mode):
     assert not np.array_equal(aux_grad(logits * 2.0, r2).cpu().numpy(), before)
 
 
+# The TF32 backward at H = 256 with d_x and dW / db requested runs as one fused
+# kernel on CTA pairs (256-token pair-tiles of one expert, 512 tokens per pair at
+# least). Shapes that stress its tiling: a pair-tile the odd CTA has no token of,
+# one it has a few of, one pair only, segments far shorter than a pair-tile
+# (32 experts), a range that crosses several expert boundaries at odd positions,
+# and more pairs than fit on the GPU at once.
+FUSED_SHAPES = [
+    wl.make_spec("fused_b100_e3_h256", 100, 1, 3, 256, 81),
+    wl.make_spec("fused_b300_e1_h256", 300, 1, 1, 256, 82),
+    wl.make_spec("fused_b333_h3_e2_h256", 333, 3, 2, 256, 83),
+    wl.make_spec("fused_b2000_h2_e32_h256", 2000, 2, 32, 256, 84, skew_expert=7, skew_value=1.5),
+    wl.make_spec("fused_b16384_h5_e5_h256", 16384, 5, 5, 256, 85),
+    wl.make_spec("fused_b5000_h9_e8_h256", 5000, 9, 8, 256, 86, logits="binary"),
+]
+
+
+@pytest.mark.parametrize("spec", FUSED_SHAPES, ids=lambda s: s.name)
+def test_fused_backward_parity(spec):
+    check_all(wl.generate(spec), ops.MOE_MATH_TF32)
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+def test_backward_outputs_requested_separately(math_mode):
+    """d_x alone, dW and db alone, db alone and all three (at H = 256 with TF32
+    the last is the fused kernel, the others the separate contraction kernels):
+    every combination against the oracle."""
+    spec = wl.make_spec("bwd_parts_b1200_h3_e6_h256", 1200, 3, 6, 256, 87)
+    inp = wl.generate(spec)
+    B, N_H, E, H, T = spec.B, spec.N_H, spec.E, spec.H, spec.T
+    mode = tf32_mode(math_mode)
+    atol, rtol = TOL[math_mode]
+    idx = oracle.route(inp.gate_logits)[0]
+    want_dx = oracle.bwd_dx(inp.W, inp.d_out, idx, mode)
+    want_dw, want_db, sW, sb = oracle.bwd_dw(inp.x, inp.d_out, idx, E, mode)
+    x, W, d_out = dev(inp.x), dev(inp.W), dev(inp.d_out)
+    r = ops.Routing.empty(T, E, "cuda")
+    ws = ops.new_workspace(T, E, H, "cuda")
+    ops.moe_top1_route(dev(inp.gate_logits), B, N_H, E, r, ws)
+    for want in (("d_x",), ("dW", "db"), ("db",), ("d_x", "dW", "db")):
+        out = {"d_x": torch.full((T, H), float("nan"), device="cuda"),
+               "dW": torch.full((E, H, H), float("nan"), device="cuda"),
+               "db": torch.full((E, H), float("nan"), device="cuda")}
+        args = {k: (out[k] if k in want else None) for k in out}
+        ops.moe_top1_bwd(x, W, d_out, r, B, N_H, E, H, math_mode, args["d_x"], args["dW"], args["db"], 0, ws)
+        torch.cuda.synchronize()
+        assert ops.moe_top1_device_flags(ws) == 0
+        for k in ("d_x", "dW", "db"):
+            g = out[k].cpu().numpy()
+            if k not in want:
+                assert np.isnan(g).all(), (want, k)  # not written
+        if "d_x" in want:
+            assert_close(f"d_x {want}", out["d_x"].cpu().numpy(), want_dx, atol, rtol)
+        if "dW" in want:
+            assert_close(f"dW {want}", out["dW"].cpu().numpy(), want_dw, atol, rtol, scale=sW)
+        if "db" in want:
+            assert_close(f"db {want}", out["db"].cpu().numpy(), want_db, atol, rtol, scale=sb)
+
+
 def test_identity_experts_bit_exact():
     inp = wl.generate(wl.WORKLOADS["tiny_identity_b8_e4_h128"])
     g = run_gpu(inp, ops.MOE_MATH_FFMA, 0.01, parts=("route", "fwd"))
