@@ -477,7 +477,7 @@ def main():
         t_roof = max(step_bytes / (hbm * 1e9), step_flops / (tf32_sus * 1e12))
         value = job_throughput(world, T, ms_per_step)
         dominant = max(["fwd", "bwd"], key=lambda n: call_ms[n])
-        fused = math_mode == ops.MOE_MATH_TF32 and H == 256
+        fused = math_mode == ops.MOE_MATH_TF32
         achieved = kbytes[dominant] / (call_ms[dominant] * 1e-3) / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

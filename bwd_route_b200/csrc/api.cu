@@ -230,13 +230,15 @@ moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
-    if (math == MOE_MATH_TF32 && H == 256 && d_x && (dW || db)) {
-        // one pass over d_out: d_x, and the dW / db partial sums, then the slot reduction
+    if (math == MOE_MATH_TF32 && d_x && (dW || db)) {
+        // one pass over d_out: d_x, and the dW / db partial sums, then the slot reduction.
+        // H = 256: pairs of CTAs (as many as run at once); H = 128: single CTAs, one
+        // per wgrad_splits(T) range
         float* part = reinterpret_cast<float*>(ws + L.wg_part);
         float* part_db = reinterpret_cast<float*>(ws + L.wg_part_db);
-        if (dev->fused_pairs < 1) return MOE_ERR_CUDA;
-        const int P = bwd_fused_pairs(T, dev->fused_pairs);
-        e = launch_bwd_fused_tf32(x, W, d_out, routing->offsets, routing->perm, T, E, P, g_div, g_scale, acc_dx, d_x,
+        if (H == 256 && dev->fused_pairs < 1) return MOE_ERR_CUDA;
+        const int P = H == 256 ? bwd_fused_pairs(T, dev->fused_pairs) : wgrad_splits(T);
+        e = launch_bwd_fused_tf32(x, W, d_out, routing->offsets, routing->perm, T, E, H, P, g_div, g_scale, acc_dx, d_x,
                                   part, part_db, flags, s);
         if (e == cudaSuccess)
             e = launch_wgrad_reduce(part, part_db, routing->offsets, T, E, H, P, g_scale, dW, db, acc_dw, acc_db, s);

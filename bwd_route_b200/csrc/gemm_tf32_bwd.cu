@@ -1,6 +1,6 @@
 // gemm_tf32_bwd.cu -- the whole backward of the expert path (d_x, dW and db) in
-// one pass over d_out and x, on pairs of CTAs that share one tcgen05 MMA
-// (cta_group::2), for H = 256.
+// one pass over d_out and x: at H = 256 on pairs of CTAs that share one tcgen05
+// MMA (cta_group::2), at H = 128 on single CTAs.
 //
 // foxhunt commit 11b96dac6a ("Top-1 Mixture-of-Experts gate per Switch
 // Transformer"), kernel list: one backward kernel produces the input gradient
@@ -40,6 +40,11 @@
 // 13 loads the W[e] slab by TMA; 14-17 sum d_out over the staged tokens for db
 // and drain dW into the slot at the end of an expert's run.
 //
+// At H = 128 a CTA's tensor memory holds all of dW (128 columns) and its d_x
+// (128 columns), so the same kernel runs on single CTAs: 128-token tiles, one
+// range per CTA (slot c + e as above), M = 128 MMAs, no relay, and every
+// barrier arrival local.
+//
 // Every wait is bounded (common.cuh); a CTA that gives up records
 // MOE_FLAG_WAIT_TIMEOUT, waits for its own TMA loads in flight and leaves
 // through the pair's final cluster barrier, after the MMAs it issued are done.
@@ -51,8 +56,7 @@
 namespace moe {
 namespace {
 
-constexpr int kH = 256;
-constexpr int kHalf = 128;
+constexpr int kHalf = 128;         // operand width each CTA holds (columns of B, rows of dW's A)
 constexpr int kThreads = 576;
 constexpr int kEpiWarps = 8;     // warps 0-7
 constexpr int kProducer0 = 256;  // warps 8-11
@@ -65,8 +69,6 @@ constexpr int kStageBytes = 32768;  // region 0 (A) and region 1 (B), 16 KiB eac
 constexpr int kRegion = 16384;
 constexpr int kGroupBytes = 4096;   // MN-major: 32 rows x 128 bytes per 32-wide column group
 constexpr int kStgBytes = kEpiWarps * 32 * 128;
-constexpr int kTmemCols = 512;      // [0, 256) d_x, [256, 512) dW
-constexpr int kTileTok = 256;       // tokens per pair-tile
 
 struct __align__(8) Ctl {
     uint64_t xfull[kXStages];   // even CTA: its 128 gather threads + the odd CTA's relay
@@ -89,8 +91,9 @@ struct __align__(8) Ctl {
 constexpr int kSmemBytes = 1024 + (kXStages + kWStages) * kStageBytes + kStgBytes + static_cast<int>(sizeof(Ctl));
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// The pair-tiles of range [lo, hi) of the sorted token list, in order: expert
-// e's run is [max(lo, off[e]), min(hi, off[e + 1])), cut into 256-token tiles.
+// The tiles of range [lo, hi) of the sorted token list, in order: expert e's
+// run is [max(lo, off[e]), min(hi, off[e + 1])), cut into TILE-token tiles.
+template <int TILE>
 struct TileIter {
     int e, p0, s, t;
     __device__ void first(const int* off, int E, int lo, int hi) {
@@ -110,13 +113,13 @@ struct TileIter {
         }
     }
     __device__ void next(const int* off, int E, int lo, int hi) {
-        p0 += kTileTok;
+        p0 += TILE;
         if (p0 >= t) next_run(off, E, lo, hi);
     }
     __device__ bool valid(int E) const { return e < E; }
-    __device__ int ntok() const { return min(kTileTok, t - p0); }
+    __device__ int ntok() const { return min(TILE, t - p0); }
     __device__ bool first_in_run() const { return p0 == s; }
-    __device__ bool last_in_run() const { return p0 + kTileTok >= t; }
+    __device__ bool last_in_run() const { return p0 + TILE >= t; }
 };
 
 __device__ __forceinline__ void advance(int& stage, uint32_t& phase, int n) {
@@ -126,14 +129,30 @@ __device__ __forceinline__ void advance(int& stage, uint32_t& phase, int n) {
     }
 }
 
+// One arrival on the even CTA's barrier `bar` (PAIR), or on this CTA's.
+template <bool PAIR>
+__device__ __forceinline__ void arrive_on_leader(uint64_t* bar) {
+    if (PAIR)
+        mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
+    else
+        mbar_arrive(bar);
+}
+
 // g_src: d_out, or the [B, H] gradient of the horizon mean (COLLAPSE: token t
 // reads row t / g_div and every result is scaled by out_scale).
-template <bool COLLAPSE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_src, const __grid_constant__ CUtensorMap tm_w,
-                      const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int T, int E, int P,
-                      int g_div, float out_scale, int acc_dx, float* __restrict__ d_x, float* __restrict__ part,
-                      float* __restrict__ part_db, uint32_t* __restrict__ dev_flags) {
+template <int H, bool PAIR, bool COLLAPSE>
+__device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, const float* __restrict__ g_src,
+                                               const CUtensorMap* tm_w, const int32_t* __restrict__ offsets,
+                                               const int32_t* __restrict__ perm, int T, int E, int P, int g_div,
+                                               float out_scale, int acc_dx, float* __restrict__ d_x,
+                                               float* __restrict__ part, float* __restrict__ part_db,
+                                               uint32_t* __restrict__ dev_flags) {
+    static_assert((PAIR && H == 256) || (!PAIR && H == 128), "pairs at H = 256, single CTAs at H = 128");
+    constexpr int kH = H;
+    constexpr int kTileTok = PAIR ? 256 : 128;   // tokens per (pair-)tile
+    constexpr int kTmemCols = 2 * H;             // [0, H) d_x, [H, 2H) dW
+    constexpr int kM = PAIR ? 256 : 128;         // MMA rows: tokens (d_x) or o (dW)
+    using Iter = TileIter<kTileTok>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* xring = smem;
@@ -141,38 +160,46 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
     float* stg = reinterpret_cast<float*>(smem + (kXStages + kWStages) * kStageBytes);
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + (kXStages + kWStages) * kStageBytes + kStgBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t v = cluster_ctarank();  // 0: the even CTA, which issues the MMAs
+    const uint32_t v = PAIR ? cluster_ctarank() : 0u;  // 0: the even CTA, which issues the MMAs
     const bool leader = (v == 0);
-    const int c = static_cast<int>(cluster_id_x());
+    const int c = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kXStages; ++s) {
-            mbar_init(&ctl->xfull[s], 128 + 1);
+            mbar_init(&ctl->xfull[s], 128 + (PAIR ? 1 : 0));
             mbar_init(&ctl->xready[s], 128);
             mbar_init(&ctl->xtma[s], 1);
             mbar_init(&ctl->xempty[s], 1);
         }
         for (int s = 0; s < kWStages; ++s) {
-            mbar_init(&ctl->wfull[s], 128 + 1);
+            mbar_init(&ctl->wfull[s], 128 + (PAIR ? 1 : 0));
             mbar_init(&ctl->wready[s], 128);
             mbar_init(&ctl->wempty[s], 1 + 4);
         }
         mbar_init(&ctl->dx_full, 1);
-        mbar_init(&ctl->dx_empty, 2 * kEpiWarps);
+        mbar_init(&ctl->dx_empty, (PAIR ? 2 : 1) * kEpiWarps);
         mbar_init(&ctl->dw_full, 1);
-        mbar_init(&ctl->dw_empty, 2 * 4);
+        mbar_init(&ctl->dw_empty, (PAIR ? 2 : 1) * 4);
         mbar_init(&ctl->done, 1);
         ctl->abort = 0;
         fence_mbar_init();
     }
     if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
-    if (warp == kWLoadWarp && lane == 0) tma_prefetch_desc(&tm_w);
+    if (warp == kWLoadWarp && lane == 0) tma_prefetch_desc(tm_w);
     if (warp == kMmaWarp) {
-        tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
-        tmem_relinquish_pair();
+        if (PAIR) {
+            tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&ctl->tmem_base, kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    cluster_sync_all();  // barriers initialised in both CTAs before any remote arrival
+    if (PAIR)
+        cluster_sync_all();  // barriers initialised in both CTAs before any remote arrival
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
     volatile int* abort = &ctl->abort;
@@ -187,7 +214,7 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
         int sx = 0, sw = 0;
         uint32_t px = 0, pw = 0;
         bool ok = true;
-        TileIter it;
+        Iter it;
         it.first(off, E, lo, hi);
         while (ok && it.valid(E)) {
             const int n = it.ntok();
@@ -249,7 +276,7 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
             uint32_t px = 0;
             int issued[kXStages] = {0, 0, 0};  // the parity + 1 of this stage's last load (0: none)
             bool ok = true;
-            TileIter it;
+            Iter it;
             it.first(off, E, lo, hi);
             while (ok && it.valid(E)) {
                 for (int kc = 0; kc < kH / 32 && ok; ++kc) {
@@ -258,7 +285,7 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
                     uint8_t* dst = xring + sx * kStageBytes + kRegion;
 #pragma unroll
                     for (int g = 0; g < kHalf / 32; ++g)
-                        tma_load_2d(dst + g * kGroupBytes, &tm_w, kHalf * static_cast<int>(v) + g * 32,
+                        tma_load_2d(dst + g * kGroupBytes, tm_w, kHalf * static_cast<int>(v) + g * 32,
                                     it.e * kH + kc * 32, &ctl->xtma[sx]);
                     issued[sx] = static_cast<int>(px) + 1;
                     advance(sx, px, kXStages);
@@ -273,13 +300,20 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
     } else if (warp == kMmaWarp) {
         if (leader && lane == 0) {
             // ---------------- MMA issuer: one thread of the even CTA, for both CTAs
-            constexpr uint32_t idesc_dx = idesc_tf32(256, 256, 0, 1);  // A K-major, B MN-major
-            constexpr uint32_t idesc_dw = idesc_tf32(256, 256, 1, 1);  // both MN-major
+            constexpr uint32_t idesc_dx = idesc_tf32(kM, kH, 0, 1);  // A K-major, B MN-major
+            constexpr uint32_t idesc_dw = idesc_tf32(kM, kH, 1, 1);  // both MN-major
             const uint32_t tmem_dx = tmem, tmem_dw = tmem + kH;
+            // completion of the MMAs issued so far -> the barrier in every CTA of the pair
+            auto commit_all = [](uint64_t* bar) {
+                if (PAIR)
+                    mma_commit_pair_mc(bar, 0x3);
+                else
+                    mma_commit(bar);
+            };
             int sx = 0, sw = 0;
             uint32_t px = 0, pw = 0, dx_phase = 0, dw_phase = 0;
             bool ok = true;
-            TileIter it;
+            Iter it;
             it.first(off, E, lo, hi);
             while (ok && it.valid(E)) {
                 // d_x of this pair-tile: the accumulator must have been drained by both CTAs
@@ -292,15 +326,20 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(xring + sx * kStageBytes);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_tf32_pair(tmem_dx, sw128_desc(a_addr + ks * 32, 16, 1024),
-                                      sw128_32b_mn_desc(a_addr + kRegion + ks * 1024, kGroupBytes, 512), idesc_dx,
-                                      (kc | ks) != 0 ? 1u : 0u);
-                    mma_commit_pair_mc(&ctl->xempty[sx], 0x3);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = sw128_desc(a_addr + ks * 32, 16, 1024);
+                        const uint64_t bd = sw128_32b_mn_desc(a_addr + kRegion + ks * 1024, kGroupBytes, 512);
+                        const uint32_t accumulate = (kc | ks) != 0 ? 1u : 0u;
+                        if (PAIR)
+                            mma_tf32_pair(tmem_dx, ad, bd, idesc_dx, accumulate);
+                        else
+                            mma_tf32(tmem_dx, ad, bd, idesc_dx, accumulate);
+                    }
+                    commit_all(&ctl->xempty[sx]);
                     advance(sx, px, kXStages);
                 }
                 if (!ok) break;
-                mma_commit_pair_mc(&ctl->dx_full, 0x3);
+                commit_all(&ctl->dx_full);
                 dx_phase ^= 1;
                 // dW of this pair-tile, accumulated over the expert's run
                 if (it.first_in_run()) {
@@ -314,31 +353,39 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(wring + sw * kStageBytes);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_tf32_pair(tmem_dw, sw128_32b_mn_desc(a_addr + ks * 1024, kGroupBytes, 512),
-                                      sw128_32b_mn_desc(a_addr + kRegion + ks * 1024, kGroupBytes, 512), idesc_dw,
-                                      (it.first_in_run() && tc == 0 && ks == 0) ? 0u : 1u);
-                    mma_commit_pair_mc(&ctl->wempty[sw], 0x3);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = sw128_32b_mn_desc(a_addr + ks * 1024, kGroupBytes, 512);
+                        const uint64_t bd = sw128_32b_mn_desc(a_addr + kRegion + ks * 1024, kGroupBytes, 512);
+                        const uint32_t accumulate = (it.first_in_run() && tc == 0 && ks == 0) ? 0u : 1u;
+                        if (PAIR)
+                            mma_tf32_pair(tmem_dw, ad, bd, idesc_dw, accumulate);
+                        else
+                            mma_tf32(tmem_dw, ad, bd, idesc_dw, accumulate);
+                    }
+                    commit_all(&ctl->wempty[sw]);
                     advance(sw, pw, kWStages);
                 }
                 if (!ok) break;
                 if (it.last_in_run()) {
-                    mma_commit_pair_mc(&ctl->dw_full, 0x3);
+                    commit_all(&ctl->dw_full);
                     dw_phase ^= 1;
                 }
                 it.next(off, E, lo, hi);
             }
             // every MMA issued (and every commit arrival on the odd CTA) is done before the pair may leave
-            mma_commit_pair(&ctl->done);
+            if (PAIR)
+                mma_commit_pair(&ctl->done);
+            else
+                mma_commit(&ctl->done);
             mbar_wait_drain(&ctl->done, 0, kWaitLimitCycles);
-        } else if (!leader && lane == 0) {
+        } else if (PAIR && !leader && lane == 0) {
             // ---------------- relay (odd CTA): this CTA's stage has landed -> the even CTA's barrier
             const uint32_t xfull0 = mapa_shared(smem_u32(&ctl->xfull[0]), 0);
             const uint32_t wfull0 = mapa_shared(smem_u32(&ctl->wfull[0]), 0);
             int sx = 0, sw = 0;
             uint32_t px = 0, pw = 0;
             bool ok = true;
-            TileIter it;
+            Iter it;
             it.first(off, E, lo, hi);
             while (ok && it.valid(E)) {
                 for (int kc = 0; kc < kH / 32; ++kc) {
@@ -363,26 +410,26 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
     } else if (warp < kEpiWarps) {
         // ---------------- d_x drain: TMEM -> registers -> shared-memory transpose -> token rows.
         // Warp w reads TMEM lanes 32 (w % 4) .. +31 (this CTA's tile rows) and the column half w / 4.
+        constexpr int kCols = kH / 2;  // d_x columns this warp drains
         const int q = warp & 3;
-        const int c0 = (warp >> 2) * kHalf;
+        const int c0 = (warp >> 2) * kCols;
         const uint32_t my_u32 = smem_u32(stg + warp * 32 * 32);
         const int j = lane & 7;
-        const int myrow = kHalf * static_cast<int>(v) + 32 * q + lane;  // position within the pair-tile
-        const uint32_t dx_empty0 = mapa_shared(smem_u32(&ctl->dx_empty), 0);
+        const int myrow = kHalf * static_cast<int>(v) + 32 * q + lane;  // position within the (pair-)tile
         uint32_t dx_phase = 0;
-        TileIter it;
+        Iter it;
         it.first(off, E, lo, hi);
         int tok_next = it.valid(E) ? ((myrow < it.ntok()) ? perm[it.p0 + myrow] : -1) : -1;
         while (it.valid(E)) {
             const int tok_mine = tok_next;
-            TileIter nx = it;
+            Iter nx = it;
             nx.next(off, E, lo, hi);
             tok_next = nx.valid(E) ? ((myrow < nx.ntok()) ? perm[nx.p0 + myrow] : -1) : -1;
             if (!mbar_wait_cl(&ctl->dx_full, dx_phase, abort, dev_flags)) break;
             __syncwarp();
             tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < kHalf / 32; ++cc) {
+            for (int cc = 0; cc < kCols / 32; ++cc) {
                 float vals[32];
                 tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0 + cc * 32),
                                    vals);
@@ -418,7 +465,7 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(dx_empty0);
+            if (lane == 0) arrive_on_leader<PAIR>(&ctl->dx_empty);
             dx_phase ^= 1;
             it = nx;
         }
@@ -428,12 +475,11 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
         const int tdb = threadIdx.x - kDbWarp0 * 32;  // 0..127
         const int dq = warp & 3;
         const int g = tdb >> 5, jo = tdb & 31;
-        const uint32_t dw_empty0 = mapa_shared(smem_u32(&ctl->dw_empty), 0);
         int sw = 0;
         uint32_t pw = 0, dw_phase = 0;
         float db_run = 0.0f;
         bool ok = true;
-        TileIter it;
+        Iter it;
         it.first(off, E, lo, hi);
         while (ok && it.valid(E)) {
             const int ntc = (it.ntok() + 31) / 32;
@@ -473,7 +519,7 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
                 db_run = 0.0f;
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(dw_empty0);
+                if (lane == 0) arrive_on_leader<PAIR>(&ctl->dw_empty);
                 dw_phase ^= 1;
             }
             it.next(off, E, lo, hi);
@@ -481,12 +527,35 @@ bwd_fused_tf32_kernel(const float* __restrict__ x, const float* __restrict__ g_s
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();  // no CTA leaves while the peer may still arrive on its barriers
+    if (PAIR) cluster_sync_all();  // no CTA leaves while the peer may still arrive on its barriers
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc_pair(tmem, kTmemCols);
+        if (PAIR)
+            tmem_dealloc_pair(tmem, kTmemCols);
+        else
+            tmem_dealloc(tmem, kTmemCols);
     }
 }
+
+#define BWD_FUSED_ARGS                                                                                           \
+    const float* __restrict__ x, const float* __restrict__ g_src, const __grid_constant__ CUtensorMap tm_w,      \
+        const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int T, int E, int P, int g_div,   \
+        float out_scale, int acc_dx, float* __restrict__ d_x, float* __restrict__ part,                          \
+        float* __restrict__ part_db, uint32_t* __restrict__ dev_flags
+
+template <bool COLLAPSE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) bwd_fused_pair_kernel(BWD_FUSED_ARGS) {
+    bwd_fused_body<256, true, COLLAPSE>(x, g_src, &tm_w, offsets, perm, T, E, P, g_div, out_scale, acc_dx, d_x, part,
+                                        part_db, dev_flags);
+}
+
+template <bool COLLAPSE>
+__global__ void __launch_bounds__(kThreads, 1) bwd_fused_single_kernel(BWD_FUSED_ARGS) {
+    bwd_fused_body<128, false, COLLAPSE>(x, g_src, &tm_w, offsets, perm, T, E, P, g_div, out_scale, acc_dx, d_x, part,
+                                         part_db, dev_flags);
+}
+
+#undef BWD_FUSED_ARGS
 
 }  // namespace
 
@@ -504,39 +573,55 @@ cudaError_t bwd_fused_max_pairs(int* out) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, bwd_fused_tf32_kernel<false>, &cfg);
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, bwd_fused_pair_kernel<false>, &cfg);
     if (e != cudaSuccess) return e;
     *out = n < 1 ? 1 : (n > kFusedMaxPairs ? kFusedMaxPairs : n);
     return cudaSuccess;
 }
 
 int bwd_fused_pairs(int64_t T, int max_pairs) {
-    int64_t p = (T + 2 * kTileTok - 1) / (2 * kTileTok);
+    int64_t p = (T + 511) / 512;
     if (p < 1) p = 1;
     if (p > max_pairs) p = max_pairs;
     return static_cast<int>(p);
 }
 
 cudaError_t launch_bwd_fused_tf32(const float* x, const float* W, const float* g_src, const int32_t* offsets,
-                                  const int32_t* perm, int64_t T, int E, int P, int g_div, float out_scale, int acc_dx,
-                                  float* d_x, float* part, float* part_db, uint32_t* dev_flags, cudaStream_t s) {
+                                  const int32_t* perm, int64_t T, int E, int H, int P, int g_div, float out_scale,
+                                  int acc_dx, float* d_x, float* part, float* part_db, uint32_t* dev_flags,
+                                  cudaStream_t s) {
     CUtensorMap tm_w;
-    if (!make_map_2d(&tm_w, W, static_cast<uint64_t>(E) * kH, kH, 32, 32, kMapSw128Atom32)) return cudaErrorInvalidValue;
-    if (g_div != 1 || out_scale != 1.0f)
-        bwd_fused_tf32_kernel<true><<<2 * P, kThreads, kSmemBytes, s>>>(
-            x, g_src, tm_w, offsets, perm, static_cast<int>(T), E, P, g_div, out_scale, acc_dx, d_x, part, part_db,
-            dev_flags);
-    else
-        bwd_fused_tf32_kernel<false><<<2 * P, kThreads, kSmemBytes, s>>>(
-            x, g_src, tm_w, offsets, perm, static_cast<int>(T), E, P, 1, 1.0f, acc_dx, d_x, part, part_db, dev_flags);
+    if (!make_map_2d(&tm_w, W, static_cast<uint64_t>(E) * H, H, 32, 32, kMapSw128Atom32)) return cudaErrorInvalidValue;
+    const bool collapse = g_div != 1 || out_scale != 1.0f;
+    const int Ti = static_cast<int>(T);
+    if (H == 256) {
+        if (collapse)
+            bwd_fused_pair_kernel<true><<<2 * P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, g_div,
+                                                                          out_scale, acc_dx, d_x, part, part_db,
+                                                                          dev_flags);
+        else
+            bwd_fused_pair_kernel<false><<<2 * P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, 1,
+                                                                           1.0f, acc_dx, d_x, part, part_db, dev_flags);
+    } else {
+        if (collapse)
+            bwd_fused_single_kernel<true><<<P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, g_div,
+                                                                        out_scale, acc_dx, d_x, part, part_db,
+                                                                        dev_flags);
+        else
+            bwd_fused_single_kernel<false><<<P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, 1,
+                                                                         1.0f, acc_dx, d_x, part, part_db, dev_flags);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t bwd_fused_set_smem_limits() {
-    cudaError_t e = cudaFuncSetAttribute(bwd_fused_tf32_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(bwd_fused_tf32_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaSuccess;
+    const void* kernels[4] = {reinterpret_cast<const void*>(bwd_fused_pair_kernel<false>),
+                              reinterpret_cast<const void*>(bwd_fused_pair_kernel<true>),
+                              reinterpret_cast<const void*>(bwd_fused_single_kernel<false>),
+                              reinterpret_cast<const void*>(bwd_fused_single_kernel<true>)};
+    for (const void* k : kernels)
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     return e;
 }
 

@@ -120,14 +120,16 @@ cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const i
                                 int E, int H, int P, float scale, float* dW, float* db, int acc_dw, int acc_db,
                                 cudaStream_t s);
 
-// The fused TF32 backward at H = 256 (d_x, and dW / db partial sums into the
-// slots, in one pass over d_out and x) on P pairs of CTAs; range c of expert e
-// gives slot c + e. Token t's gradient row is g_src[t / g_div]; d_x is scaled by
-// out_scale (the slot reduction applies it to dW and db).
+// The fused TF32 backward (d_x, and dW / db partial sums into the slots, in one
+// pass over d_out and x): H = 256 on P pairs of CTAs, H = 128 on P single CTAs;
+// range c of expert e gives slot c + e. Token t's gradient row is
+// g_src[t / g_div]; d_x is scaled by out_scale (the slot reduction applies it to
+// dW and db).
 constexpr int kFusedMaxPairs = 74;
 cudaError_t launch_bwd_fused_tf32(const float* x, const float* W, const float* g_src, const int32_t* offsets,
-                                  const int32_t* perm, int64_t T, int E, int P, int g_div, float out_scale, int acc_dx,
-                                  float* d_x, float* part, float* part_db, uint32_t* dev_flags, cudaStream_t s);
+                                  const int32_t* perm, int64_t T, int E, int H, int P, int g_div, float out_scale,
+                                  int acc_dx, float* d_x, float* part, float* part_db, uint32_t* dev_flags,
+                                  cudaStream_t s);
 // Pairs that run at once on the current device (at most kFusedMaxPairs).
 cudaError_t bwd_fused_max_pairs(int* out);
 // Pairs used for T tokens: one per 512 tokens, at most max_pairs (<= wgrad_splits(T),

@@ -120,6 +120,13 @@ FWD_SPECS = [
     wl.make_spec("mcf_b300_h32_e32_h128", 300, 32, 32, 128, 55),        # N_H and E at their maximum
     wl.make_spec("mcf_b257_h7_e4_h128", 257, 7, 4, 128, 56, skew_expert=2, skew_value=3.0),  # > 2 tokens per (b, e)
     wl.make_spec("mcf_b130_h5_e4_h128", 130, 5, 4, 128, 57, logits="binary"),               # frequent ties
+    # the row-range split of the staged kernel (E <= 8): fewer rows than SMs, ranges
+    # of several tiles with a partial last one, the largest horizon (raw stages of
+    # 8 x 32 tokens), one expert
+    wl.make_spec("mcf_b100_h16_e8_h256", 100, 16, 8, 256, 62),
+    wl.make_spec("mcf_b40000_h5_e8_h128", 40000, 5, 8, 128, 63),
+    wl.make_spec("mcf_b3000_h32_e8_h256", 3000, 32, 8, 256, 64),
+    wl.make_spec("mcf_b500_h7_e1_h256", 500, 7, 1, 256, 65),
 ]
 
 
@@ -209,6 +216,28 @@ def test_fwd_mean_collapse_check_catches_one_token_on_the_wrong_expert(math_mode
     n_bad = fwd_outside(bad, want, math_mode)
     assert n_bad > spec.H // 2, n_bad   # row 5 is off almost everywhere
     assert fwd_outside(np.delete(bad, 5, axis=0), np.delete(want, 5, axis=0), math_mode) == 0  # other rows intact
+
+
+@pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
+@pytest.mark.parametrize("E", [5, 12])
+def test_fwd_mean_collapse_ignores_expert_indices_out_of_range(math_mode, E):
+    """The call reads only expert_idx; an index outside [0, E) contributes nothing
+    (neither its W x nor a bias), as the oracle's reading of such a token."""
+    spec = wl.make_spec(f"mcf_badidx_b300_h6_e{E}_h128", 300, 6, E, 128, 66)
+    inp = wl.generate(spec)
+    idx = oracle.route(inp.gate_logits)[0].copy()
+    idx[::7] = E
+    idx[3::11] = -1
+    r = ops.Routing.empty(spec.T, E, "cuda")
+    r.expert_idx.copy_(dev(idx))
+    out = Guarded(spec.B * spec.H, shape=(spec.B, spec.H))
+    ws = ops.new_workspace(spec.T, E, spec.H, "cuda")
+    ops.moe_top1_fwd_mean_collapse(dev(inp.x), dev(inp.W), dev(inp.bias), r, spec.B, spec.N_H, E, spec.H, math_mode,
+                                   out.t, ws)
+    torch.cuda.synchronize()
+    assert ops.moe_top1_device_flags(ws) == 0 and out.guards_intact()
+    want = oracle.fwd_mean_collapse_presum(inp.x, inp.W, inp.bias, idx, spec.N_H, tf32_mode(math_mode))
+    assert_close("ctx_mean", out.host(), want, *TOL[math_mode])
 
 
 @pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)

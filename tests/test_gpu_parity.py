@@ -164,13 +164,17 @@ def test_straight_through_expert_path_gives_the_logits_no_gradient(math_mode):
     assert not np.array_equal(aux_grad(logits * 2.0, r2).cpu().numpy(), before)
 
 
-# The TF32 backward at H = 256 with d_x and dW / db requested runs as one fused
-# kernel on CTA pairs (256-token pair-tiles of one expert, 512 tokens per pair at
-# least). Shapes that stress its tiling: a pair-tile the odd CTA has no token of,
-# one it has a few of, one pair only, segments far shorter than a pair-tile
-# (32 experts), a range that crosses several expert boundaries at odd positions,
-# and more pairs than fit on the GPU at once.
+# The TF32 backward with d_x and dW / db requested runs as one fused kernel: on
+# CTA pairs at H = 256 (256-token pair-tiles of one expert, 512 tokens per pair at
+# least), on single CTAs at H = 128 (128-token tiles). Shapes that stress the
+# tiling: a pair-tile the odd CTA has no token of, one it has a few of, one pair
+# only, segments far shorter than a tile (32 experts), a range that crosses
+# several expert boundaries at odd positions, more pairs than fit on the GPU at
+# once; and the same kinds of shapes at H = 128.
 FUSED_SHAPES = [
+    wl.make_spec("fused_b90_e3_h128", 90, 1, 3, 128, 91),
+    wl.make_spec("fused_b1000_h3_e32_h128", 1000, 3, 32, 128, 92, skew_expert=2, skew_value=1.0),
+    wl.make_spec("fused_b30000_h3_e5_h128", 30000, 3, 5, 128, 93),
     wl.make_spec("fused_b100_e3_h256", 100, 1, 3, 256, 81),
     wl.make_spec("fused_b300_e1_h256", 300, 1, 1, 256, 82),
     wl.make_spec("fused_b333_h3_e2_h256", 333, 3, 2, 256, 83),
