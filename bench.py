@@ -243,15 +243,20 @@ def cpu_oracle_tokens_per_s(inp, n_tokens: int):
     return sample.spec.T / dt, dt, sample.spec.T
 
 
-def _oracle_shard(args):
+def _oracle_shard(shard):
     """One worker of the all-cores CPU baseline: the oracle, unchanged, on one
     token shard; returns its dW and db (the sums the shards share)."""
-    inp, lo, hi = args
     import oracle
-    shard = wl.token_sample(wl.dataclasses.replace(inp, gate_logits=inp.gate_logits[lo:hi], x=inp.x[lo:hi],
-                                                   d_out=inp.d_out[lo:hi]), hi - lo)
     out = oracle.step(shard)
     return out["dW"], out["db"]
+
+
+def _shard(inp, lo: int, hi: int):
+    """Tokens lo .. hi - 1 of a workload as a workload of their own (only these
+    rows travel to a worker process)."""
+    spec = wl.dataclasses.replace(inp.spec, name=inp.spec.name + f"_{lo}_{hi}", B=hi - lo, N_H=1)
+    return wl.dataclasses.replace(inp, spec=spec, gate_logits=inp.gate_logits[lo:hi], x=inp.x[lo:hi],
+                                  d_out=inp.d_out[lo:hi])
 
 
 def cpu_oracle_all_cores(inp, tokens_per_core: int, cores: int):
@@ -260,12 +265,11 @@ def cpu_oracle_all_cores(inp, tokens_per_core: int, cores: int):
     shards added in shard order. Returns (tokens/s, seconds, tokens)."""
     import multiprocessing as mp
     n = min(inp.spec.T, tokens_per_core * cores)
-    bounds = [(n * k // cores, n * (k + 1) // cores) for k in range(cores)]
-    small = wl.token_sample(inp, n)
+    shards = [_shard(inp, n * k // cores, n * (k + 1) // cores) for k in range(cores)]
     with mp.get_context("spawn").Pool(cores) as pool:
-        pool.map(_oracle_shard, [(wl.token_sample(small, 64), 0, 64)] * cores)  # start-up and oracle build
+        pool.map(_oracle_shard, [_shard(inp, 0, 64)] * cores)  # start-up and the oracle's build
         t0 = time.perf_counter()
-        parts = pool.map(_oracle_shard, [(small, lo, hi) for lo, hi in bounds])
+        parts = pool.map(_oracle_shard, shards, chunksize=1)
         dW, db = parts[0]
         for pw, pb in parts[1:]:
             dW = dW + pw

@@ -34,7 +34,8 @@
 // HBM once: the second read, by the same or the peer CTA, hits L2.
 //
 // Warp roles (each CTA): 0-7 drain the d_x accumulator (TMEM -> transpose in
-// shared memory -> token rows); 8-11 gather token rows with cp.async; 12: the
+// shared memory -> token rows); 8-9 gather the X stages' rows and 10-11 the W
+// stages' rows with cp.async, each pair of warps running ahead on its own; 12: the
 // MMA issuer (even CTA) or the relay (odd CTA: once its stage has landed, it
 // makes it visible to the tensor core and arrives on the even CTA's barrier);
 // 13 loads the W[e] slab by TMA; 14-17 sum d_out over the staged tokens for db
@@ -71,12 +72,12 @@ constexpr int kGroupBytes = 4096;   // MN-major: 32 rows x 128 bytes per 32-wide
 constexpr int kStgBytes = kEpiWarps * 32 * 128;
 
 struct __align__(8) Ctl {
-    uint64_t xfull[kXStages];   // even CTA: its 128 gather threads + the odd CTA's relay
-    uint64_t xready[kXStages];  // odd CTA: its 128 gather threads
+    uint64_t xfull[kXStages];   // even CTA: its 64 X gather threads + the odd CTA's relay
+    uint64_t xready[kXStages];  // odd CTA: its 64 X gather threads
     uint64_t xtma[kXStages];    // each CTA: its own W-slab TMA (arrival + bytes)
     uint64_t xempty[kXStages];  // each CTA: the pair's MMA commit
-    uint64_t wfull[kWStages];   // even CTA: 128 gather threads + relay
-    uint64_t wready[kWStages];  // odd CTA: 128 gather threads
+    uint64_t wfull[kWStages];   // even CTA: its 64 W gather threads + relay
+    uint64_t wready[kWStages];  // odd CTA: its 64 W gather threads
     uint64_t wempty[kWStages];  // each CTA: MMA commit + its 4 db warps
     uint64_t dx_full;           // each CTA: MMA commit
     uint64_t dx_empty;          // even CTA: the 8 d_x drain warps of both CTAs
@@ -166,14 +167,14 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kXStages; ++s) {
-            mbar_init(&ctl->xfull[s], 128 + (PAIR ? 1 : 0));
-            mbar_init(&ctl->xready[s], 128);
+            mbar_init(&ctl->xfull[s], 64 + (PAIR ? 1 : 0));
+            mbar_init(&ctl->xready[s], 64);
             mbar_init(&ctl->xtma[s], 1);
             mbar_init(&ctl->xempty[s], 1);
         }
         for (int s = 0; s < kWStages; ++s) {
-            mbar_init(&ctl->wfull[s], 128 + (PAIR ? 1 : 0));
-            mbar_init(&ctl->wready[s], 128);
+            mbar_init(&ctl->wfull[s], 64 + (PAIR ? 1 : 0));
+            mbar_init(&ctl->wready[s], 64);
             mbar_init(&ctl->wempty[s], 1 + 4);
         }
         mbar_init(&ctl->dx_full, 1);
@@ -206,44 +207,60 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
     const int lo = static_cast<int>(split_lo(c, T, P)), hi = static_cast<int>(split_lo(c + 1, T, P));
     const int* off = ctl->off;
 
-    if (warp >= kProducer0 / 32 && warp < kProducer0 / 32 + 4) {
-        // ---------------- producers: cp.async gathers of the stages' token rows
-        const int ptid = threadIdx.x - kProducer0;  // 0..127
-        const int prow = ptid >> 3, pg = ptid & 7;  // X stages: row within a 16-row block, 16-byte granule
-        const int q16 = ptid & 7, gq = (ptid >> 3) & 3, rsub = ptid >> 5;  // W stages
-        int sx = 0, sw = 0;
-        uint32_t px = 0, pw = 0;
+    if (warp >= kProducer0 / 32 && warp < kProducer0 / 32 + 2) {
+        // ---------------- X-stage producers (warps 8-9): A = the d_out rows of this
+        // CTA's 128 tokens, 32 o per stage, K-major (128-byte swizzle). They run
+        // ahead of the W-stage producers independently, so that both rings stay
+        // full while the d_x accumulator is being drained.
+        const int ptid = threadIdx.x - kProducer0;  // 0..63
+        const int prow = ptid >> 3, pg = ptid & 7;  // row within an 8-row block, 16-byte granule
+        int sx = 0;
+        uint32_t px = 0;
         bool ok = true;
         Iter it;
         it.first(off, E, lo, hi);
         while (ok && it.valid(E)) {
             const int n = it.ntok();
-            // this CTA's tokens for the X stages (rows r = j * 16 + prow) and the
-            // pair-tile's tokens for the W stages (lane l: token 32 tc + l)
-            int tx[8], tw[8];
+            int tx[16];  // the token of rows r = j * 8 + prow
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = kHalf * static_cast<int>(v) + j * 16 + prow;
+            for (int j = 0; j < 16; ++j) {
+                const int r = kHalf * static_cast<int>(v) + j * 8 + prow;
                 tx[j] = (r < n) ? perm[it.p0 + r] : -1;
-                const int q = j * 32 + lane;
-                tw[j] = (q < n) ? perm[it.p0 + q] : -1;
+                if (COLLAPSE && tx[j] >= 0) tx[j] = tx[j] / g_div;  // the token's gradient row
             }
-            // X stages: A = d_out rows of this CTA's tokens, 32 o per stage, K-major
             for (int kc = 0; kc < kH / 32 && ok; ++kc) {
                 if (!(ok = mbar_wait(&ctl->xempty[sx], px ^ 1, abort, dev_flags))) break;
                 const uint32_t a_u32 = smem_u32(xring + sx * kStageBytes);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = j * 16 + prow;
-                    const int tk = tx[j];
-                    const int gr = (COLLAPSE && tk >= 0) ? tk / g_div : tk;
+                for (int j = 0; j < 16; ++j) {
+                    const int r = j * 8 + prow;
+                    const int gr = tx[j];
                     const float* src = g_src + static_cast<int64_t>(gr < 0 ? 0 : gr) * kH + kc * 32 + pg * 4;
-                    cp_async_16_l2_256(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), src, tk < 0 ? 0u : 16u);
+                    cp_async_16_l2_256(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), src, gr < 0 ? 0u : 16u);
                 }
                 cp_async_arrive_noinc(leader ? &ctl->xfull[sx] : &ctl->xready[sx]);
                 advance(sx, px, kXStages);
             }
-            // W stages: 32 tokens each; A = d_out[., o-half v], B = x[., i-half v], MN-major
+            it.next(off, E, lo, hi);
+        }
+    } else if (warp >= kProducer0 / 32 + 2 && warp < kProducer0 / 32 + 4) {
+        // ---------------- W-stage producers (warps 10-11): 32 tokens per stage; A =
+        // d_out[., o-half v], B = x[., i-half v], MN-major (32-byte granules)
+        const int ptid = threadIdx.x - kProducer0 - 64;  // 0..63
+        const int q16 = ptid & 7, gq = (ptid >> 3) & 3, rsub = ptid >> 5;
+        int sw = 0;
+        uint32_t pw = 0;
+        bool ok = true;
+        Iter it;
+        it.first(off, E, lo, hi);
+        while (ok && it.valid(E)) {
+            const int n = it.ntok();
+            int tw[8];  // lane l: the token at position 32 tc + l of the tile
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int q = j * 32 + lane;
+                tw[j] = (q < n) ? perm[it.p0 + q] : -1;
+            }
             const int ntc = (n + 31) / 32;
             for (int tc = 0; tc < ntc && ok; ++tc) {
                 if (!(ok = mbar_wait(&ctl->wempty[sw], pw ^ 1, abort, dev_flags))) break;
@@ -253,13 +270,13 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                 for (int j = 1; j < 8; ++j)
                     if (j == tc) tok_l = tw[j];
                 const int gtok_l = (COLLAPSE && tok_l >= 0) ? tok_l / g_div : tok_l;
+                const int64_t col = kHalf * static_cast<int64_t>(v) + gq * 32 + q16 * 4;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = j * 4 + rsub;
+                for (int j = 0; j < 16; ++j) {
+                    const int r = j * 2 + rsub;
                     const int tk = __shfl_sync(0xffffffffu, tok_l, r);
                     const int gtk = __shfl_sync(0xffffffffu, gtok_l, r);
                     const uint32_t o = gq * kGroupBytes + r * 128 + ((((q16 >> 1) ^ (r & 3)) << 5) | ((q16 & 1) << 4));
-                    const int64_t col = kHalf * static_cast<int64_t>(v) + gq * 32 + q16 * 4;
                     const uint32_t nb = tk < 0 ? 0u : 16u;
                     cp_async_16(a_u32 + o, g_src + static_cast<int64_t>(tk < 0 ? 0 : gtk) * kH + col, nb);
                     cp_async_16(a_u32 + kRegion + o, x + static_cast<int64_t>(tk < 0 ? 0 : tk) * kH + col, nb);
