@@ -325,22 +325,25 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, abort, dev_flags)) break;
             __syncwarp();
             tc_fence_after();
+            // 32-column chunks, double-buffered: the TMEM load of chunk c + 1 is in
+            // flight while chunk c is transposed and stored
+            constexpr int NCH = HALF / 32;
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * H + c0);
+            uint32_t buf[2][32];
+            tmem_ld_32x32b_x32_async(tbase, buf[0]);
+            tmem_ld_wait_tied(buf[0]);
 #pragma unroll
-            for (int cc = 0; cc < HALF / 64; ++cc) {
-                float v[64];
-                tmem_ld_32x32b_x64(tmem + (static_cast<uint32_t>(32 * q) << 16) +
-                                       static_cast<uint32_t>(acc * H + c0 + cc * 64), v);
-                if (COLLAPSE) {
+            for (int c = 0; c < NCH; ++c) {
+                if (c + 1 < NCH) tmem_ld_32x32b_x32_async(tbase + static_cast<uint32_t>((c + 1) * 32), buf[(c + 1) & 1]);
+                float v[32];
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) v[i] *= out_scale;
-                }
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int c = cc * 2 + h;  // 32-column chunk within the half
+                for (int i = 0; i < 32; ++i) v[i] = COLLAPSE ? __uint_as_float(buf[c & 1][i]) * out_scale
+                                                             : __uint_as_float(buf[c & 1][i]);
+                {
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj)
-                        st_shared_v4(my_u32 + 4 * (lane * 32 + ((jj ^ (lane & 7)) * 4)), v[32 * h + 4 * jj],
-                                     v[32 * h + 4 * jj + 1], v[32 * h + 4 * jj + 2], v[32 * h + 4 * jj + 3]);
+                        st_shared_v4(my_u32 + 4 * (lane * 32 + ((jj ^ (lane & 7)) * 4)), v[4 * jj], v[4 * jj + 1],
+                                     v[4 * jj + 2], v[4 * jj + 3]);
                     __syncwarp();
                     if (accumulate) {
 #pragma unroll
@@ -377,6 +380,7 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
                     }
                     __syncwarp();
                 }
+                if (c + 1 < NCH) tmem_ld_wait_tied(buf[(c + 1) & 1]);
             }
             tc_fence_before();
             __syncwarp();

@@ -445,15 +445,21 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
             if (!mbar_wait_cl(&ctl->dx_full, dx_phase, abort, dev_flags)) break;
             __syncwarp();
             tc_fence_after();
-#pragma unroll 1
-            for (int cc = 0; cc < kCols / 32; ++cc) {
-                float vals[32];
-                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0 + cc * 32),
-                                   vals);
-                if (COLLAPSE) {
+            // 32-column chunks, double-buffered: the TMEM load of chunk cc + 1 is in
+            // flight while chunk cc is transposed and stored
+            constexpr int NCH = kCols / 32;
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0);
+            uint32_t buf[2][32];
+            tmem_ld_32x32b_x32_async(tbase, buf[0]);
+            tmem_ld_wait_tied(buf[0]);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) vals[i] *= out_scale;
-                }
+            for (int cc = 0; cc < NCH; ++cc) {
+                if (cc + 1 < NCH)
+                    tmem_ld_32x32b_x32_async(tbase + static_cast<uint32_t>((cc + 1) * 32), buf[(cc + 1) & 1]);
+                float vals[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) vals[i] = COLLAPSE ? __uint_as_float(buf[cc & 1][i]) * out_scale
+                                                                : __uint_as_float(buf[cc & 1][i]);
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj)
                     st_shared_v4(my_u32 + 4 * (lane * 32 + ((jj ^ (lane & 7)) * 4)), vals[4 * jj], vals[4 * jj + 1],
@@ -479,6 +485,7 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                     }
                 }
                 __syncwarp();
+                if (cc + 1 < NCH) tmem_ld_wait_tied(buf[(cc + 1) & 1]);
             }
             tc_fence_before();
             __syncwarp();
