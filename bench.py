@@ -199,6 +199,10 @@ class ClockSampler:
 
     def __enter__(self):
         if self.nvml is not None:
+            # the launching thread holds the interpreter lock between its library
+            # calls; a short switch interval lets the sampler wake on time
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(2e-4)
             self._thr = threading.Thread(target=self._run, daemon=True)
             self._thr.start()
         return self
@@ -207,6 +211,7 @@ class ClockSampler:
         self._stop.set()
         if self._thr:
             self._thr.join()
+            sys.setswitchinterval(self._switch)
 
     def summary(self):
         if not self.samples:

@@ -58,7 +58,7 @@ def _rank_exchange(rank, port, out):
 
 @pytest.mark.timeout(120)
 def test_exchange_gives_every_rank_the_full_batch_results():
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_exchange, args=(_free_port(), out), nprocs=WORLD, join=True)
     inp = wl.generate(SPEC)
     E, H, T = SPEC.E, SPEC.H, SPEC.T
@@ -99,7 +99,7 @@ def _rank_unequal(rank, port, out):
 
 @pytest.mark.timeout(120)
 def test_unequal_shards_are_rejected_on_every_rank():
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_unequal, args=(_free_port(), out), nprocs=WORLD, join=True)
     assert "differ in size" in out[0] and "differ in size" in out[1]
 

@@ -66,7 +66,8 @@ def _corrupt(kind):
     elif kind == "expert index out of range":
         idx[perm[offsets[5]]] = E
     elif kind == "routing of another batch":
-        (idx, counts, offsets, perm), _, _ = _good(seed=4)
+        # this batch's expert indices with another batch's counts, offsets and perm
+        (_, counts, offsets, perm), _, _ = _good(seed=4)
     else:
         raise ValueError(kind)
     return idx, counts, offsets, perm, T, E

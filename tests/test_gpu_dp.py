@@ -107,7 +107,8 @@ def _rank_gate(rank, port, out):
 
 @pytest.mark.timeout(600)
 def test_two_ranks_on_the_gpu_hold_the_full_batch_gradients_of_the_oracle():
-    out = mp.Manager().dict()
+    # every helper process is spawned: this process already holds a CUDA context
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_gate, args=(_free_port(), out), nprocs=DP_WORLD, join=True)
     s = DP_SPEC
     inp = wl.generate(s)

@@ -31,7 +31,7 @@ def _rank(rank, world, port, out):
 
 def test_max_over_two_gloo_ranks():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank, args=(world, _free_port(), out), nprocs=world, join=True)
     assert dict(out) == {0: 2.25, 1: 2.25}
 
@@ -61,7 +61,7 @@ def test_a_replica_that_leaves_between_steps_ends_the_next_timing_with_an_error(
     """A rank that drops out between steps must not hang the others: the next
     max-over-ranks reduction raises (peer closed or the short group timeout)."""
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_leaves, args=(world, _free_port(), out), nprocs=world, join=True)
     assert out[(0, 0)] == 2.0 and out[(1, 0)] == 2.0
     assert out[(0, 1)] == "error"
