@@ -536,17 +536,22 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
             if (lane < 16) {
                 const int m = rw * 16 + lane;
                 uint16_t* ord = order + m * kHMaxHorizon;
-                int cnt[kSMaxE + 1];
-#pragma unroll
-                for (int e = 0; e <= kSMaxE; ++e) cnt[e] = 0;
                 const bool valid = m < nrows;
                 const int32_t* idx = expert_idx + (b0 + m) * N_H;
-                for (int h = 0; h < N_H; ++h) {
-                    const int e = valid ? idx[h] : -1;
-                    const int k = (e >= 0 && e < E) ? e : kSMaxE;
+                // all of the row's expert indices are requested before the first is used
+                int ek[kHMaxHorizon];  // expert of horizon token h, kSMaxE for none / out of range
 #pragma unroll
-                    for (int f = 0; f <= kSMaxE; ++f) cnt[f] += (f == k) ? 1 : 0;
+                for (int h = 0; h < kHMaxHorizon; ++h) {
+                    const int e = (valid && h < N_H) ? idx[h] : -1;
+                    ek[h] = (e >= 0 && e < E) ? e : kSMaxE;
                 }
+                int cnt[kSMaxE + 1];
+#pragma unroll
+                for (int f = 0; f <= kSMaxE; ++f) cnt[f] = 0;
+#pragma unroll
+                for (int h = 0; h < kHMaxHorizon; ++h)
+#pragma unroll
+                    for (int f = 0; f <= kSMaxE; ++f) cnt[f] += (h < N_H && f == ek[h]) ? 1 : 0;
                 int pos[kSMaxE + 1];
                 int acc = 0;
 #pragma unroll
@@ -554,14 +559,14 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
                     pos[f] = acc;
                     acc += cnt[f];
                 }
-                for (int h = 0; h < N_H; ++h) {
-                    const int e = valid ? idx[h] : -1;
-                    const int k = (e >= 0 && e < E) ? e : kSMaxE;
+#pragma unroll
+                for (int h = 0; h < kHMaxHorizon; ++h) {
+                    if (h >= N_H) break;
                     int p = 0;
 #pragma unroll
                     for (int f = 0; f <= kSMaxE; ++f)
-                        if (f == k) p = pos[f]++;
-                    ord[p] = static_cast<uint16_t>(h | ((k == kSMaxE ? 0xFF : k) << 8));
+                        if (f == ek[h]) p = pos[f]++;
+                    ord[p] = static_cast<uint16_t>(h | ((ek[h] == kSMaxE ? 0xFF : ek[h]) << 8));
                 }
             }
             __syncwarp();
@@ -673,12 +678,14 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
             int cnt[kSMaxE];
 #pragma unroll
             for (int e = 0; e < kSMaxE; ++e) cnt[e] = 0;
-            if (valid) {
-                for (int h = 0; h < N_H; ++h) {
-                    const int e = expert_idx[b * N_H + h];
+            {
+                int ev[kHMaxHorizon];  // requested together, then counted
 #pragma unroll
-                    for (int f = 0; f < kSMaxE; ++f) cnt[f] += (f == e) ? 1 : 0;
-                }
+                for (int h = 0; h < kHMaxHorizon; ++h) ev[h] = (valid && h < N_H) ? expert_idx[b * N_H + h] : -1;
+#pragma unroll
+                for (int h = 0; h < kHMaxHorizon; ++h)
+#pragma unroll
+                    for (int f = 0; f < kSMaxE; ++f) cnt[f] += (f == ev[h]) ? 1 : 0;
             }
             const bool ok = mbar_wait(&ctl->t_full[acc], acc_phase, abort, dev_flags);
             if (!__all_sync(0xffffffffu, ok)) break;
