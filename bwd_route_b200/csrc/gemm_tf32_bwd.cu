@@ -219,8 +219,31 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
         bool ok = true;
         Iter it;
         it.first(off, E, lo, hi);
+        // The rows of this CTA's tokens of tile `t` go to L2 ahead of their gathers:
+        // thread (prow, pg) takes rows j * 8 + prow for j = pg and pg + 8, the whole
+        // 1 KiB x row and d_out row of each (the [B, H] gradient of the horizon mean
+        // is small and stays in L2 by itself). Each CTA fetches its own tokens; the
+        // W stages of both CTAs read those rows.
+        auto prefetch_tile = [&](const Iter& t) {
+            const int n = t.ntok();
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int r = kHalf * static_cast<int>(v) + (pg + 8 * jj) * 8 + prow;
+                if (r < n) {
+                    const int tk = perm[t.p0 + r];
+                    prefetch_bulk_l2(x + static_cast<int64_t>(tk) * kH, kH * 4);
+                    if (!COLLAPSE) prefetch_bulk_l2(g_src + static_cast<int64_t>(tk) * kH, kH * 4);
+                }
+            }
+        };
+        if (it.valid(E)) prefetch_tile(it);
         while (ok && it.valid(E)) {
             const int n = it.ntok();
+            {
+                Iter nx = it;
+                nx.next(off, E, lo, hi);
+                if (nx.valid(E)) prefetch_tile(nx);
+            }
             int tx[16];  // the token of rows r = j * 8 + prow
 #pragma unroll
             for (int j = 0; j < 16; ++j) {

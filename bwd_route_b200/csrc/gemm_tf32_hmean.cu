@@ -590,21 +590,35 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
                         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                         int cur = -1;
                         uint32_t present = 0;
-                        for (int j = 0; j < N_H; ++j) {
-                            const uint32_t o = ord[j];
-                            const int e = static_cast<int>(o >> 8);
-                            if (e >= E) break;  // out-of-range experts sort last and add nothing
-                            const float4 v = ld_shared_v4(rb + (o & 0xFFu) * 64);
-                            if (e != cur) {
-                                if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
-                                acc = v;
-                                cur = e;
-                                present |= 1u << e;
-                            } else {
-                                acc.x += v.x;
-                                acc.y += v.y;
-                                acc.z += v.z;
-                                acc.w += v.w;
+                        // eight tokens at a time: their list entries (one 16-byte load) and
+                        // their rows are requested together, then added in list order
+                        for (int j0 = 0; j0 < N_H; j0 += 8) {
+                            const uint4 o4 = *reinterpret_cast<const uint4*>(ord + j0);
+                            uint32_t o[8] = {o4.x & 0xFFFFu, o4.x >> 16, o4.y & 0xFFFFu, o4.y >> 16,
+                                             o4.z & 0xFFFFu, o4.z >> 16, o4.w & 0xFFFFu, o4.w >> 16};
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                if (j0 + u >= N_H) o[u] = 0xFF00u;  // past the row's tokens: no expert
+                            float4 vv[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                vv[u] = (static_cast<int>(o[u] >> 8) < E) ? ld_shared_v4(rb + (o[u] & 0xFFu) * 64)
+                                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int e = static_cast<int>(o[u] >> 8);
+                                if (e >= E) continue;  // out-of-range experts sort last and add nothing
+                                if (e != cur) {
+                                    if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
+                                    acc = vv[u];
+                                    cur = e;
+                                    present |= 1u << e;
+                                } else {
+                                    acc.x += vv[u].x;
+                                    acc.y += vv[u].y;
+                                    acc.z += vv[u].z;
+                                    acc.w += vv[u].w;
+                                }
                             }
                         }
                         if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
