@@ -104,12 +104,6 @@ __device__ __forceinline__ void cp_async_16_l2_256(uint32_t dst, const void* src
     asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                  : "memory");
 }
-// Brings `bytes` (a multiple of 16) at the 16-byte-aligned global address p into
-// L2 (no data is returned): one bulk prefetch per token row, issued a tile ahead,
-// turns the later gathers of that row into L2 hits.
-__device__ __forceinline__ void prefetch_bulk_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 // Waits until every cp.async this thread issued has landed in shared memory.
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");

@@ -197,17 +197,7 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
         uint32_t pa = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-            if (tile + static_cast<int>(gridDim.x) < ntiles) {
-                load_tokens(tile + gridDim.x, nxt);
-                // the next tile's whole rows go to L2 now (one bulk prefetch per row,
-                // thread (prow, pg) taking row it * 16 + prow for it = pg), so that its
-                // gathers are L2 hits
-                int t = -1;
-#pragma unroll
-                for (int it = 0; it < 8; ++it)
-                    if (it == pg) t = nxt[it];
-                if (!COLLAPSE && t >= 0) prefetch_bulk_l2(src + static_cast<int64_t>(t) * H, H * 4);
-            }
+            if (tile + static_cast<int>(gridDim.x) < ntiles) load_tokens(tile + gridDim.x, nxt);
             for (int kc = 0; kc < C::KCH; ++kc) {
                 if (!(ok = mbar_wait(&ctl->aempty[sa], pa ^ 1, abort, dev_flags))) break;
                 const uint32_t a_u32 = smem_u32(aring + sa * C::A_BYTES);

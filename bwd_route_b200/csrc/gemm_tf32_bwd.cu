@@ -64,32 +64,31 @@ constexpr int kProducer0 = 256;  // warps 8-11
 constexpr int kMmaWarp = 12;
 constexpr int kWLoadWarp = 13;
 constexpr int kDbWarp0 = 14;     // warps 14-17
-constexpr int kXStages = 3;
-constexpr int kWStages = 3;
+// One ring of stages, filled and consumed in the MMA's order: each tile's X
+// stages (d_x: 32 o each), then its W stages (dW: 32 tokens each). A single
+// ring keeps all of its slots loading whichever kind of stage comes next.
+constexpr int kStages = 6;
 constexpr int kStageBytes = 32768;  // region 0 (A) and region 1 (B), 16 KiB each
 constexpr int kRegion = 16384;
 constexpr int kGroupBytes = 4096;   // MN-major: 32 rows x 128 bytes per 32-wide column group
 constexpr int kStgBytes = kEpiWarps * 32 * 128;
 
 struct __align__(8) Ctl {
-    uint64_t xfull[kXStages];   // even CTA: its 64 X gather threads + the odd CTA's relay
-    uint64_t xready[kXStages];  // odd CTA: its 64 X gather threads
-    uint64_t xtma[kXStages];    // each CTA: its own W-slab TMA (arrival + bytes)
-    uint64_t xempty[kXStages];  // each CTA: the pair's MMA commit
-    uint64_t wfull[kWStages];   // even CTA: its 64 W gather threads + relay
-    uint64_t wready[kWStages];  // odd CTA: its 64 W gather threads
-    uint64_t wempty[kWStages];  // each CTA: MMA commit + its 4 db warps
-    uint64_t dx_full;           // each CTA: MMA commit
-    uint64_t dx_empty;          // even CTA: the 8 d_x drain warps of both CTAs
-    uint64_t dw_full;           // each CTA: MMA commit
-    uint64_t dw_empty;          // even CTA: the 4 db / dW warps of both CTAs
-    uint64_t done;              // even CTA: the last commit
+    uint64_t full[kStages];   // even CTA: the 64 threads that gather the stage + the odd CTA's relay
+    uint64_t ready[kStages];  // odd CTA: the 64 threads that gather the stage
+    uint64_t tma[kStages];    // each CTA: its own W-slab TMA of an X stage (arrival + bytes)
+    uint64_t empty[kStages];  // each CTA: the pair's MMA commit + its 4 db warps
+    uint64_t dx_full;         // each CTA: MMA commit
+    uint64_t dx_empty;        // even CTA: the 8 d_x drain warps of both CTAs
+    uint64_t dw_full;         // each CTA: MMA commit
+    uint64_t dw_empty;        // even CTA: the 4 db / dW warps of both CTAs
+    uint64_t done;            // even CTA: the last commit
     uint32_t tmem_base;
     int abort;
     int off[33];
 };
 
-constexpr int kSmemBytes = 1024 + (kXStages + kWStages) * kStageBytes + kStgBytes + static_cast<int>(sizeof(Ctl));
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kStgBytes + static_cast<int>(sizeof(Ctl));
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 // The tiles of range [lo, hi) of the sorted token list, in order: expert e's
@@ -123,12 +122,9 @@ struct TileIter {
     __device__ bool last_in_run() const { return p0 + TILE >= t; }
 };
 
-__device__ __forceinline__ void advance(int& stage, uint32_t& phase, int n) {
-    if (++stage == n) {
-        stage = 0;
-        phase ^= 1;
-    }
-}
+// Ring slot and phase parity of the k-th stage of the launch.
+__device__ __forceinline__ int slot_of(int k) { return k % kStages; }
+__device__ __forceinline__ uint32_t parity_of(int k) { return static_cast<uint32_t>((k / kStages) & 1); }
 
 // One arrival on the even CTA's barrier `bar` (PAIR), or on this CTA's.
 template <bool PAIR>
@@ -156,26 +152,21 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
     using Iter = TileIter<kTileTok>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* xring = smem;
-    uint8_t* wring = smem + kXStages * kStageBytes;
-    float* stg = reinterpret_cast<float*>(smem + (kXStages + kWStages) * kStageBytes);
-    Ctl* ctl = reinterpret_cast<Ctl*>(smem + (kXStages + kWStages) * kStageBytes + kStgBytes);
+    uint8_t* ring = smem;
+    float* stg = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes + kStgBytes);
+    constexpr int nX = kH / 32;  // X stages per tile
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t v = PAIR ? cluster_ctarank() : 0u;  // 0: the even CTA, which issues the MMAs
     const bool leader = (v == 0);
     const int c = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kXStages; ++s) {
-            mbar_init(&ctl->xfull[s], 64 + (PAIR ? 1 : 0));
-            mbar_init(&ctl->xready[s], 64);
-            mbar_init(&ctl->xtma[s], 1);
-            mbar_init(&ctl->xempty[s], 1);
-        }
-        for (int s = 0; s < kWStages; ++s) {
-            mbar_init(&ctl->wfull[s], 64 + (PAIR ? 1 : 0));
-            mbar_init(&ctl->wready[s], 64);
-            mbar_init(&ctl->wempty[s], 1 + 4);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&ctl->full[s], 64 + (PAIR ? 1 : 0));
+            mbar_init(&ctl->ready[s], 64);
+            mbar_init(&ctl->tma[s], 1);
+            mbar_init(&ctl->empty[s], 1 + 4);
         }
         mbar_init(&ctl->dx_full, 1);
         mbar_init(&ctl->dx_empty, (PAIR ? 2 : 1) * kEpiWarps);
@@ -214,36 +205,12 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
         // full while the d_x accumulator is being drained.
         const int ptid = threadIdx.x - kProducer0;  // 0..63
         const int prow = ptid >> 3, pg = ptid & 7;  // row within an 8-row block, 16-byte granule
-        int sx = 0;
-        uint32_t px = 0;
+        int kbase = 0;  // the stage index of the tile's first X stage
         bool ok = true;
         Iter it;
         it.first(off, E, lo, hi);
-        // The rows of this CTA's tokens of tile `t` go to L2 ahead of their gathers:
-        // thread (prow, pg) takes rows j * 8 + prow for j = pg and pg + 8, the whole
-        // 1 KiB x row and d_out row of each (the [B, H] gradient of the horizon mean
-        // is small and stays in L2 by itself). Each CTA fetches its own tokens; the
-        // W stages of both CTAs read those rows.
-        auto prefetch_tile = [&](const Iter& t) {
-            const int n = t.ntok();
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int r = kHalf * static_cast<int>(v) + (pg + 8 * jj) * 8 + prow;
-                if (r < n) {
-                    const int tk = perm[t.p0 + r];
-                    prefetch_bulk_l2(x + static_cast<int64_t>(tk) * kH, kH * 4);
-                    if (!COLLAPSE) prefetch_bulk_l2(g_src + static_cast<int64_t>(tk) * kH, kH * 4);
-                }
-            }
-        };
-        if (it.valid(E)) prefetch_tile(it);
         while (ok && it.valid(E)) {
             const int n = it.ntok();
-            {
-                Iter nx = it;
-                nx.next(off, E, lo, hi);
-                if (nx.valid(E)) prefetch_tile(nx);
-            }
             int tx[16];  // the token of rows r = j * 8 + prow
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -251,9 +218,10 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                 tx[j] = (r < n) ? perm[it.p0 + r] : -1;
                 if (COLLAPSE && tx[j] >= 0) tx[j] = tx[j] / g_div;  // the token's gradient row
             }
-            for (int kc = 0; kc < kH / 32 && ok; ++kc) {
-                if (!(ok = mbar_wait(&ctl->xempty[sx], px ^ 1, abort, dev_flags))) break;
-                const uint32_t a_u32 = smem_u32(xring + sx * kStageBytes);
+            for (int kc = 0; kc < nX && ok; ++kc) {
+                const int k = kbase + kc, sl = slot_of(k);
+                if (!(ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags))) break;
+                const uint32_t a_u32 = smem_u32(ring + sl * kStageBytes);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int r = j * 8 + prow;
@@ -261,9 +229,9 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                     const float* src = g_src + static_cast<int64_t>(gr < 0 ? 0 : gr) * kH + kc * 32 + pg * 4;
                     cp_async_16_l2_256(a_u32 + r * 128 + ((pg ^ (r & 7)) << 4), src, gr < 0 ? 0u : 16u);
                 }
-                cp_async_arrive_noinc(leader ? &ctl->xfull[sx] : &ctl->xready[sx]);
-                advance(sx, px, kXStages);
+                cp_async_arrive_noinc(leader ? &ctl->full[sl] : &ctl->ready[sl]);
             }
+            kbase += nX + (n + 31) / 32;
             it.next(off, E, lo, hi);
         }
     } else if (warp >= kProducer0 / 32 + 2 && warp < kProducer0 / 32 + 4) {
@@ -271,8 +239,7 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
         // d_out[., o-half v], B = x[., i-half v], MN-major (32-byte granules)
         const int ptid = threadIdx.x - kProducer0 - 64;  // 0..63
         const int q16 = ptid & 7, gq = (ptid >> 3) & 3, rsub = ptid >> 5;
-        int sw = 0;
-        uint32_t pw = 0;
+        int kbase = 0;  // the stage index of the tile's first X stage
         bool ok = true;
         Iter it;
         it.first(off, E, lo, hi);
@@ -286,8 +253,9 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
             }
             const int ntc = (n + 31) / 32;
             for (int tc = 0; tc < ntc && ok; ++tc) {
-                if (!(ok = mbar_wait(&ctl->wempty[sw], pw ^ 1, abort, dev_flags))) break;
-                const uint32_t a_u32 = smem_u32(wring + sw * kStageBytes);
+                const int k = kbase + nX + tc, sl = slot_of(k);
+                if (!(ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags))) break;
+                const uint32_t a_u32 = smem_u32(ring + sl * kStageBytes);
                 int tok_l = tw[0];
 #pragma unroll
                 for (int j = 1; j < 8; ++j)
@@ -304,37 +272,40 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                     cp_async_16(a_u32 + o, g_src + static_cast<int64_t>(tk < 0 ? 0 : gtk) * kH + col, nb);
                     cp_async_16(a_u32 + kRegion + o, x + static_cast<int64_t>(tk < 0 ? 0 : tk) * kH + col, nb);
                 }
-                cp_async_arrive_noinc(leader ? &ctl->wfull[sw] : &ctl->wready[sw]);
-                advance(sw, pw, kWStages);
+                cp_async_arrive_noinc(leader ? &ctl->full[sl] : &ctl->ready[sl]);
             }
+            kbase += nX + ntc;
             it.next(off, E, lo, hi);
         }
     } else if (warp == kWLoadWarp) {
         // ---------------- W[e] slab (columns i of this CTA's half) for the X stages, by TMA
         if (lane == 0) {
-            int sx = 0;
-            uint32_t px = 0;
-            int issued[kXStages] = {0, 0, 0};  // the parity + 1 of this stage's last load (0: none)
+            int kbase = 0;
+            uint32_t tbits = 0;     // bit s: parity of slot s's next W-slab load
+            uint32_t issued = 0;    // bit s: slot s has had a load
             bool ok = true;
             Iter it;
             it.first(off, E, lo, hi);
             while (ok && it.valid(E)) {
-                for (int kc = 0; kc < kH / 32 && ok; ++kc) {
-                    if (!(ok = mbar_wait(&ctl->xempty[sx], px ^ 1, abort, dev_flags))) break;
-                    mbar_arrive_expect_tx(&ctl->xtma[sx], kRegion);
-                    uint8_t* dst = xring + sx * kStageBytes + kRegion;
+                for (int kc = 0; kc < nX && ok; ++kc) {
+                    const int k = kbase + kc, sl = slot_of(k);
+                    if (!(ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags))) break;
+                    mbar_arrive_expect_tx(&ctl->tma[sl], kRegion);
+                    uint8_t* dst = ring + sl * kStageBytes + kRegion;
 #pragma unroll
                     for (int g = 0; g < kHalf / 32; ++g)
                         tma_load_2d(dst + g * kGroupBytes, tm_w, kHalf * static_cast<int>(v) + g * 32,
-                                    it.e * kH + kc * 32, &ctl->xtma[sx]);
-                    issued[sx] = static_cast<int>(px) + 1;
-                    advance(sx, px, kXStages);
+                                    it.e * kH + kc * 32, &ctl->tma[sl]);
+                    tbits ^= 1u << sl;
+                    issued |= 1u << sl;
                 }
+                kbase += nX + (it.ntok() + 31) / 32;
                 it.next(off, E, lo, hi);
             }
             // let this CTA's loads land before it can leave (already so unless a wait gave up)
-            for (int s = 0; s < kXStages; ++s)
-                if (issued[s]) mbar_wait_drain(&ctl->xtma[s], static_cast<uint32_t>(issued[s] - 1), kWaitLimitCycles);
+            for (int sl = 0; sl < kStages; ++sl)
+                if ((issued >> sl) & 1u)
+                    mbar_wait_drain(&ctl->tma[sl], ((tbits >> sl) & 1u) ^ 1u, kWaitLimitCycles);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -350,8 +321,9 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                 else
                     mma_commit(bar);
             };
-            int sx = 0, sw = 0;
-            uint32_t px = 0, pw = 0, dx_phase = 0, dw_phase = 0;
+            int kbase = 0;
+            uint32_t tbits = 0;  // bit s: parity of slot s's next W-slab load
+            uint32_t dx_phase = 0, dw_phase = 0;
             bool ok = true;
             Iter it;
             it.first(off, E, lo, hi);
@@ -359,12 +331,14 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                 // d_x of this pair-tile: the accumulator must have been drained by both CTAs
                 if (!(ok = mbar_wait_cl(&ctl->dx_empty, dx_phase ^ 1, abort, dev_flags))) break;
                 tc_fence_after();
-                for (int kc = 0; kc < kH / 32; ++kc) {
-                    if (!(ok = mbar_wait_cl(&ctl->xfull[sx], px, abort, dev_flags))) break;
-                    if (!(ok = mbar_wait(&ctl->xtma[sx], px, abort, dev_flags))) break;
+                for (int kc = 0; kc < nX; ++kc) {
+                    const int k = kbase + kc, sl = slot_of(k);
+                    if (!(ok = mbar_wait_cl(&ctl->full[sl], parity_of(k), abort, dev_flags))) break;
+                    if (!(ok = mbar_wait(&ctl->tma[sl], (tbits >> sl) & 1u, abort, dev_flags))) break;
+                    tbits ^= 1u << sl;
                     fence_proxy_async_smem();
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(xring + sx * kStageBytes);
+                    const uint32_t a_addr = smem_u32(ring + sl * kStageBytes);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t ad = sw128_desc(a_addr + ks * 32, 16, 1024);
@@ -375,8 +349,7 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                         else
                             mma_tf32(tmem_dx, ad, bd, idesc_dx, accumulate);
                     }
-                    commit_all(&ctl->xempty[sx]);
-                    advance(sx, px, kXStages);
+                    commit_all(&ctl->empty[sl]);
                 }
                 if (!ok) break;
                 commit_all(&ctl->dx_full);
@@ -388,10 +361,11 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                 }
                 const int ntc = (it.ntok() + 31) / 32;
                 for (int tc = 0; tc < ntc; ++tc) {
-                    if (!(ok = mbar_wait_cl(&ctl->wfull[sw], pw, abort, dev_flags))) break;
+                    const int k = kbase + nX + tc, sl = slot_of(k);
+                    if (!(ok = mbar_wait_cl(&ctl->full[sl], parity_of(k), abort, dev_flags))) break;
                     fence_proxy_async_smem();
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(wring + sw * kStageBytes);
+                    const uint32_t a_addr = smem_u32(ring + sl * kStageBytes);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t ad = sw128_32b_mn_desc(a_addr + ks * 1024, kGroupBytes, 512);
@@ -402,14 +376,14 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                         else
                             mma_tf32(tmem_dw, ad, bd, idesc_dw, accumulate);
                     }
-                    commit_all(&ctl->wempty[sw]);
-                    advance(sw, pw, kWStages);
+                    commit_all(&ctl->empty[sl]);
                 }
                 if (!ok) break;
                 if (it.last_in_run()) {
                     commit_all(&ctl->dw_full);
                     dw_phase ^= 1;
                 }
+                kbase += nX + ntc;
                 it.next(off, E, lo, hi);
             }
             // every MMA issued (and every commit arrival on the odd CTA) is done before the pair may leave
@@ -420,29 +394,30 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
             mbar_wait_drain(&ctl->done, 0, kWaitLimitCycles);
         } else if (PAIR && !leader && lane == 0) {
             // ---------------- relay (odd CTA): this CTA's stage has landed -> the even CTA's barrier
-            const uint32_t xfull0 = mapa_shared(smem_u32(&ctl->xfull[0]), 0);
-            const uint32_t wfull0 = mapa_shared(smem_u32(&ctl->wfull[0]), 0);
-            int sx = 0, sw = 0;
-            uint32_t px = 0, pw = 0;
+            const uint32_t full0 = mapa_shared(smem_u32(&ctl->full[0]), 0);
+            int kbase = 0;
+            uint32_t tbits = 0;
             bool ok = true;
             Iter it;
             it.first(off, E, lo, hi);
             while (ok && it.valid(E)) {
-                for (int kc = 0; kc < kH / 32; ++kc) {
-                    if (!(ok = mbar_wait(&ctl->xready[sx], px, abort, dev_flags))) break;
-                    if (!(ok = mbar_wait(&ctl->xtma[sx], px, abort, dev_flags))) break;
+                for (int kc = 0; kc < nX; ++kc) {
+                    const int k = kbase + kc, sl = slot_of(k);
+                    if (!(ok = mbar_wait(&ctl->ready[sl], parity_of(k), abort, dev_flags))) break;
+                    if (!(ok = mbar_wait(&ctl->tma[sl], (tbits >> sl) & 1u, abort, dev_flags))) break;
+                    tbits ^= 1u << sl;
                     fence_proxy_async_smem();
-                    mbar_arrive_cluster(xfull0 + sx * 8);
-                    advance(sx, px, kXStages);
+                    mbar_arrive_cluster(full0 + sl * 8);
                 }
                 if (!ok) break;
                 const int ntc = (it.ntok() + 31) / 32;
                 for (int tc = 0; tc < ntc; ++tc) {
-                    if (!(ok = mbar_wait(&ctl->wready[sw], pw, abort, dev_flags))) break;
+                    const int k = kbase + nX + tc, sl = slot_of(k);
+                    if (!(ok = mbar_wait(&ctl->ready[sl], parity_of(k), abort, dev_flags))) break;
                     fence_proxy_async_smem();
-                    mbar_arrive_cluster(wfull0 + sw * 8);
-                    advance(sw, pw, kWStages);
+                    mbar_arrive_cluster(full0 + sl * 8);
                 }
+                kbase += nX + ntc;
                 it.next(off, E, lo, hi);
             }
         }
@@ -522,28 +497,33 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
         const int tdb = threadIdx.x - kDbWarp0 * 32;  // 0..127
         const int dq = warp & 3;
         const int g = tdb >> 5, jo = tdb & 31;
-        int sw = 0;
-        uint32_t pw = 0, dw_phase = 0;
+        int kbase = 0;
+        uint32_t dw_phase = 0;
         float db_run = 0.0f;
         bool ok = true;
         Iter it;
         it.first(off, E, lo, hi);
         while (ok && it.valid(E)) {
+            // every stage of the ring passes here once (its slot is released by the MMA's
+            // commit and these four warps); only the W stages hold d_out rows to sum
             const int ntc = (it.ntok() + 31) / 32;
-            for (int tc = 0; tc < ntc; ++tc) {
-                ok = leader ? mbar_wait_cl(&ctl->wfull[sw], pw, abort, dev_flags)
-                            : mbar_wait(&ctl->wready[sw], pw, abort, dev_flags);
+            for (int j = 0; j < nX + ntc; ++j) {
+                const int k = kbase + j, sl = slot_of(k);
+                ok = leader ? mbar_wait_cl(&ctl->full[sl], parity_of(k), abort, dev_flags)
+                            : mbar_wait(&ctl->ready[sl], parity_of(k), abort, dev_flags);
                 if (!ok) break;
-                const uint8_t* colbase = wring + sw * kStageBytes + g * kGroupBytes + (jo & 7) * 4;
-                float acc = 0.0f;
+                if (j >= nX) {
+                    const uint8_t* colbase = ring + sl * kStageBytes + g * kGroupBytes + (jo & 7) * 4;
+                    float acc = 0.0f;
 #pragma unroll 8
-                for (int rr = 0; rr < 32; ++rr)
-                    acc += *reinterpret_cast<const float*>(colbase + rr * 128 + (((jo >> 3) ^ (rr & 3)) << 5));
-                db_run += acc;
+                    for (int rr = 0; rr < 32; ++rr)
+                        acc += *reinterpret_cast<const float*>(colbase + rr * 128 + (((jo >> 3) ^ (rr & 3)) << 5));
+                    db_run += acc;
+                }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->wempty[sw]);
-                advance(sw, pw, kWStages);
+                if (lane == 0) mbar_arrive(&ctl->empty[sl]);
             }
+            kbase += nX + ntc;
             if (!ok) break;
             if (it.last_in_run()) {
                 if (!(ok = mbar_wait_cl(&ctl->dw_full, dw_phase, abort, dev_flags))) break;
