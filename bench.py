@@ -122,13 +122,14 @@ def host_cpu() -> dict:
     return {"cpu_model": model, "cores_available": avail}
 
 
-TRAFFIC_RECORD = os.path.join(HERE, "profiles", "launch_list_large_b65536_e8_h256.md")
+TRAFFIC_RECORD = os.path.join(HERE, "profiles", "traffic_mid_b16384_e8_h256.md")
 
-# The library kernels each timed call launches, per (call, fused TF32 H = 256 backward).
+# The library kernels each timed call launches, per (call, fused TF32 backward).
 CALL_KERNELS = {
-    ("fwd", True): ["grouped_tf32_kernel"], ("fwd", False): ["grouped_tf32_kernel or grouped_ffma_kernel"],
-    ("bwd", True): ["bwd_fused_tf32_kernel", "wgrad_reduce_kernel"],
-    ("bwd", False): ["grouped d_x kernel", "weight-gradient kernel", "wgrad_reduce_kernel"],
+    ("fwd", True): ["grouped_tf32_kernel (hmean_fwd_tf32_sum_kernel with the horizon mean)"],
+    ("fwd", False): ["grouped_ffma_kernel"],
+    ("bwd", True): ["bwd_fused_pair_kernel (H = 256) / bwd_fused_single_kernel (H = 128)", "wgrad_reduce_kernel"],
+    ("bwd", False): ["grouped_ffma_kernel (d_x)", "wgrad_ffma_kernel", "wgrad_reduce_kernel"],
 }
 
 
@@ -147,20 +148,31 @@ def code_sha1(paths) -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(call: str, workload: str, math_name: str):
-    """DRAM bytes (read + write) of one launch of `call` from the committed ncu
-    launch list, or None when there is no record for this workload and math
-    mode, or when the kernel code changed since the counters were taken."""
+def scale_traffic(measured: int, fixed: int, scale: float) -> int:
+    """DRAM bytes of a full launch from a capture of a smaller one: the part that
+    moves with the tokens grows by the token ratio, the part that does not (W, the
+    partial-sum slots, bias) is taken as its algorithmic size at both sizes."""
+    return int(round(fixed + (measured - fixed) * scale))
+
+
+def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "token"):
+    """DRAM bytes (read + write) of one launch of `call`, from the committed ncu
+    record (counters taken on a smaller case of the same shape and scaled to the
+    workload), or None when there is no record for this workload, gradient mode
+    and math mode, or when the kernel code changed since the counters were taken."""
     try:
         text = open(TRAFFIC_RECORD).read()
-        rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
-        digest = code_sha1([os.path.join(HERE, f) for f in rec["source_files"]])
+        data = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
+        digest = code_sha1([os.path.join(HERE, f) for f in data["source_files"]])
     except (OSError, IndexError, KeyError, ValueError):
         return None
-    if rec.get("workload") != workload or rec.get("math") != math_name or digest != rec.get("code_sha1"):
+    if digest != data.get("code_sha1"):
         return None
-    v = rec.get("traffic_bytes_per_call", {}).get(call)
-    return int(v) if v is not None else None
+    for rec in data.get("records", []):
+        if rec.get("workload") == workload and rec.get("math") == math_name and rec.get("grad") == grad:
+            v = rec.get("traffic_bytes_per_call", {}).get(call)
+            return int(v) if v is not None else None
+    return None
 
 
 class ClockSampler:
@@ -499,7 +511,7 @@ def main():
             "roofline": {"bound": "hbm", "kernel": dominant, "launches_in_call": CALL_KERNELS[(dominant, fused)],
                          "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm,
-                         "traffic": None if collapse else recorded_traffic(dominant, spec.name, args.math),
+                         "traffic": recorded_traffic(dominant, spec.name, args.math, args.grad),
                          "algorithmic_bytes": kbytes[dominant], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "flops": step_flops, "t_roofline_ms": t_roof * 1e3,
                               "frac": t_roof * 1e3 / ms_per_step,

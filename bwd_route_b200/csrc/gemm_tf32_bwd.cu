@@ -35,7 +35,8 @@
 //
 // Warp roles (each CTA): 0-7 drain the d_x accumulator (TMEM -> transpose in
 // shared memory -> token rows); 8-9 gather the X stages' rows and 10-11 the W
-// stages' rows with cp.async, each pair of warps running ahead on its own; 12: the
+// stages' rows with cp.async (each pair of warps fills the stages of its kind and
+// passes the others, see the ring below); 12: the
 // MMA issuer (even CTA) or the relay (odd CTA: once its stage has landed, it
 // makes it visible to the tensor core and arrives on the even CTA's barrier);
 // 13 loads the W[e] slab by TMA; 14-17 sum d_out over the staged tokens for db
@@ -67,15 +68,24 @@ constexpr int kDbWarp0 = 14;     // warps 14-17
 // One ring of stages, filled and consumed in the MMA's order: each tile's X
 // stages (d_x: 32 o each), then its W stages (dW: 32 tokens each). A single
 // ring keeps all of its slots loading whichever kind of stage comes next.
+// Every role that waits on a slot's empty barrier passes every stage in order,
+// the ones it does not fill included, and arrives on that stage's full (ready)
+// barrier: a stage cannot be consumed before each such role has reached it, so
+// no role is ever more than one phase away from a slot's current phase and the
+// parity waits stay unambiguous. (A role that skipped the other kind's stages
+// could reach a slot two phases on and see a stale phase as its own.)
 constexpr int kStages = 6;
+// full / ready arrivals: the 64 threads that gather the stage's rows (cp.async),
+// the 64 threads of the other producer kind and the W-slab loader
+constexpr int kFullArrivals = 64 + 64 + 1;
 constexpr int kStageBytes = 32768;  // region 0 (A) and region 1 (B), 16 KiB each
 constexpr int kRegion = 16384;
 constexpr int kGroupBytes = 4096;   // MN-major: 32 rows x 128 bytes per 32-wide column group
 constexpr int kStgBytes = kEpiWarps * 32 * 128;
 
 struct __align__(8) Ctl {
-    uint64_t full[kStages];   // even CTA: the 64 threads that gather the stage + the odd CTA's relay
-    uint64_t ready[kStages];  // odd CTA: the 64 threads that gather the stage
+    uint64_t full[kStages];   // even CTA: kFullArrivals + the odd CTA's relay
+    uint64_t ready[kStages];  // odd CTA: kFullArrivals
     uint64_t tma[kStages];    // each CTA: its own W-slab TMA of an X stage (arrival + bytes)
     uint64_t empty[kStages];  // each CTA: the pair's MMA commit + its 4 db warps
     uint64_t dx_full;         // each CTA: MMA commit
@@ -163,8 +173,8 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&ctl->full[s], 64 + (PAIR ? 1 : 0));
-            mbar_init(&ctl->ready[s], 64);
+            mbar_init(&ctl->full[s], kFullArrivals + (PAIR ? 1 : 0));
+            mbar_init(&ctl->ready[s], kFullArrivals);
             mbar_init(&ctl->tma[s], 1);
             mbar_init(&ctl->empty[s], 1 + 4);
         }
@@ -200,9 +210,7 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
 
     if (warp >= kProducer0 / 32 && warp < kProducer0 / 32 + 2) {
         // ---------------- X-stage producers (warps 8-9): A = the d_out rows of this
-        // CTA's 128 tokens, 32 o per stage, K-major (128-byte swizzle). They run
-        // ahead of the W-stage producers independently, so that both rings stay
-        // full while the d_x accumulator is being drained.
+        // CTA's 128 tokens, 32 o per stage, K-major (128-byte swizzle).
         const int ptid = threadIdx.x - kProducer0;  // 0..63
         const int prow = ptid >> 3, pg = ptid & 7;  // row within an 8-row block, 16-byte granule
         int kbase = 0;  // the stage index of the tile's first X stage
@@ -231,9 +239,16 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                 }
                 cp_async_arrive_noinc(leader ? &ctl->full[sl] : &ctl->ready[sl]);
             }
-            kbase += nX + (n + 31) / 32;
+            const int ntc = (n + 31) / 32;
+            for (int tc = 0; tc < ntc && ok; ++tc) {  // pass the W stages
+                const int k = kbase + nX + tc, sl = slot_of(k);
+                if (!(ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags))) break;
+                mbar_arrive(leader ? &ctl->full[sl] : &ctl->ready[sl]);
+            }
+            kbase += nX + ntc;
             it.next(off, E, lo, hi);
         }
+        cp_async_wait_all();  // nothing in flight into this CTA's shared memory when it leaves
     } else if (warp >= kProducer0 / 32 + 2 && warp < kProducer0 / 32 + 4) {
         // ---------------- W-stage producers (warps 10-11): 32 tokens per stage; A =
         // d_out[., o-half v], B = x[., i-half v], MN-major (32-byte granules)
@@ -252,9 +267,15 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                 tw[j] = (q < n) ? perm[it.p0 + q] : -1;
             }
             const int ntc = (n + 31) / 32;
+            for (int kc = 0; kc < nX && ok; ++kc) {  // pass the X stages
+                const int k = kbase + kc, sl = slot_of(k);
+                if (!(ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags))) break;
+                mbar_arrive(leader ? &ctl->full[sl] : &ctl->ready[sl]);
+            }
             for (int tc = 0; tc < ntc && ok; ++tc) {
                 const int k = kbase + nX + tc, sl = slot_of(k);
-                if (!(ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags))) break;
+                ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags);
+                if (!(ok = __all_sync(0xffffffffu, ok))) break;  // the gather below shuffles across the warp
                 const uint32_t a_u32 = smem_u32(ring + sl * kStageBytes);
                 int tok_l = tw[0];
 #pragma unroll
@@ -277,6 +298,7 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
             kbase += nX + ntc;
             it.next(off, E, lo, hi);
         }
+        cp_async_wait_all();
     } else if (warp == kWLoadWarp) {
         // ---------------- W[e] slab (columns i of this CTA's half) for the X stages, by TMA
         if (lane == 0) {
@@ -298,8 +320,15 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
                                     it.e * kH + kc * 32, &ctl->tma[sl]);
                     tbits ^= 1u << sl;
                     issued |= 1u << sl;
+                    mbar_arrive(leader ? &ctl->full[sl] : &ctl->ready[sl]);
                 }
-                kbase += nX + (it.ntok() + 31) / 32;
+                const int ntc = (it.ntok() + 31) / 32;
+                for (int tc = 0; tc < ntc && ok; ++tc) {  // pass the W stages
+                    const int k = kbase + nX + tc, sl = slot_of(k);
+                    if (!(ok = mbar_wait(&ctl->empty[sl], parity_of(k) ^ 1, abort, dev_flags))) break;
+                    mbar_arrive(leader ? &ctl->full[sl] : &ctl->ready[sl]);
+                }
+                kbase += nX + ntc;
                 it.next(off, E, lo, hi);
             }
             // let this CTA's loads land before it can leave (already so unless a wait gave up)
