@@ -163,15 +163,15 @@ def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "toke
     try:
         text = open(TRAFFIC_RECORD).read()
         data = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
-        digest = code_sha1([os.path.join(HERE, f) for f in data["source_files"]])
-    except (OSError, IndexError, KeyError, ValueError):
-        return None
-    if digest != data.get("code_sha1"):
-        return None
-    for rec in data.get("records", []):
-        if rec.get("workload") == workload and rec.get("math") == math_name and rec.get("grad") == grad:
-            v = rec.get("traffic_bytes_per_call", {}).get(call)
+        for rec in data["records"]:
+            if rec["workload"] != workload or rec["math"] != math_name or rec["grad"] != grad:
+                continue
+            if code_sha1([os.path.join(HERE, f) for f in rec["source_files"]]) != rec["code_sha1"]:
+                return None
+            v = rec["traffic_bytes_per_call"].get(call)
             return int(v) if v is not None else None
+    except (OSError, IndexError, KeyError, ValueError, TypeError):
+        return None
     return None
 
 

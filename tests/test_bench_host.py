@@ -51,11 +51,31 @@ def test_fp32_simt_ceiling_and_l2_note():
 
 def test_traffic_record_is_well_formed_and_keyed_to_the_sources():
     text = open(bench.TRAFFIC_RECORD).read()
-    rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
-    assert rec["workload"] == LARGE.name and rec["math"] == "tf32"
-    for f in rec["source_files"]:
-        assert os.path.exists(os.path.join(bench.HERE, f)), f
-    assert set(rec["traffic_bytes_per_call"]) == {"fwd", "d_x", "wgrad"}
-    # the lookup refuses other workloads and the FFMA path
+    data = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
+    recs = {(r["workload"], r["grad"]): r for r in data["records"]}
+    assert set(recs) == {(LARGE.name, "token"), (LARGE.name, "mean_collapse")}
+    for (_, grad), rec in recs.items():
+        assert rec["math"] == "tf32"
+        for f in rec["source_files"]:
+            assert os.path.exists(os.path.join(bench.HERE, f)), f
+        mid = wl.WORKLOADS[rec["measured_workload"]]
+        assert (mid.E, mid.H, mid.N_H) == (LARGE.E, LARGE.H, LARGE.N_H) and rec["token_scale"] == LARGE.T / mid.T
+        _, _, per = bench.algorithmic(LARGE, grad)
+        assert set(rec["traffic_bytes_per_call"]) == {"fwd", "bwd"}
+        for call, v in rec["traffic_bytes_per_call"].items():
+            # the scaled figure is the stated rule applied to the stored measurement
+            assert v == bench.scale_traffic(rec["measured_bytes_per_call"][call], rec["fixed_bytes_per_call"][call],
+                                            rec["token_scale"])
+            # the fixed part is W (and bias, or the partial-sum slots): far below the token part
+            assert LARGE.E * LARGE.H * LARGE.H * 4 <= rec["fixed_bytes_per_call"][call] < 0.05 * v
+            assert 0.85 < v / per[call] < 1.1, (grad, call, v / per[call])
+    # the lookup refuses other workloads, the FFMA path and a gradient mode with no record
     assert bench.recorded_traffic("fwd", "mid_b16384_e8_h256", "tf32") is None
     assert bench.recorded_traffic("fwd", LARGE.name, "ffma") is None
+    assert bench.recorded_traffic("fwd", LARGE.name, "tf32", "other") is None
+
+
+def test_traffic_scaling_rule():
+    # fixed part kept, token part times the ratio
+    assert bench.scale_traffic(1000, 100, 4) == 100 + 900 * 4
+    assert bench.scale_traffic(100, 100, 4) == 100
