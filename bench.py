@@ -128,8 +128,9 @@ TRAFFIC_RECORD = os.path.join(HERE, "profiles", "traffic_mid_b16384_e8_h256.md")
 CALL_KERNELS = {
     ("fwd", True): ["grouped_tf32_kernel (hmean_fwd_tf32_sum_kernel with the horizon mean)"],
     ("fwd", False): ["grouped_ffma_kernel"],
-    ("bwd", True): ["bwd_fused_pair_kernel (H = 256) / bwd_fused_single_kernel (H = 128)", "wgrad_reduce_kernel"],
+    ("bwd", True): ["grouped_tf32_kernel (d_x)", "wgrad_tf32_kernel", "wgrad_reduce_kernel"],
     ("bwd", False): ["grouped_ffma_kernel (d_x)", "wgrad_ffma_kernel", "wgrad_reduce_kernel"],
+    ("bwd", "mean_collapse"): ["bwd_fused_pair_kernel", "wgrad_reduce_kernel"],
 }
 
 
@@ -155,11 +156,18 @@ def scale_traffic(measured: int, fixed: int, scale: float) -> int:
     return int(round(fixed + (measured - fixed) * scale))
 
 
-def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "token"):
+def bwd_passes(math_name: str, grad: str, H: int) -> int:
+    """Contraction passes of the library's default TF32 backward: one fused pass for
+    the horizon-mean gradient at H = 256, two (d_x; dW and db) otherwise."""
+    return 1 if (math_name == "tf32" and grad == "mean_collapse" and H == 256) else 2
+
+
+def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "token", H: int = 256):
     """DRAM bytes (read + write) of one launch of `call`, from the committed ncu
     record (counters taken on a smaller case of the same shape and scaled to the
     workload), or None when there is no record for this workload, gradient mode
-    and math mode, or when the kernel code changed since the counters were taken."""
+    and math mode, when the recorded backward ran another number of passes than
+    the default path, or when the kernel code changed since the counters were taken."""
     try:
         text = open(TRAFFIC_RECORD).read()
         data = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
@@ -167,6 +175,8 @@ def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "toke
             if rec["workload"] != workload or rec["math"] != math_name or rec["grad"] != grad:
                 continue
             if code_sha1([os.path.join(HERE, f) for f in rec["source_files"]]) != rec["code_sha1"]:
+                return None
+            if call == "bwd" and rec.get("bwd_passes") != bwd_passes(math_name, grad, H):
                 return None
             v = rec["traffic_bytes_per_call"].get(call)
             return int(v) if v is not None else None
@@ -508,10 +518,12 @@ def main():
                        "N_H": spec.N_H, "E": E, "H": H, "tokens": T, "grad": args.grad,
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": l2_note(spec, collapse, flush is not None)},
-            "roofline": {"bound": "hbm", "kernel": dominant, "launches_in_call": CALL_KERNELS[(dominant, fused)],
+            "roofline": {"bound": "hbm", "kernel": dominant, "launches_in_call": CALL_KERNELS[
+                             (dominant, "mean_collapse") if (fused and collapse and H == 256 and dominant == "bwd")
+                             else (dominant, fused)],
                          "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm,
-                         "traffic": recorded_traffic(dominant, spec.name, args.math, args.grad),
+                         "traffic": recorded_traffic(dominant, spec.name, args.math, args.grad, H),
                          "algorithmic_bytes": kbytes[dominant], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "flops": step_flops, "t_roofline_ms": t_roof * 1e3,
                               "frac": t_roof * 1e3 / ms_per_step,
@@ -524,7 +536,7 @@ def main():
                       + ("; 256 MB written between steps, outside their events" if flush is not None else ""),
             "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
                     "h2d_bytes_per_step": (T * (E + H) + g_host.shape[0] * H) * 4, "d2h_bytes_per_step": 8},
-            "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode, H, T, E),
+            "gpu_launches": args.steps * MoETop1Gate.launches_per_step(math_mode, H, T, E, collapse),
             "clocks": clocks.summary(),
             "device_flags": flags,
         }

@@ -178,9 +178,10 @@ bool encode_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t 
 }
 
 // Body of both backward entry points: token t's output gradient is
-// g_scale * d_out[t / g_div] (d_out has g_rows rows).
+// g_scale * d_out[t / g_div] (d_out has g_rows rows; collapse: the [B, H]
+// gradient of the horizon mean).
 moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_t g_rows, int g_div, float g_scale,
-                      const moe_routing_t* routing,
+                      bool collapse, const moe_routing_t* routing,
                           int64_t B, int64_t N_H, int32_t E, int32_t H, moe_math_t math, float* d_x, float* dW,
                           float* db, uint32_t accumulate_flags, void* workspace, size_t workspace_bytes,
                           void* stream) {
@@ -188,7 +189,7 @@ moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_
     moe_status_t st = tokens(B, N_H, &T);
     if (st != MOE_OK) return st;
     if (math != MOE_MATH_TF32 && math != MOE_MATH_FFMA) return MOE_ERR_INVALID_ARG;
-    if (accumulate_flags & ~(MOE_ACC_DX | MOE_ACC_DW | MOE_ACC_DB)) return MOE_ERR_INVALID_ARG;
+    if (accumulate_flags & ~(MOE_ACC_DX | MOE_ACC_DW | MOE_ACC_DB | MOE_BWD_SINGLE_PASS)) return MOE_ERR_INVALID_ARG;
     if (E < 1 || E > 32 || !h_supported(H, math)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!routing) return MOE_ERR_INVALID_ARG;
     if (!d_x && !dW && !db) return MOE_OK;
@@ -230,8 +231,15 @@ moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
-    if (math == MOE_MATH_TF32 && d_x && (dW || db)) {
-        // one pass over d_out: d_x, and the dW / db partial sums, then the slot reduction.
+    // One pass over d_out (d_x and the dW / db partial sums together), or two (d_x,
+    // then dW / db): the single pass reads d_out and x once, but on the B200 the two
+    // passes take less time for the per-token gradient (0.735 against 0.792 ms at
+    // 1,048,576 tokens, H 256), so the single pass is the default only for the
+    // [B, H] gradient of the horizon mean at H = 256 (0.733 against 0.757 ms), and
+    // on request (MOE_BWD_SINGLE_PASS).
+    const bool single_pass = math == MOE_MATH_TF32 && d_x && (dW || db) &&
+                             ((accumulate_flags & MOE_BWD_SINGLE_PASS) || (collapse && H == 256));
+    if (single_pass) {
         // H = 256: pairs of CTAs (as many as run at once); H = 128: single CTAs, one
         // per wgrad_splits(T) range
         float* part = reinterpret_cast<float*>(ws + L.wg_part);
@@ -435,8 +443,8 @@ moe_status_t moe_top1_bwd(const float* x, const float* W, const float* d_out, co
     int64_t T = 0;
     moe_status_t st = tokens(B, N_H, &T);
     if (st != MOE_OK) return st;
-    return bwd_impl(x, W, d_out, T, 1, 1.0f, routing, B, N_H, E, H, math, d_x, dW, db, accumulate_flags, workspace,
-                    workspace_bytes, stream);
+    return bwd_impl(x, W, d_out, T, 1, 1.0f, false, routing, B, N_H, E, H, math, d_x, dW, db, accumulate_flags,
+                    workspace, workspace_bytes, stream);
 }
 
 moe_status_t moe_top1_bwd_mean_collapse(const float* x, const float* W, const float* grad_ctx_mean,
@@ -449,7 +457,7 @@ moe_status_t moe_top1_bwd_mean_collapse(const float* x, const float* W, const fl
     if (N_H > (int64_t{1} << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const int g_div = T > 0 ? static_cast<int>(N_H) : 1;
     const float g_scale = T > 0 ? static_cast<float>(1.0 / static_cast<double>(N_H)) : 1.0f;
-    return bwd_impl(x, W, grad_ctx_mean, B, g_div, g_scale, routing, B, N_H, E, H, math, d_x, dW, db,
+    return bwd_impl(x, W, grad_ctx_mean, B, g_div, g_scale, true, routing, B, N_H, E, H, math, d_x, dW, db,
                     accumulate_flags, workspace, workspace_bytes, stream);
 }
 

@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
                                                       float* __restrict__ d_logits, float* __restrict__ blk_psum,
                                                       uint32_t* __restrict__ ticket, float* __restrict__ loss_out,
                                                       float* __restrict__ mean_p, float* __restrict__ stats) {
+    griddep_wait();  // every global access below comes after the previous grid
     constexpr int Q = EMAX / 4;          // float4s per staged row
     constexpr int BUF4 = kChunk * Q;     // float4s per chunk buffer
     extern __shared__ float4 s_dyn4[];   // kWarps x kChunksPerWarp chunk buffers
@@ -281,11 +282,13 @@ __global__ void __launch_bounds__(kThreads) aux_finalize_kernel(const int32_t* _
                                                                const float* __restrict__ lambda_eff,
                                                                float* __restrict__ loss_out, float* __restrict__ mean_p,
                                                                float* __restrict__ stats) {
+    griddep_wait();  // every global access below comes after the previous grid
     aux_finalize_block(nullptr, 0, counts, 0, E, lambda_eff, loss_out, mean_p, stats);
 }
 
 __global__ void lambda_eff_kernel(const float* __restrict__ ent_ema, float lambda_floor, float lambda_max_extra,
                                   float ent_target, float* __restrict__ lambda_eff) {
+    griddep_wait();  // every global access below comes after the previous grid
     float deficit = ent_target - *ent_ema;
     if (!(deficit > 0.0f)) deficit = 0.0f;  // max(0, .); a NaN entropy gives the floor
     *lambda_eff = lambda_floor + lambda_max_extra * deficit / ent_target;
@@ -299,6 +302,7 @@ __global__ void lambda_eff_kernel(const float* __restrict__ ent_ema, float lambd
 __global__ void usage_entropy_ema_kernel(const int32_t* __restrict__ counts, int64_t T, int E, float alpha,
                                          int reset, float* __restrict__ usage_ema, float* __restrict__ ent_ema,
                                          float* __restrict__ ent_step) {
+    griddep_wait();  // every global access below comes after the previous grid
     const int lane = threadIdx.x;
     const bool on = lane < E;
     const double f = (on && T > 0) ? static_cast<double>(counts[lane]) / static_cast<double>(T) : 0.0;
@@ -320,7 +324,8 @@ __global__ void usage_entropy_ema_kernel(const int32_t* __restrict__ counts, int
 
 cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, float alpha, int reset,
                                      float* usage_ema, float* ent_ema, float* ent_step, cudaStream_t s) {
-    usage_entropy_ema_kernel<<<1, 32, 0, s>>>(counts, T, E, alpha, reset, usage_ema, ent_ema, ent_step);
+    launch_pdl(usage_entropy_ema_kernel, dim3(1), dim3(32), 0, s,
+               counts, T, E, alpha, reset, usage_ema, ent_ema, ent_step);
     return cudaGetLastError();
 }
 
@@ -328,29 +333,31 @@ cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, in
                        float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,
                        uint32_t* ticket, cudaStream_t s) {
     if (T == 0) {
-        aux_finalize_kernel<<<1, kThreads, 0, s>>>(counts, E, lambda_eff, loss_out, mean_p, stats);
+        launch_pdl(aux_finalize_kernel, dim3(1), dim3(kThreads), 0, s,
+                   counts, E, lambda_eff, loss_out, mean_p, stats);
         return cudaGetLastError();
     }
     const int64_t nblk = (T + kAuxTokPerBlk - 1) / kAuxTokPerBlk;
     const size_t smem = sizeof(float) * kWarps * kChunksPerWarp * kChunk * (E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32);
     if (E <= 4)
-        aux_kernel<4><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
-                                                            ticket, loss_out, mean_p, stats);
+        launch_pdl(aux_kernel<4>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
+                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
     else if (E <= 8)
-        aux_kernel<8><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
-                                                            ticket, loss_out, mean_p, stats);
+        launch_pdl(aux_kernel<8>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
+                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
     else if (E <= 16)
-        aux_kernel<16><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
-                                                             ticket, loss_out, mean_p, stats);
+        launch_pdl(aux_kernel<16>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
+                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
     else
-        aux_kernel<32><<<(unsigned)nblk, kThreads, smem, s>>>(logits, counts, T, E, lambda_eff, d_logits, blk_psum,
-                                                             ticket, loss_out, mean_p, stats);
+        launch_pdl(aux_kernel<32>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
+                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
     return cudaGetLastError();
 }
 
 cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float lambda_max_extra, float ent_target,
                               float* lambda_eff, cudaStream_t s) {
-    lambda_eff_kernel<<<1, 1, 0, s>>>(ent_ema, lambda_floor, lambda_max_extra, ent_target, lambda_eff);
+    launch_pdl(lambda_eff_kernel, dim3(1), dim3(1), 0, s,
+               ent_ema, lambda_floor, lambda_max_extra, ent_target, lambda_eff);
     return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@
 // expert in ascending t, with every expert index in [0, E).
 #include <cstdint>
 
+#include "common.cuh"
 #include "internal.h"
 #include "moe_top1.h"
 
@@ -33,6 +34,7 @@ __global__ void __launch_bounds__(kThreads)
 check_routing_kernel(const int32_t* __restrict__ expert_idx, const int32_t* __restrict__ counts,
                      const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int64_t T, int E,
                      uint32_t* __restrict__ flags) {
+    griddep_wait();  // every global access below comes after the previous grid
     __shared__ int32_t s_off[33];
     __shared__ int s_offsets_ok;
     if (threadIdx.x == 0) {
@@ -93,8 +95,7 @@ extern "C" moe_status_t moe_top1_check_routing(const moe_routing_t* routing, int
     const int64_t want = (T + kThreads - 1) / kThreads;
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
-    check_routing_kernel<<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        routing->expert_idx, routing->counts, routing->offsets, routing->perm, T, E,
-        static_cast<uint32_t*>(workspace));
+    launch_pdl(check_routing_kernel, dim3(grid), dim3(kThreads), 0, static_cast<cudaStream_t>(stream),
+               routing->expert_idx, routing->counts, routing->offsets, routing->perm, T, E, static_cast<uint32_t*>(workspace));
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

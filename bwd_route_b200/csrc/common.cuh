@@ -18,6 +18,16 @@ namespace moe {
 // kernel return instead of hanging the GPU.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
+// Programmatic dependent launch: this kernel waits here until the grid before it
+// in the stream has completed and its memory operations are visible. Every kernel
+// calls it before its first global-memory access (read or write); a no-op when the
+// launch did not allow an early start. No kernel triggers its dependents early
+// (griddepcontrol.launch_dependents): with a trigger at kernel start the next
+// kernel's CTAs sat resident through the whole kernel and steps of 20k-80k tokens
+// ran 5-7 % slower; the implicit trigger at exit lets the next kernel's prologue
+// overlap only this kernel's teardown (2-5 % faster steps at 40-20k tokens).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -150,6 +160,27 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::tf32, one CTA, with A read from tensor
+// memory: row m of A in lane m, its K = 8 values in 8 consecutive columns from
+// a_tmem (A from tensor memory is K-major only).
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Copies a 128-row x 32-byte matrix from shared memory, described like a
+// K-major MMA operand, into tensor-memory lanes 0-127, 8 consecutive 32-bit
+// columns from taddr. Asynchronous like the MMAs: the tcgen05 operations one
+// thread issues run in issue order, and mma_commit covers it.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t s_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
 }
 
 // The mbarrier gets one arrival when every tcgen05 op issued so far by this
@@ -395,6 +426,11 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, fl
 __device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
 }
 

@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(kGThreads) grouped_ffma_kernel(const float* __
                                                                 const int32_t* __restrict__ perm, int E,
                                                                 int H, int b_kmajor, int accumulate, int src_div,
                                                                 float out_scale, float* __restrict__ out) {
+    griddep_wait();  // every global access below comes after the previous grid
     __shared__ int s_off[33];
     __shared__ int s_tstart[33];
     __shared__ int s_tok[kGBM];
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(kGThreads) hmean_fwd_ffma_kernel(const float* 
                                                                   const int32_t* __restrict__ expert_idx, int B,
                                                                   int N_H, int E, int H, float inv_nh,
                                                                   float* __restrict__ out) {
+    griddep_wait();  // every global access below comes after the previous grid
     __shared__ uint32_t s_mask[kGBM][32];  // [row][e], bit h: horizon token h (N_H <= 32) chose expert e
     __shared__ __align__(16) float sA[kGBK][kGBM + 4];    // X_be^T: [k][row]
     __shared__ __align__(16) float sB[kGBK][kGBN + 4];    // [k][n]
@@ -259,6 +261,7 @@ __global__ void __launch_bounds__(kWThreads) wgrad_ffma_kernel(const float* __re
                                                               const int32_t* __restrict__ perm, int64_t T, int E,
                                                               int H, int P, int g_div, float* __restrict__ part,
                                                               float* __restrict__ part_db) {
+    griddep_wait();  // every global access below comes after the previous grid
     __shared__ __align__(16) float sG[kWChunk][kWT];  // d_out rows
     __shared__ __align__(16) float sX[kWChunk][kWT];  // x rows
     __shared__ int s_tok[kWChunk];
@@ -387,6 +390,7 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
                                                           const int32_t* __restrict__ offsets, int64_t T, int E,
                                                           int H, int P, float scale, float* __restrict__ dW,
                                                           float* __restrict__ db, int acc_dw, int acc_db) {
+    griddep_wait();  // every global access below comes after the previous grid
     __shared__ int s_c[2];
     const int e = blockIdx.y;
     // the ranges c that overlap expert e's tokens [a, b) are contiguous: thread c
@@ -445,8 +449,8 @@ cudaError_t launch_grouped_ffma(const float* src, const float* Wsrc, const float
                                 int src_div, float out_scale, float* out, cudaStream_t s) {
     const int64_t tiles = (T + kGBM - 1) / kGBM + E;  // upper bound; extra CTAs exit
     dim3 grid(static_cast<unsigned>(tiles), H / kGBN);
-    grouped_ffma_kernel<<<grid, kGThreads, 0, s>>>(src, Wsrc, bias, offsets, perm, E, H, b_kmajor, accumulate,
-                                                   src_div, out_scale, out);
+    launch_pdl(grouped_ffma_kernel, dim3(grid), dim3(kGThreads), 0, s,
+               src, Wsrc, bias, offsets, perm, E, H, b_kmajor, accumulate, src_div, out_scale, out);
     return cudaGetLastError();
 }
 
@@ -454,8 +458,8 @@ cudaError_t launch_hmean_fwd_ffma(const float* x, const float* W, const float* b
                                   int64_t B, int N_H, int E, int H, float* out, cudaStream_t s) {
     const dim3 grid(static_cast<unsigned>((B + kGBM - 1) / kGBM), static_cast<unsigned>(H / kGBN));
     const float inv_nh = static_cast<float>(1.0 / static_cast<double>(N_H));
-    hmean_fwd_ffma_kernel<<<grid, kGThreads, 0, s>>>(x, W, bias, expert_idx, static_cast<int>(B), N_H, E, H, inv_nh,
-                                                     out);
+    launch_pdl(hmean_fwd_ffma_kernel, dim3(grid), dim3(kGThreads), 0, s,
+               x, W, bias, expert_idx, static_cast<int>(B), N_H, E, H, inv_nh, out);
     return cudaGetLastError();
 }
 
@@ -463,7 +467,8 @@ cudaError_t launch_wgrad_ffma(const float* x, const float* d_out, const int32_t*
                               int64_t T, int E, int H, int g_div, float* part, float* part_db, cudaStream_t s) {
     const int P = wgrad_splits(T);
     dim3 grid(P, H / kWT, H / kWT);
-    wgrad_ffma_kernel<<<grid, kWThreads, 0, s>>>(x, d_out, offsets, perm, T, E, H, P, g_div, part, part_db);
+    launch_pdl(wgrad_ffma_kernel, dim3(grid), dim3(kWThreads), 0, s,
+               x, d_out, offsets, perm, T, E, H, P, g_div, part, part_db);
     return cudaGetLastError();
 }
 
@@ -473,7 +478,8 @@ cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const i
     const int64_t HH = static_cast<int64_t>(H) * H;
     const int nb_w = static_cast<int>((HH / 4 + 255) / 256);
     dim3 grid(nb_w + 1, E);
-    wgrad_reduce_kernel<<<grid, 256, 0, s>>>(part, part_db, offsets, T, E, H, P, scale, dW, db, acc_dw, acc_db);
+    launch_pdl(wgrad_reduce_kernel, dim3(grid), dim3(256), 0, s,
+               part, part_db, offsets, T, E, H, P, scale, dW, db, acc_dw, acc_db);
     return cudaGetLastError();
 }
 

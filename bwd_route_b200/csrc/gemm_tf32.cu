@@ -154,12 +154,13 @@ grouped_tf32_kernel(const float* __restrict__ src, const __grid_constant__ CUten
         ctl->abort = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
     if (warp == kGBLoadWarp && lane == 0) tma_prefetch_desc(&tm_b);
     if (warp == kGMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
+    griddep_wait();  // the prologue above overlaps the previous kernel; global memory from here on
+    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
     __syncthreads();
     if (threadIdx.x == 0) {
         int ts = 0;
@@ -441,11 +442,12 @@ wgrad_tf32_kernel(const float* __restrict__ g_src, const float* __restrict__ x_s
         ctl->abort = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
     if (warp == kMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
+    griddep_wait();  // the prologue above overlaps the previous kernel; global memory from here on
+    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -633,11 +635,11 @@ cudaError_t launch_grouped_tf32_t(const float* src, const CUtensorMap& tm_b, con
                                   const int32_t* offsets, const int32_t* perm, int E, int accumulate, int src_div,
                                   float out_scale, float* out, uint32_t* dev_flags, int grid, cudaStream_t s) {
     if (src_div != 1 || out_scale != 1.0f)
-        grouped_tf32_kernel<H, B_MN, true><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(
-            src, tm_b, bias, offsets, perm, E, accumulate, src_div, out_scale, out, dev_flags);
+        launch_pdl(grouped_tf32_kernel<H, B_MN, true>, dim3(grid), dim3(kThreadsGrouped), GCfg<H>::SMEM_BYTES, s,
+                   src, tm_b, bias, offsets, perm, E, accumulate, src_div, out_scale, out, dev_flags);
     else
-        grouped_tf32_kernel<H, B_MN, false><<<grid, kThreadsGrouped, GCfg<H>::SMEM_BYTES, s>>>(
-            src, tm_b, bias, offsets, perm, E, accumulate, 1, 1.0f, out, dev_flags);
+        launch_pdl(grouped_tf32_kernel<H, B_MN, false>, dim3(grid), dim3(kThreadsGrouped), GCfg<H>::SMEM_BYTES, s,
+                   src, tm_b, bias, offsets, perm, E, accumulate, 1, 1.0f, out, dev_flags);
     return cudaGetLastError();
 }
 
@@ -667,13 +669,11 @@ cudaError_t launch_wgrad_tf32(const float* x, const float* d_out, const int32_t*
                               cudaStream_t s) {
     const int P = wgrad_splits(T);
     if (H == 256) {
-        wgrad_tf32_kernel<256><<<P, kThreads, WCfg<256>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
-                                                                         static_cast<int>(T), E, P, g_div, part, part_db,
-                                                                         dev_flags);
+        launch_pdl(wgrad_tf32_kernel<256>, dim3(P), dim3(kThreads), WCfg<256>::SMEM_BYTES, s,
+                   d_out, x, offsets, perm, static_cast<int>(T), E, P, g_div, part, part_db, dev_flags);
     } else {
-        wgrad_tf32_kernel<128><<<P, kThreads, WCfg<128>::SMEM_BYTES, s>>>(d_out, x, offsets, perm,
-                                                                         static_cast<int>(T), E, P, g_div, part, part_db,
-                                                                         dev_flags);
+        launch_pdl(wgrad_tf32_kernel<128>, dim3(P), dim3(kThreads), WCfg<128>::SMEM_BYTES, s,
+                   d_out, x, offsets, perm, static_cast<int>(T), E, P, g_div, part, part_db, dev_flags);
     }
     return cudaGetLastError();
 }

@@ -186,7 +186,6 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
         ctl->abort = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
     if (warp == kWLoadWarp && lane == 0) tma_prefetch_desc(tm_w);
     if (warp == kMmaWarp) {
         if (PAIR) {
@@ -197,6 +196,8 @@ __device__ __forceinline__ void bwd_fused_body(const float* __restrict__ x, cons
             tmem_relinquish();
         }
     }
+    griddep_wait();  // the prologue above overlaps the previous kernel; global memory from here on
+    if (threadIdx.x <= E) ctl->off[threadIdx.x] = offsets[threadIdx.x];
     tc_fence_before();
     if (PAIR)
         cluster_sync_all();  // barriers initialised in both CTAs before any remote arrival
@@ -652,20 +653,18 @@ cudaError_t launch_bwd_fused_tf32(const float* x, const float* W, const float* g
     const int Ti = static_cast<int>(T);
     if (H == 256) {
         if (collapse)
-            bwd_fused_pair_kernel<true><<<2 * P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, g_div,
-                                                                          out_scale, acc_dx, d_x, part, part_db,
-                                                                          dev_flags);
+            launch_pdl(bwd_fused_pair_kernel<true>, dim3(2 * P), dim3(kThreads), kSmemBytes, s,
+                       x, g_src, tm_w, offsets, perm, Ti, E, P, g_div, out_scale, acc_dx, d_x, part, part_db, dev_flags);
         else
-            bwd_fused_pair_kernel<false><<<2 * P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, 1,
-                                                                           1.0f, acc_dx, d_x, part, part_db, dev_flags);
+            launch_pdl(bwd_fused_pair_kernel<false>, dim3(2 * P), dim3(kThreads), kSmemBytes, s,
+                       x, g_src, tm_w, offsets, perm, Ti, E, P, 1, 1.0f, acc_dx, d_x, part, part_db, dev_flags);
     } else {
         if (collapse)
-            bwd_fused_single_kernel<true><<<P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, g_div,
-                                                                        out_scale, acc_dx, d_x, part, part_db,
-                                                                        dev_flags);
+            launch_pdl(bwd_fused_single_kernel<true>, dim3(P), dim3(kThreads), kSmemBytes, s,
+                       x, g_src, tm_w, offsets, perm, Ti, E, P, g_div, out_scale, acc_dx, d_x, part, part_db, dev_flags);
         else
-            bwd_fused_single_kernel<false><<<P, kThreads, kSmemBytes, s>>>(x, g_src, tm_w, offsets, perm, Ti, E, P, 1,
-                                                                         1.0f, acc_dx, d_x, part, part_db, dev_flags);
+            launch_pdl(bwd_fused_single_kernel<false>, dim3(P), dim3(kThreads), kSmemBytes, s,
+                       x, g_src, tm_w, offsets, perm, Ti, E, P, 1, 1.0f, acc_dx, d_x, part, part_db, dev_flags);
     }
     return cudaGetLastError();
 }

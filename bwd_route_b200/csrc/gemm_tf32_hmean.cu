@@ -103,13 +103,14 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
         ctl->abort = 0;
         fence_mbar_init();
     }
-    for (int k = threadIdx.x; k < E * H / 4; k += blockDim.x)
-        reinterpret_cast<float4*>(bias_s)[k] = __ldg(reinterpret_cast<const float4*>(bias) + k);
     if (warp == kHBLoadWarp && lane == 0) tma_prefetch_desc(&tm_b);
     if (warp == kHMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
+    griddep_wait();  // the prologue above overlaps the previous kernel; global memory from here on
+    for (int k = threadIdx.x; k < E * H / 4; k += blockDim.x)
+        reinterpret_cast<float4*>(bias_s)[k] = __ldg(reinterpret_cast<const float4*>(bias) + k);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -348,7 +349,7 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
     }
 }
 
-// ------------------------------------------------------------------ the same mean, raw rows staged by TMA (E <= 8)
+// ------------------------------------------------------------------ the same mean, raw rows staged by TMA (E <= 8, N_H <= 16)
 // Same result definition and the same arithmetic as hmean_fwd_tf32_kernel (X_be
 // summed in fp32 in ascending h; the MMA products of (e, k) added into TMEM;
 // then sum_e n_be bias[e] and the 1/N_H scale), organised so that memory
@@ -357,12 +358,20 @@ hmean_fwd_tf32_kernel(const float* __restrict__ x, const __grid_constant__ CUten
 // contiguous block of x), and reducer warps build X_be for all experts of one
 // 16-column k-chunk from them. Every CTA owns a contiguous range of batch rows
 // (B / grid each), walked in tiles of 128 rows, so no wave of tiles is left
-// half-empty.
-//   warps 0-3   epilogue: TMEM lane quadrant = warp, all H columns
-//   warps 4-11  reducers: raw stage (k-chunk kc, row group g) goes to warp g % 8
-//   warp 12     MMA issuer: per k-chunk, for each expert, 2 MMAs of K = 8 on
-//               X_be (64-byte swizzle, K-major) and the W[e] k-chunk
-//   warp 13     raw x stages by TMA (no swizzle: rows of 16 floats)
+// half-empty. The reducers write X_be into one shared-memory staging buffer
+// (64-byte swizzle, K-major); the MMA thread copies it into one of two
+// tensor-memory A buffers (tcgen05.cp) and releases the staging buffer as soon
+// as the copy is done, so the reducers build k-chunk kc + 1 while the MMAs of
+// k-chunk kc run from tensor memory.
+//   warps 0-3   epilogue: TMEM lane quadrant = warp, all H columns; they also
+//               build each tile's token lists (tokens of a row sorted by expert)
+//               one tile ahead, into two list buffers
+//   warps 4-11  reducers: raw stage q (launch-wide index) goes to warp q % 8
+//   warp 12     MMA issuer: per k-chunk, the copy of X_be into tensor memory,
+//               then for each expert 2 MMAs of K = 8 on X_be (A in tensor
+//               memory) and the W[e] k-chunk (shared memory)
+//   warp 13     raw x stages by TMA (rows of 16 floats, 64-byte swizzle, so that
+//               the eight rows a reducer warp reads at once fall in different banks)
 //   warp 14     W[e] k-chunks by TMA (64-byte swizzle)
 constexpr int kSThreads = 480;
 constexpr int kSEpiWarps = 4;
@@ -373,9 +382,10 @@ constexpr int kSRawWarp = 13;
 constexpr int kSWWarp = 14;
 constexpr int kSMaxE = 8;
 constexpr int kSRowsPerStage = 8;
-constexpr int kSGroups = 16;  // row groups per 128-row tile
+constexpr int kSMaxHorizon = 16;  // tokens per batch row on this path
 constexpr int kSRawMaxStages = 16;
-constexpr int kSBStages = 3;
+static_assert(kSRawMaxStages % 8 == 0, "raw slots come in multiples of the reducer warps");
+constexpr int kSBStages = 5;
 
 struct __align__(8) SCtl {
     uint64_t raw_full[kSRawMaxStages];
@@ -385,7 +395,7 @@ struct __align__(8) SCtl {
     uint64_t b_empty[kSBStages];
     uint64_t t_full[2];
     uint64_t t_empty[2];
-    uint64_t order_full, order_empty;
+    uint64_t ord_full[2], ord_empty[2];  // the two token-list buffers
     uint32_t tmem_base;
     int abort;
 };
@@ -397,10 +407,16 @@ struct SCfg {
     static constexpr int A_BYTES = BM * 64;                     // X_be of one expert and k-chunk: 8 KiB
     static constexpr int A_REGION = kSMaxE * A_BYTES;           // 64 KiB
     static constexpr int B_BYTES = H * 64;                      // W[e] k-chunk
-    static constexpr int RAW_BUDGET = 96 * 1024;
-    static constexpr int ORDER_BYTES = BM * kHMaxHorizon * 2;   // uint16 (h | e << 8) per row and slot
+    static constexpr int RAW_BUDGET = 64 * 1024;
+    static constexpr int ORDER_BYTES = 2 * BM * kSMaxHorizon * 2;  // two lists of uint16 (h | e << 8)
     static constexpr int BIAS_BYTES = kSMaxE * H * 4;
-    static constexpr int TMEM_COLS = 2 * H;
+    // tensor memory: D_BUFS accumulators of H columns, then two A buffers of
+    // kSMaxE x 16 columns (X_be of one k-chunk for every expert)
+    static constexpr int D_BUFS = H == 256 ? 1 : 2;
+    static constexpr int A_TCOLS = kSMaxE * 16;
+    static constexpr int A_TCOL0 = D_BUFS * H;
+    static constexpr int TMEM_COLS = 512;
+    static_assert(A_TCOL0 + 2 * A_TCOLS <= TMEM_COLS, "tensor memory");
     static constexpr int SMEM_BYTES = 1024 + A_REGION + kSBStages * B_BYTES + RAW_BUDGET + ORDER_BYTES + BIAS_BYTES +
                                       static_cast<int>(sizeof(SCtl));
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -438,7 +454,7 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
             mbar_init(&ctl->raw_full[s], 1);   // arrive.expect_tx + TMA bytes
             mbar_init(&ctl->raw_empty[s], 1);  // the reducer warp that read it
         }
-        mbar_init(&ctl->a_full, kSGroups);     // one arrival per row group of the k-chunk
+        mbar_init(&ctl->a_full, kSReducers);   // one arrival per reducer warp and k-chunk
         mbar_init(&ctl->a_empty, 1);           // tcgen05.commit
         for (int s = 0; s < kSBStages; ++s) {
             mbar_init(&ctl->b_full[s], 1);
@@ -448,19 +464,22 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
             mbar_init(&ctl->t_full[b], 1);
             mbar_init(&ctl->t_empty[b], kSEpiWarps);
         }
-        mbar_init(&ctl->order_full, kSReducers);
-        mbar_init(&ctl->order_empty, kSReducers);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->ord_full[b], kSEpiWarps);
+            mbar_init(&ctl->ord_empty[b], kSReducers);
+        }
         ctl->abort = 0;
         fence_mbar_init();
     }
-    for (int k = threadIdx.x; k < E * H / 4; k += blockDim.x)
-        reinterpret_cast<float4*>(bias_s)[k] = __ldg(reinterpret_cast<const float4*>(bias) + k);
     if (warp == kSRawWarp && lane == 0) tma_prefetch_desc(&tm_x);
     if (warp == kSWWarp && lane == 0) tma_prefetch_desc(&tm_w);
     if (warp == kSMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
+    griddep_wait();  // the prologue above overlaps the previous kernel; global memory from here on
+    for (int k = threadIdx.x; k < E * H / 4; k += blockDim.x)
+        reinterpret_cast<float4*>(bias_s)[k] = __ldg(reinterpret_cast<const float4*>(bias) + k);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -499,7 +518,8 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
         if (lane == 0) {
             int sb = 0;
             uint32_t pb = 0;
-            int issued[kSBStages] = {0, 0, 0};
+            int issued[kSBStages];
+            for (int k = 0; k < kSBStages; ++k) issued[k] = 0;
             bool ok = true;
             for (int tile = 0; tile < ntiles && ok; ++tile) {
                 for (int kc = 0; kc < C::KC && ok; ++kc) {
@@ -529,112 +549,79 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
             const int64_t b0 = b_lo + static_cast<int64_t>(tile) * C::BM;
             const int nrows = static_cast<int>(b_hi - b0 < C::BM ? b_hi - b0 : C::BM);
             const int ngroups = (nrows + kSRowsPerStage - 1) / kSRowsPerStage;
-            // the tile's tokens of each row, grouped by expert in ascending h: this
-            // warp builds rows 16 rw .. 16 rw + 15 once every warp is done with the
-            // previous tile's list
-            if (!(ok = mbar_wait(&ctl->order_empty, (tile & 1) ^ 1, abort, dev_flags))) break;
-            if (lane < 16) {
-                const int m = rw * 16 + lane;
-                uint16_t* ord = order + m * kHMaxHorizon;
-                const bool valid = m < nrows;
-                const int32_t* idx = expert_idx + (b0 + m) * N_H;
-                // all of the row's expert indices are requested before the first is used
-                int ek[kHMaxHorizon];  // expert of horizon token h, kSMaxE for none / out of range
-#pragma unroll
-                for (int h = 0; h < kHMaxHorizon; ++h) {
-                    const int e = (valid && h < N_H) ? idx[h] : -1;
-                    ek[h] = (e >= 0 && e < E) ? e : kSMaxE;
-                }
-                int cnt[kSMaxE + 1];
-#pragma unroll
-                for (int f = 0; f <= kSMaxE; ++f) cnt[f] = 0;
-#pragma unroll
-                for (int h = 0; h < kHMaxHorizon; ++h)
-#pragma unroll
-                    for (int f = 0; f <= kSMaxE; ++f) cnt[f] += (h < N_H && f == ek[h]) ? 1 : 0;
-                int pos[kSMaxE + 1];
-                int acc = 0;
-#pragma unroll
-                for (int f = 0; f <= kSMaxE; ++f) {
-                    pos[f] = acc;
-                    acc += cnt[f];
-                }
-#pragma unroll
-                for (int h = 0; h < kHMaxHorizon; ++h) {
-                    if (h >= N_H) break;
-                    int p = 0;
-#pragma unroll
-                    for (int f = 0; f <= kSMaxE; ++f)
-                        if (f == ek[h]) p = pos[f]++;
-                    ord[p] = static_cast<uint16_t>(h | ((ek[h] == kSMaxE ? 0xFF : ek[h]) << 8));
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->order_full);
-            if (!(ok = mbar_wait(&ctl->order_full, tile & 1, abort, dev_flags))) break;
+            // the tile's token lists (built by the epilogue warps a tile ahead)
+            if (!(ok = mbar_wait(&ctl->ord_full[tile & 1], static_cast<uint32_t>((tile >> 1) & 1), abort, dev_flags)))
+                break;
+            const uint32_t obuf = smem_u32(order + (tile & 1) * (C::BM * kSMaxHorizon));
             for (int kc = 0; kc < C::KC && ok; ++kc) {
-                // the MMAs of the previous k-chunk have read the X_be region
+                // the previous k-chunk's X_be has been copied out of the staging buffer
                 if (!(ok = mbar_wait(&ctl->a_empty, pa ^ 1, abort, dev_flags))) break;
+                // raw stage q (launch-wide index) is reduced by warp q % 8, and the ring has
+                // a multiple of 8 slots: every use of a slot has the same reducer warp, which
+                // waits for its uses in order, so its parity waits cannot alias a stage two
+                // uses back (as they could if a slot's uses went to different warps)
+                const int64_t qbase = qtile + static_cast<int64_t>(kc) * ngroups;
+                const int g0 = static_cast<int>((rw - qbase % kSReducers + kSReducers) % kSReducers);
 #pragma unroll 1
-                for (int g = rw; g < kSGroups; g += kSReducers) {
-                    if (g < ngroups) {
-                        const int64_t q = qtile + static_cast<int64_t>(kc) * ngroups + g;
-                        const int slot = static_cast<int>(q % raw_stages);
-                        if (!(ok = mbar_wait(&ctl->raw_full[slot], static_cast<uint32_t>((q / raw_stages) & 1), abort,
-                                             dev_flags)))
-                            break;
-                        const int m = g * kSRowsPerStage + r;
-                        const uint16_t* ord = order + m * kHMaxHorizon;
-                        const uint32_t rb = raw_u32 + slot * raw_bytes + r * N_H * 64 + q4 * 16;
-                        const uint32_t arow = a_u32 + m * 64 + ((q4 ^ ((m >> 1) & 3)) << 4);
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                        int cur = -1;
-                        uint32_t present = 0;
-                        // eight tokens at a time: their list entries (one 16-byte load) and
-                        // their rows are requested together, then added in list order
-                        for (int j0 = 0; j0 < N_H; j0 += 8) {
-                            const uint4 o4 = *reinterpret_cast<const uint4*>(ord + j0);
-                            uint32_t o[8] = {o4.x & 0xFFFFu, o4.x >> 16, o4.y & 0xFFFFu, o4.y >> 16,
-                                             o4.z & 0xFFFFu, o4.z >> 16, o4.w & 0xFFFFu, o4.w >> 16};
+                for (int g = g0; g < ngroups; g += kSReducers) {
+                    const int64_t q = qbase + g;
+                    const int slot = static_cast<int>(q % raw_stages);
+                    const int m = g * kSRowsPerStage + r;
+                    // the row's list: 16 entries (h | e << 8), sorted by expert, ascending h
+                    // within one; entries of no expert (e = 0xFF) come last
+                    const uint4 oa = ld_shared_u4(obuf + m * (kSMaxHorizon * 2));
+                    const uint4 ob = ld_shared_u4(obuf + m * (kSMaxHorizon * 2) + 16);
+                    const uint32_t o[16] = {oa.x & 0xFFFFu, oa.x >> 16, oa.y & 0xFFFFu, oa.y >> 16,
+                                            oa.z & 0xFFFFu, oa.z >> 16, oa.w & 0xFFFFu, oa.w >> 16,
+                                            ob.x & 0xFFFFu, ob.x >> 16, ob.y & 0xFFFFu, ob.y >> 16,
+                                            ob.z & 0xFFFFu, ob.z >> 16, ob.w & 0xFFFFu, ob.w >> 16};
+                    if (!(ok = mbar_wait(&ctl->raw_full[slot], static_cast<uint32_t>((q / raw_stages) & 1), abort,
+                                         dev_flags)))
+                        break;
+                    // token row rr = r N_H + h of the stage holds 16 floats, stored with the
+                    // 64-byte swizzle: 16-byte granule q4 sits at granule q4 ^ ((rr >> 1) & 3)
+                    const uint32_t sbase = raw_u32 + slot * raw_bytes;
+                    float4 vv[16];  // every listed row is requested before the first add
 #pragma unroll
-                            for (int u = 0; u < 8; ++u)
-                                if (j0 + u >= N_H) o[u] = 0xFF00u;  // past the row's tokens: no expert
-                            float4 vv[8];
-#pragma unroll
-                            for (int u = 0; u < 8; ++u)
-                                vv[u] = (static_cast<int>(o[u] >> 8) < E) ? ld_shared_v4(rb + (o[u] & 0xFFu) * 64)
-                                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int e = static_cast<int>(o[u] >> 8);
-                                if (e >= E) continue;  // out-of-range experts sort last and add nothing
-                                if (e != cur) {
-                                    if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
-                                    acc = vv[u];
-                                    cur = e;
-                                    present |= 1u << e;
-                                } else {
-                                    acc.x += vv[u].x;
-                                    acc.y += vv[u].y;
-                                    acc.z += vv[u].z;
-                                    acc.w += vv[u].w;
-                                }
-                            }
-                        }
-                        if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
-                        for (int e = 0; e < E; ++e)
-                            if (!((present >> e) & 1u)) st_shared_v4(arow + e * C::A_BYTES, 0.f, 0.f, 0.f, 0.f);
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&ctl->raw_empty[slot]);
+                    for (int u = 0; u < 16; ++u) {
+                        const int rr = r * N_H + static_cast<int>(o[u] & 0xFFu);
+                        vv[u] = (static_cast<int>(o[u] >> 8) < E)
+                                    ? ld_shared_v4(sbase + rr * 64 + ((q4 ^ ((rr >> 1) & 3)) << 4))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
-                    fence_proxy_async_smem();  // the MMA reads these stores through the async proxy
+                    const uint32_t arow = a_u32 + m * 64 + ((q4 ^ ((m >> 1) & 3)) << 4);
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    int cur = -1;
+                    uint32_t present = 0;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int e = static_cast<int>(o[u] >> 8);
+                        if (e >= E) continue;  // no expert (past the row's tokens, or out of range)
+                        if (e != cur) {
+                            if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
+                            acc = vv[u];
+                            cur = e;
+                            present |= 1u << e;
+                        } else {
+                            acc.x += vv[u].x;
+                            acc.y += vv[u].y;
+                            acc.z += vv[u].z;
+                            acc.w += vv[u].w;
+                        }
+                    }
+                    if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
+                    for (int e = 0; e < E; ++e)
+                        if (!((present >> e) & 1u)) st_shared_v4(arow + e * C::A_BYTES, 0.f, 0.f, 0.f, 0.f);
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->a_full);
+                    if (lane == 0) mbar_arrive(&ctl->raw_empty[slot]);
                 }
+                fence_proxy_async_smem();  // the copy to tensor memory reads these stores through the async proxy
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->a_full);  // once per warp and k-chunk
                 pa ^= 1;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->order_empty);
+            if (lane == 0) mbar_arrive(&ctl->ord_empty[tile & 1]);
             qtile += static_cast<int64_t>(C::KC) * ngroups;
         }
     } else if (warp == kSMmaWarp) {
@@ -646,61 +633,111 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
             uint32_t pb = 0, pa = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
+            int abuf = 0;  // tensor-memory A buffer of the next k-chunk
             bool ok = true;
             for (int tile = 0; tile < ntiles && ok; ++tile) {
-                if (!(ok = mbar_wait(&ctl->t_empty[acc], acc_phase ^ 1, abort, dev_flags))) break;
-                tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * H);
                 uint32_t accumulate = 0;
                 for (int kc = 0; kc < C::KC && ok; ++kc) {
                     if (!(ok = mbar_wait(&ctl->a_full, pa, abort, dev_flags))) break;
                     fence_proxy_async_smem();
                     tc_fence_after();
+                    // X_be of this k-chunk -> A buffer abuf. The buffer was last read by the
+                    // MMAs of k-chunk kc - 2, which completed before the staging buffer was
+                    // released for k-chunk kc (the commit below covers every earlier op).
+                    const uint32_t a_t = tmem + static_cast<uint32_t>(C::A_TCOL0 + abuf * C::A_TCOLS);
+                    for (int e = 0; e < E; ++e)
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks)
+                            tmem_cp_128x256b(a_t + static_cast<uint32_t>(e * 16 + ks * 8),
+                                             sw64_desc(a_u32 + e * C::A_BYTES + ks * 32, 512));
+                    mma_commit(&ctl->a_empty);  // the staging buffer is free once the copies are done
+                    pa ^= 1;
+                    if (kc == 0) {
+                        // the accumulator must have been read out by the epilogue
+                        if (!(ok = mbar_wait(&ctl->t_empty[acc], acc_phase ^ 1, abort, dev_flags))) break;
+                        tc_fence_after();
+                    }
                     for (int e = 0; e < E; ++e) {
                         if (!(ok = mbar_wait(&ctl->b_full[sb], pb, abort, dev_flags))) break;
                         tc_fence_after();
                         const uint32_t b_addr = smem_u32(bring + sb * C::B_BYTES);
 #pragma unroll
                         for (int ks = 0; ks < 2; ++ks) {
-                            mma_tf32(d, sw64_desc(a_u32 + e * C::A_BYTES + ks * 32, 512), sw64_desc(b_addr + ks * 32, 512),
-                                     idesc, accumulate);
+                            mma_tf32_ts(d, a_t + static_cast<uint32_t>(e * 16 + ks * 8), sw64_desc(b_addr + ks * 32, 512),
+                                        idesc, accumulate);
                             accumulate = 1u;
                         }
                         mma_commit(&ctl->b_empty[sb]);
                         advance_stage(sb, pb, kSBStages);
                     }
-                    if (!ok) break;
-                    mma_commit(&ctl->a_empty);
-                    pa ^= 1;
+                    abuf ^= 1;
                 }
                 if (!ok) break;
                 mma_commit(&ctl->t_full[acc]);
-                acc ^= 1;
+                if (C::D_BUFS > 1) acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
         }
         __syncwarp();
     } else if (warp < kSEpiWarps) {
         // ---------------- epilogue: row m = 32 q + lane of the tile, all H columns;
-        // (acc + sum_e n_be bias[e]) / N_H with n_be counted from the row's experts
+        // (acc + sum_e n_be bias[e]) / N_H with n_be counted from the row's experts.
+        // These warps also build the reducers' token lists, one tile ahead.
         const int q = warp;
+        const int m = 32 * q + lane;  // this thread's row of every tile
+        // Tile t's list for row m into order buffer t & 1: 16 entries (h | e << 8)
+        // sorted by expert, ascending h within one, entries of no expert (past N_H,
+        // or an index outside [0, E)) last; and the row's token count per expert.
+        auto build = [&](int t, int (&cnt)[kSMaxE]) -> bool {
+            const bool ok = mbar_wait(&ctl->ord_empty[t & 1], static_cast<uint32_t>(((t >> 1) & 1) ^ 1), abort,
+                                      dev_flags);
+            if (!__all_sync(0xffffffffu, ok)) return false;
+            const int64_t b = b_lo + static_cast<int64_t>(t) * C::BM + m;
+            const bool valid = b < b_hi;
+            int ek[kSMaxHorizon];  // requested together, then sorted
+#pragma unroll
+            for (int h = 0; h < kSMaxHorizon; ++h) {
+                const int e = (valid && h < N_H) ? expert_idx[b * N_H + h] : -1;
+                ek[h] = (e >= 0 && e < E) ? e : kSMaxE;
+            }
+            int pos[kSMaxE + 1];
+#pragma unroll
+            for (int f = 0; f <= kSMaxE; ++f) pos[f] = 0;
+#pragma unroll
+            for (int h = 0; h < kSMaxHorizon; ++h)
+#pragma unroll
+                for (int f = 0; f <= kSMaxE; ++f) pos[f] += (f == ek[h]) ? 1 : 0;
+#pragma unroll
+            for (int f = 0; f < kSMaxE; ++f) cnt[f] = pos[f];
+            int run = 0;
+#pragma unroll
+            for (int f = 0; f <= kSMaxE; ++f) {
+                const int c = pos[f];
+                pos[f] = run;
+                run += c;
+            }
+            uint16_t* ord = order + (t & 1) * (C::BM * kSMaxHorizon) + m * kSMaxHorizon;
+#pragma unroll
+            for (int h = 0; h < kSMaxHorizon; ++h) {
+                int p = 0;
+#pragma unroll
+                for (int f = 0; f <= kSMaxE; ++f)
+                    if (f == ek[h]) p = pos[f]++;
+                ord[p] = static_cast<uint16_t>(h | ((ek[h] == kSMaxE ? 0xFF : ek[h]) << 8));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->ord_full[t & 1]);
+            return true;
+        };
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = 0; tile < ntiles; ++tile) {
-            const int64_t b = b_lo + static_cast<int64_t>(tile) * C::BM + 32 * q + lane;
+        int cnt[kSMaxE], cnt_next[kSMaxE];
+        bool eok = build(0, cnt);
+        for (int tile = 0; tile < ntiles && eok; ++tile) {
+            if (tile + 1 < ntiles && !(eok = build(tile + 1, cnt_next))) break;
+            const int64_t b = b_lo + static_cast<int64_t>(tile) * C::BM + m;
             const bool valid = b < b_hi;
-            int cnt[kSMaxE];
-#pragma unroll
-            for (int e = 0; e < kSMaxE; ++e) cnt[e] = 0;
-            {
-                int ev[kHMaxHorizon];  // requested together, then counted
-#pragma unroll
-                for (int h = 0; h < kHMaxHorizon; ++h) ev[h] = (valid && h < N_H) ? expert_idx[b * N_H + h] : -1;
-#pragma unroll
-                for (int h = 0; h < kHMaxHorizon; ++h)
-#pragma unroll
-                    for (int f = 0; f < kSMaxE; ++f) cnt[f] += (f == ev[h]) ? 1 : 0;
-            }
             const bool ok = mbar_wait(&ctl->t_full[acc], acc_phase, abort, dev_flags);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
@@ -735,8 +772,10 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->t_empty[acc]);
-            acc ^= 1;
+            if (C::D_BUFS > 1) acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
+#pragma unroll
+            for (int f = 0; f < kSMaxE; ++f) cnt[f] = cnt_next[f];
         }
     }
     tc_fence_before();
@@ -757,24 +796,25 @@ cudaError_t set_smem(K kernel, int bytes) {
 cudaError_t launch_hmean_fwd_tf32(const float* x, const float* W, const float* bias, const int32_t* expert_idx,
                                   int64_t B, int N_H, int E, int H, float* out, uint32_t* dev_flags, int num_sms,
                                   cudaStream_t s) {
-    if (E <= kSMaxE) {
+    const int raw_bytes = kSRowsPerStage * N_H * 64;
+    int raw_stages = SCfg<256>::RAW_BUDGET / raw_bytes;
+    if (raw_stages > kSRawMaxStages) raw_stages = kSRawMaxStages;
+    raw_stages -= raw_stages % kSReducers;  // a multiple of the reducer warps (N_H <= 16: at least 8)
+    if (E <= kSMaxE && N_H <= kSMaxHorizon && raw_stages >= kSReducers) {
         // raw rows staged by TMA; every CTA owns B / grid batch rows
         CUtensorMap tm_x, tm_w;
         const uint64_t T = static_cast<uint64_t>(B) * N_H;
-        if (!make_map_2d(&tm_x, x, T, H, 16, static_cast<uint32_t>(kSRowsPerStage * N_H), kMapPlain) ||
+        if (!make_map_2d(&tm_x, x, T, H, 16, static_cast<uint32_t>(kSRowsPerStage * N_H), kMapSw64) ||
             !make_map_2d(&tm_w, W, static_cast<uint64_t>(E) * H, H, 16, H, kMapSw64))
             return cudaErrorInvalidValue;
-        const int raw_bytes = kSRowsPerStage * N_H * 64;
-        int raw_stages = SCfg<256>::RAW_BUDGET / raw_bytes;
-        if (raw_stages > kSRawMaxStages) raw_stages = kSRawMaxStages;
         const int grid = static_cast<int>(B < num_sms ? B : num_sms);
         const float inv_nh = static_cast<float>(1.0 / static_cast<double>(N_H));
         if (H == 256)
-            hmean_fwd_tf32_sum_kernel<256><<<grid, kSThreads, SCfg<256>::SMEM_BYTES, s>>>(
-                tm_x, tm_w, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, raw_stages, out, dev_flags);
+            launch_pdl(hmean_fwd_tf32_sum_kernel<256>, dim3(grid), dim3(kSThreads), SCfg<256>::SMEM_BYTES, s,
+                       tm_x, tm_w, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, raw_stages, out, dev_flags);
         else
-            hmean_fwd_tf32_sum_kernel<128><<<grid, kSThreads, SCfg<128>::SMEM_BYTES, s>>>(
-                tm_x, tm_w, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, raw_stages, out, dev_flags);
+            launch_pdl(hmean_fwd_tf32_sum_kernel<128>, dim3(grid), dim3(kSThreads), SCfg<128>::SMEM_BYTES, s,
+                       tm_x, tm_w, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, raw_stages, out, dev_flags);
         return cudaGetLastError();
     }
     CUtensorMap tm_b;
@@ -783,11 +823,11 @@ cudaError_t launch_hmean_fwd_tf32(const float* x, const float* W, const float* b
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     const float inv_nh = static_cast<float>(1.0 / static_cast<double>(N_H));
     if (H == 256)
-        hmean_fwd_tf32_kernel<256><<<grid, kThreadsHmean, HCfg<256>::SMEM_BYTES, s>>>(
-            x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
+        launch_pdl(hmean_fwd_tf32_kernel<256>, dim3(grid), dim3(kThreadsHmean), HCfg<256>::SMEM_BYTES, s,
+                   x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
     else
-        hmean_fwd_tf32_kernel<128><<<grid, kThreadsHmean, HCfg<128>::SMEM_BYTES, s>>>(
-            x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
+        launch_pdl(hmean_fwd_tf32_kernel<128>, dim3(grid), dim3(kThreadsHmean), HCfg<128>::SMEM_BYTES, s,
+                   x, tm_b, bias, expert_idx, static_cast<int>(B), N_H, E, inv_nh, out, dev_flags);
     return cudaGetLastError();
 }
 

@@ -154,6 +154,27 @@ enum MapLayout : int {
 // 2D fp32 tensor [rows][cols] with a box of box_cols x box_rows in the given
 // layout. make_map_2d returns a cached copy when the same map was encoded before
 // on this device; encode_map_2d always encodes.
+// Every library kernel is launched with programmatic stream serialization: it may
+// be scheduled while the kernel before it in the stream is still tearing down, runs
+// its prologue (barrier init, tensor-memory allocation, tensor-map prefetch), and
+// waits (griddep_wait in common.cuh: all of the previous grid complete and its
+// memory visible) before its first global-memory access. After a kernel that is
+// not the library's it behaves like a plain launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 bool make_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                  uint32_t box_rows, int layout = kMapSw128);
 bool encode_map_2d(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols, uint32_t box_cols,

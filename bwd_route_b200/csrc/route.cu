@@ -38,6 +38,7 @@ template <int LPT>  // lanes per token: a power of two >= E
 __global__ void __launch_bounds__(kThreads) route_count_kernel(const float* __restrict__ logits, int64_t T, int E,
                                                               int32_t* __restrict__ expert_idx,
                                                               int32_t* __restrict__ blk_counts) {
+    griddep_wait();  // every global access below comes after the previous grid
     __shared__ int s_idx[kRouteTokPerBlk];
     __shared__ int s_wcnt[kWarps][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,6 +108,7 @@ template <int E>
 __global__ void __launch_bounds__(kThreads, 8) route_count_vec_kernel(const float* __restrict__ logits, int64_t T,
                                                                   int32_t* __restrict__ expert_idx,
                                                                   int32_t* __restrict__ blk_counts) {
+    griddep_wait();  // every global access below comes after the previous grid
     constexpr int Q = E / 4;                               // float4s per row
     constexpr int TOK = (Q == 1) ? 4 : (Q == 2 ? 2 : 1);   // tokens in flight per thread
     constexpr int PER = kRouteTokPerBlk / kThreads;         // 4 tokens per thread
@@ -161,6 +163,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
                                                          int E, int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ blk_base) {
+    griddep_wait();  // every global access below comes after the previous grid
     // Each expert gets Q = 32 / E warps; warp q of expert e owns a contiguous
     // run of routing blocks. Pass 1 sums each run, one thread turns the run sums
     // into the expert totals, the offsets and each run's starting base, and pass
@@ -242,6 +245,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
 __global__ void __launch_bounds__(kThreads) route_scatter_kernel(const int32_t* __restrict__ expert_idx, int64_t T,
                                                                 int E, const int32_t* __restrict__ blk_base,
                                                                 int32_t* __restrict__ perm) {
+    griddep_wait();  // every global access below comes after the previous grid
     // s_pos[w][e]: first the number of warp w's tokens on expert e, then warp w's
     // next free position in expert e's segment. Lanes holding the same expert are
     // grouped with __match_any_sync: a token's rank is the number of lower lanes
@@ -305,6 +309,7 @@ __global__ void __launch_bounds__(kThreads) route_scatter_prefix_kernel(const in
                                                                        int32_t* __restrict__ counts,
                                                                        int32_t* __restrict__ offsets,
                                                                        int32_t* __restrict__ perm) {
+    griddep_wait();  // every global access below comes after the previous grid
     __shared__ int s_before[32], s_total[32], s_base[32];
     __shared__ int s_pos[kWarps][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -392,30 +397,40 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
                          cudaStream_t s) {
     const int64_t nblk = (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk;
     if (E == 4)
-        route_count_vec_kernel<4><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+        launch_pdl(route_count_vec_kernel<4>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, expert_idx, blk_counts);
     else if (E == 8)
-        route_count_vec_kernel<8><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+        launch_pdl(route_count_vec_kernel<8>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, expert_idx, blk_counts);
     else if (E == 16)
-        route_count_vec_kernel<16><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+        launch_pdl(route_count_vec_kernel<16>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, expert_idx, blk_counts);
     else if (E == 32)
-        route_count_vec_kernel<32><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, expert_idx, blk_counts);
+        launch_pdl(route_count_vec_kernel<32>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, expert_idx, blk_counts);
     else if (E <= 4)
-        route_count_kernel<4><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        launch_pdl(route_count_kernel<4>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, E, expert_idx, blk_counts);
     else if (E <= 8)
-        route_count_kernel<8><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        launch_pdl(route_count_kernel<8>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, E, expert_idx, blk_counts);
     else if (E <= 16)
-        route_count_kernel<16><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        launch_pdl(route_count_kernel<16>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, E, expert_idx, blk_counts);
     else
-        route_count_kernel<32><<<(unsigned)nblk, kThreads, 0, s>>>(logits, T, E, expert_idx, blk_counts);
+        launch_pdl(route_count_kernel<32>, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   logits, T, E, expert_idx, blk_counts);
     if (nblk * E <= kPrefixMaxEntries) {
         int ep = 1;
         while (ep < E) ep <<= 1;
-        route_scatter_prefix_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(expert_idx, T, E, ep, nblk, blk_counts, counts,
-                                                                        offsets, perm);
+        launch_pdl(route_scatter_prefix_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+                   expert_idx, T, E, ep, nblk, blk_counts, counts, offsets, perm);
         return cudaGetLastError();
     }
-    route_scan_kernel<<<1, 1024, 0, s>>>(blk_counts, nblk, E, counts, offsets, blk_base);
-    route_scatter_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(expert_idx, T, E, blk_base, perm);
+    launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, s,
+               blk_counts, nblk, E, counts, offsets, blk_base);
+    launch_pdl(route_scatter_kernel, dim3((unsigned)nblk), dim3(kThreads), 0, s,
+               expert_idx, T, E, blk_base, perm);
     return cudaGetLastError();
 }
 

@@ -19,6 +19,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_top
 MOE_MATH_TF32 = 0
 MOE_MATH_FFMA = 1
 MOE_ACC_DX, MOE_ACC_DW, MOE_ACC_DB = 0x1, 0x2, 0x4
+MOE_BWD_SINGLE_PASS = 0x100  # one pass over d_out for d_x, dW and db (TF32)
 MOE_FLAG_WAIT_TIMEOUT = 0x1
 MOE_FLAG_BAD_ROUTING = 0x2
 

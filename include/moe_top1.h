@@ -58,8 +58,11 @@ extern "C" {
  *    version-1 call is unchanged).
  * 3: adds moe_top1_fwd_mean_collapse (every earlier call is unchanged).
  * 4: adds moe_top1_check_routing and MOE_FLAG_BAD_ROUTING (every earlier call is
- *    unchanged). */
-#define MOE_TOP1_ABI_VERSION 4
+ *    unchanged).
+ * 5: adds the MOE_BWD_SINGLE_PASS flag of the backward calls; moe_top1_bwd with
+ *    TF32 and every output requested takes two contraction passes by default
+ *    (results within fp32 rounding of version 4's single pass). */
+#define MOE_TOP1_ABI_VERSION 5
 
 typedef enum {
     MOE_OK = 0,
@@ -212,6 +215,17 @@ moe_status_t moe_top1_fwd_mean_collapse(const float* x, const float* W, const fl
 #define MOE_ACC_DX 0x1u
 #define MOE_ACC_DW 0x2u
 #define MOE_ACC_DB 0x4u
+/* Strategy bit of the same argument. With MOE_MATH_TF32 and d_x and dW (or db)
+ * requested, the backward runs either two contraction passes (d_x; then dW and
+ * db) or a single pass that computes all three from one read of d_out (or
+ * grad_ctx_mean) and x ([P1] kernel list: one backward produces d_fused_ctx and
+ * dW / db). The single pass moves about a third less DRAM traffic, but on a B200
+ * the two passes take less time for the per-token gradient, so moe_top1_bwd uses
+ * them by default; moe_top1_bwd_mean_collapse uses the single pass at H = 256,
+ * where it is the faster. This bit requests the single pass in both calls. The
+ * two strategies add the dW / db partial sums in different fixed orders: each is
+ * bitwise reproducible, and they agree to fp32 rounding. Ignored for FFMA. */
+#define MOE_BWD_SINGLE_PASS 0x100u
 
 /*
  * Backward (straight-through). [P1] kernel list (gradients flow only through

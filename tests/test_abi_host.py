@@ -53,7 +53,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_top1_abi_version() == 4
+    assert L.moe_top1_abi_version() == 5
     for s, name in enumerate(ops._STATUS):
         assert L.moe_status_string(s).decode() == name
     assert L.moe_status_string(99).decode() == "MOE_ERR_UNKNOWN"
@@ -114,6 +114,9 @@ def test_fwd_bwd_reject_bad_arguments_before_launch(L):
     g = L.moe_top1_bwd
     dx, dW, db = _p(A + 0x5000000), _p(A + 0x6000000), _p(A + 0x7000000)
     assert g(x, W, x, ctypes.byref(r), 8, 5, 4, 128, tf32, dx, dW, db, 0x8, ws, wsb, None) == INVALID
+    assert g(x, W, x, ctypes.byref(r), 8, 5, 4, 128, tf32, dx, dW, db, 0x200, ws, wsb, None) == INVALID
+    # the single-pass bit is a known flag: the call gets past argument checks to the aliasing check
+    assert g(x, W, x, ctypes.byref(r), 8, 5, 4, 128, tf32, dx, dx, db, 0x100, ws, wsb, None) == ALIAS
     assert g(x, W, x, ctypes.byref(r), 8, 5, 4, 128, tf32, dx, dx, db, 0, ws, wsb, None) == ALIAS  # dW on d_x
     assert g(x, W, x, ctypes.byref(r), 8, 5, 4, 128, tf32, x, dW, db, 0, ws, wsb, None) == ALIAS   # d_x on x
     assert g(x, W, x, ctypes.byref(r), 8, 5, 4, 128, tf32, dx, dW, db, 0, ws, 4096, None) == WORKSPACE

@@ -54,9 +54,9 @@ def lam_of(inp):
                                               inp.ent_target)))
 
 
-def check_all(inp, math, full=True):
+def check_all(inp, math, full=True, acc_flags=0):
     lam = lam_of(inp)
-    g = run_gpu(inp, math, lam)
+    g = run_gpu(inp, math, lam, acc_flags=acc_flags)
     assert g["flags"] == 0
     assert g["guards_ok"], "a kernel wrote outside its output"
     idx, counts, offsets, perm = oracle.route(inp.gate_logits)
@@ -164,10 +164,10 @@ def test_straight_through_expert_path_gives_the_logits_no_gradient(math_mode):
     assert not np.array_equal(aux_grad(logits * 2.0, r2).cpu().numpy(), before)
 
 
-# The TF32 backward with d_x and dW / db requested runs as one fused kernel: on
-# CTA pairs at H = 256 (256-token pair-tiles of one expert, 512 tokens per pair at
-# least), on single CTAs at H = 128 (128-token tiles). Shapes that stress the
-# tiling: a pair-tile the odd CTA has no token of, one it has a few of, one pair
+# The single-pass TF32 backward (MOE_BWD_SINGLE_PASS, or the horizon-mean gradient
+# at H = 256) runs d_x and dW / db as one fused kernel: on CTA pairs at H = 256
+# (256-token pair-tiles of one expert, 512 tokens per pair at least), on single
+# CTAs at H = 128 (128-token tiles). Shapes that stress the tiling: a pair-tile the odd CTA has no token of, one it has a few of, one pair
 # only, segments far shorter than a tile (32 experts), a range that crosses
 # several expert boundaries at odd positions, more pairs than fit on the GPU at
 # once; and the same kinds of shapes at H = 128.
@@ -186,14 +186,32 @@ FUSED_SHAPES = [
 
 @pytest.mark.parametrize("spec", FUSED_SHAPES, ids=lambda s: s.name)
 def test_fused_backward_parity(spec):
-    check_all(wl.generate(spec), ops.MOE_MATH_TF32)
+    check_all(wl.generate(spec), ops.MOE_MATH_TF32, acc_flags=ops.MOE_BWD_SINGLE_PASS)
+
+
+@pytest.mark.parametrize("H", [128, 256])
+def test_backward_strategies_agree_and_repeat(H):
+    """The two TF32 strategies (two passes by default, one with the flag) agree
+    within the TF32 tolerance (different MMA shapes for d_x, different fixed
+    summation trees for dW / db), and each repeats bit for bit."""
+    inp = wl.generate(wl.make_spec(f"strat_b3000_h3_e6_h{H}", 3000, 3, 6, H, 88))
+    two = [run_gpu(inp, ops.MOE_MATH_TF32, 0.01, parts=("route", "bwd")) for _ in range(2)]
+    one = [run_gpu(inp, ops.MOE_MATH_TF32, 0.01, parts=("route", "bwd"), acc_flags=ops.MOE_BWD_SINGLE_PASS)
+           for _ in range(2)]
+    for k in ("d_x", "dW", "db"):
+        np.testing.assert_array_equal(two[0][k], two[1][k], err_msg=k)
+        np.testing.assert_array_equal(one[0][k], one[1][k], err_msg=k)
+    atol, rtol = TOL[ops.MOE_MATH_TF32]
+    assert_close("d_x", one[0]["d_x"], two[0]["d_x"].astype(np.float64), atol, rtol)
+    for k in ("dW", "db"):
+        assert_close(k, one[0][k], two[0][k].astype(np.float64), atol, rtol, scale=np.abs(two[0][k]).max())
 
 
 @pytest.mark.parametrize("math_mode", MATHS, ids=MATH_ID.get)
 def test_backward_outputs_requested_separately(math_mode):
-    """d_x alone, dW and db alone, db alone and all three (at H = 256 with TF32
-    the last is the fused kernel, the others the separate contraction kernels):
-    every combination against the oracle."""
+    """d_x alone, dW and db alone, db alone and all three by default (the separate
+    contraction kernels), then d_x with db and all three in one pass (with TF32 the
+    fused kernel): every combination against the oracle."""
     spec = wl.make_spec("bwd_parts_b1200_h3_e6_h256", 1200, 3, 6, 256, 87)
     inp = wl.generate(spec)
     B, N_H, E, H, T = spec.B, spec.N_H, spec.E, spec.H, spec.T
@@ -206,12 +224,13 @@ def test_backward_outputs_requested_separately(math_mode):
     r = ops.Routing.empty(T, E, "cuda")
     ws = ops.new_workspace(T, E, H, "cuda")
     ops.moe_top1_route(dev(inp.gate_logits), B, N_H, E, r, ws)
-    for want in (("d_x",), ("dW", "db"), ("db",), ("d_x", "dW", "db")):
+    for want, flags in ((("d_x",), 0), (("dW", "db"), 0), (("db",), 0), (("d_x", "dW", "db"), 0),
+                        (("d_x", "db"), ops.MOE_BWD_SINGLE_PASS), (("d_x", "dW", "db"), ops.MOE_BWD_SINGLE_PASS)):
         out = {"d_x": torch.full((T, H), float("nan"), device="cuda"),
                "dW": torch.full((E, H, H), float("nan"), device="cuda"),
                "db": torch.full((E, H), float("nan"), device="cuda")}
         args = {k: (out[k] if k in want else None) for k in out}
-        ops.moe_top1_bwd(x, W, d_out, r, B, N_H, E, H, math_mode, args["d_x"], args["dW"], args["db"], 0, ws)
+        ops.moe_top1_bwd(x, W, d_out, r, B, N_H, E, H, math_mode, args["d_x"], args["dW"], args["db"], flags, ws)
         torch.cuda.synchronize()
         assert ops.moe_top1_device_flags(ws) == 0
         for k in ("d_x", "dW", "db"):
@@ -299,11 +318,12 @@ def test_accumulate_flags(math_mode, H):
     pre = {"d_x": rng.standard_normal((T, H)).astype(np.float32),
            "dW": rng.standard_normal((E, H, H)).astype(np.float32),
            "db": rng.standard_normal((E, H)).astype(np.float32)}
-    plain = run_gpu(inp, math_mode, 0.01, parts=("route", "bwd"))
-    acc = run_gpu(inp, math_mode, 0.01, parts=("route", "bwd"), preset=pre,
-                  acc_flags=ops.MOE_ACC_DX | ops.MOE_ACC_DW | ops.MOE_ACC_DB)
-    for k in ("d_x", "dW", "db"):
-        np.testing.assert_array_equal(acc[k], (pre[k] + plain[k]).astype(np.float32), err_msg=k)
+    for strategy in (0, ops.MOE_BWD_SINGLE_PASS):
+        plain = run_gpu(inp, math_mode, 0.01, parts=("route", "bwd"), acc_flags=strategy)
+        acc = run_gpu(inp, math_mode, 0.01, parts=("route", "bwd"), preset=pre,
+                      acc_flags=strategy | ops.MOE_ACC_DX | ops.MOE_ACC_DW | ops.MOE_ACC_DB)
+        for k in ("d_x", "dW", "db"):
+            np.testing.assert_array_equal(acc[k], (pre[k] + plain[k]).astype(np.float32), err_msg=(strategy, k))
 
 
 def test_empty_batch():
