@@ -585,33 +585,32 @@ hmean_fwd_tf32_sum_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const int rr = r * N_H + static_cast<int>(o[u] & 0xFFu);
-                        vv[u] = (static_cast<int>(o[u] >> 8) < E)
-                                    ? ld_shared_v4(sbase + rr * 64 + ((q4 ^ ((rr >> 1) & 3)) << 4))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                        vv[u] = ld_shared_v4_if(sbase + rr * 64 + ((q4 ^ ((rr >> 1) & 3)) << 4),
+                                                static_cast<int>(o[u] >> 8) < E);
                     }
                     const uint32_t arow = a_u32 + m * 64 + ((q4 ^ ((m >> 1) & 3)) << 4);
+                    // the list is sorted by expert, so each expert's tokens are one run: the sum
+                    // restarts at a run's first token and is stored after its last (no branches;
+                    // the same additions in the same order as a token-by-token walk). Entries of no
+                    // expert (e >= E) come last and are never stored.
                     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    int cur = -1;
                     uint32_t present = 0;
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const int e = static_cast<int>(o[u] >> 8);
-                        if (e >= E) continue;  // no expert (past the row's tokens, or out of range)
-                        if (e != cur) {
-                            if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
-                            acc = vv[u];
-                            cur = e;
-                            present |= 1u << e;
-                        } else {
-                            acc.x += vv[u].x;
-                            acc.y += vv[u].y;
-                            acc.z += vv[u].z;
-                            acc.w += vv[u].w;
-                        }
+                        const bool first = (u == 0) || static_cast<int>(o[u - 1] >> 8) != e;
+                        const bool last = e < E && (u == 15 || static_cast<int>(o[u + 1] >> 8) != e);
+                        acc.x = first ? vv[u].x : acc.x + vv[u].x;
+                        acc.y = first ? vv[u].y : acc.y + vv[u].y;
+                        acc.z = first ? vv[u].z : acc.z + vv[u].z;
+                        acc.w = first ? vv[u].w : acc.w + vv[u].w;
+                        st_shared_v4_if(arow + (e < E ? e : 0) * C::A_BYTES, acc, last);
+                        present |= (e < E) ? (1u << e) : 0u;
                     }
-                    if (cur >= 0) st_shared_v4(arow + cur * C::A_BYTES, acc.x, acc.y, acc.z, acc.w);
-                    for (int e = 0; e < E; ++e)
-                        if (!((present >> e) & 1u)) st_shared_v4(arow + e * C::A_BYTES, 0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int e = 0; e < kSMaxE; ++e)  // experts with no token of this row: zeros
+                        st_shared_v4_if(arow + e * C::A_BYTES, make_float4(0.f, 0.f, 0.f, 0.f),
+                                        e < E && !((present >> e) & 1u));
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ctl->raw_empty[slot]);
                 }
