@@ -423,3 +423,27 @@ def test_large_workload_sampled(large, math_mode):
     db, sb = oracle.bwd_db(inp.d_out, idx, inp.spec.E)
     assert_close("db", g["db"], db, atol, rtol, scale=sb)
     check_aux(inp, g, counts, lam)
+
+
+def test_large_workload_single_pass_backward(large):
+    """The single-pass TF32 backward (MOE_BWD_SINGLE_PASS) at the full size, in the
+    same sampled form: d_x on sampled tokens, the ends and the expert boundaries,
+    dW on sampled entries, db in full."""
+    inp = large
+    g = run_gpu(inp, ops.MOE_MATH_TF32, lam_of(inp), parts=("route", "bwd"), acc_flags=ops.MOE_BWD_SINGLE_PASS)
+    assert g["flags"] == 0 and g["guards_ok"]
+    idx, counts, offsets, perm = oracle.route(inp.gate_logits)
+    atol, rtol = TOL[ops.MOE_MATH_TF32]
+    mode = tf32_mode(ops.MOE_MATH_TF32)
+    rng = np.random.default_rng(98)
+    rows = np.sort(rng.choice(inp.spec.T, 512, replace=False))
+    rows = np.concatenate([rows, [0, inp.spec.T - 1], perm[offsets[1:-1]]])
+    assert_close("d_x", g["d_x"][rows], oracle.bwd_dx(inp.W, inp.d_out[rows], idx[rows], mode), atol, rtol)
+    n = 96
+    e_l = rng.integers(0, inp.spec.E, n)
+    o_l = rng.integers(0, inp.spec.H, n)
+    i_l = rng.integers(0, inp.spec.H, n)
+    vals, scales = oracle.bwd_dw_entries(inp.x, inp.d_out, idx, e_l, o_l, i_l, mode)
+    assert_close("dW", g["dW"][e_l, o_l, i_l], vals, atol, rtol, scale=scales)
+    db, sb = oracle.bwd_db(inp.d_out, idx, inp.spec.E)
+    assert_close("db", g["db"], db, atol, rtol, scale=sb)
