@@ -513,7 +513,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "tf32" if fused else "f32", "data": "synthetic",
             "config": {"workload": spec.name + ("+mean_collapse" if collapse else ""), "B": spec.B,
                        "N_H": spec.N_H, "E": E, "H": H, "tokens": T, "grad": args.grad,
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
