@@ -368,23 +368,15 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
-// Sum of n slots (slot k at src[k * stride]) in a fixed tree: slots are taken in
-// groups of eight added as ((s0+s1)+(s2+s3))+((s4+s5)+(s6+s7)) (missing slots of
-// the last group count as 0), and the group sums are added pairwise. The eight
-// loads of a group are independent, so they are in flight together.
-__device__ __forceinline__ float4 sum_slots(const float4* __restrict__ src, int64_t stride, int n) {
-    PairwiseSum ps;
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k0 = 0; k0 < n; k0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = (k0 + u < n) ? __ldg(src + static_cast<int64_t>(k0 + u) * stride) : z;
-        ps.add(add4(add4(add4(v[0], v[1]), add4(v[2], v[3])), add4(add4(v[4], v[5]), add4(v[6], v[7]))));
-    }
-    return ps.result();
-}
-
-// grid.x: float4 groups of dW[e] (plus one trailing block for db), grid.y = E.
+// Sum of the n slots of each element in a fixed tree: slots are taken in groups
+// of eight added as ((s0+s1)+(s2+s3))+((s4+s5)+(s6+s7)) (missing slots of the last
+// group count as 0), and the group sums are added pairwise in order
+// (PairwiseSum). The group sums are independent, so the 8 warps of a block
+// compute the groups g = warp, warp + 8, ... of the block's 32 elements at once
+// (eight loads in flight each), and one thread per element then combines them in
+// order. grid.x: blocks of 32 float4 elements of dW[e], then of db[e]; grid.y = E.
+constexpr int kRedElems = 32;
+constexpr int kRedMaxGroups = (kWgradMaxSplits + 7) / 8;  // slots of one expert <= ranges <= kWgradMaxSplits
 __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ part,
                                                           const float* __restrict__ part_db,
                                                           const int32_t* __restrict__ offsets, int64_t T, int E,
@@ -392,6 +384,7 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
                                                           float* __restrict__ db, int acc_dw, int acc_db) {
     griddep_wait();  // every global access below comes after the previous grid
     __shared__ int s_c[2];
+    __shared__ float4 s_g[kRedMaxGroups][kRedElems];
     const int e = blockIdx.y;
     // the ranges c that overlap expert e's tokens [a, b) are contiguous: thread c
     // tests range c (P <= blockDim.x) and the first / last overlapping one record it
@@ -411,35 +404,40 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
     }
     __syncthreads();
     const int c_lo = s_c[0], c_hi = s_c[1];
+    const int n = c_hi - c_lo + 1;  // slots of expert e (0 for an expert with no tokens)
+    const int ng = (n + 7) / 8;
     const int64_t HH = static_cast<int64_t>(H) * H;
-    const int nb_w = static_cast<int>((HH / 4 + 255) / 256);
-    if (static_cast<int>(blockIdx.x) < nb_w) {
-        if (!dW) return;
-        const int64_t j = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;  // float4 index
-        if (j >= HH / 4) return;
-        float4 r = sum_slots(reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c_lo) + e) * HH) + j,
-                             HH / 4, c_hi - c_lo + 1);
-        r = make_float4(r.x * scale, r.y * scale, r.z * scale, r.w * scale);
-        float4* dst = reinterpret_cast<float4*>(dW + e * HH) + j;
-        if (acc_dw) {
-            const float4 o = *dst;
-            r = make_float4(o.x + r.x, o.y + r.y, o.z + r.z, o.w + r.w);
+    const int nb_w = static_cast<int>((HH / 4 + kRedElems - 1) / kRedElems);
+    const bool is_w = static_cast<int>(blockIdx.x) < nb_w;
+    if (is_w ? !dW : !db) return;  // block-uniform
+    const int64_t count = is_w ? HH / 4 : H / 4;  // float4 elements of dW[e] or db[e]
+    const int jj = threadIdx.x & (kRedElems - 1), gs = threadIdx.x >> 5;
+    const int64_t j = static_cast<int64_t>(is_w ? blockIdx.x : blockIdx.x - nb_w) * kRedElems + jj;
+    const bool valid = j < count;
+    const float4* src = is_w ? reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c_lo) + e) * HH)
+                             : reinterpret_cast<const float4*>(part_db + (static_cast<int64_t>(c_lo) + e) * H);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g = gs; g < ng; g += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int k = g * 8 + u;
+            v[u] = (valid && k < n) ? __ldg(src + static_cast<int64_t>(k) * count + j) : z;
         }
-        *dst = r;
-    } else {
-        if (!db) return;
-        const int j = threadIdx.x;  // float4 index into db[e]
-        if (j >= H / 4) return;
-        float4 r = sum_slots(reinterpret_cast<const float4*>(part_db + (static_cast<int64_t>(c_lo) + e) * H) + j,
-                             H / 4, c_hi - c_lo + 1);
-        r = make_float4(r.x * scale, r.y * scale, r.z * scale, r.w * scale);
-        float4* dst = reinterpret_cast<float4*>(db + static_cast<int64_t>(e) * H) + j;
-        if (acc_db) {
-            const float4 o = *dst;
-            r = make_float4(o.x + r.x, o.y + r.y, o.z + r.z, o.w + r.w);
-        }
-        *dst = r;
+        s_g[g][jj] = add4(add4(add4(v[0], v[1]), add4(v[2], v[3])), add4(add4(v[4], v[5]), add4(v[6], v[7])));
     }
+    __syncthreads();
+    if (gs != 0 || !valid) return;
+    PairwiseSum ps;
+    for (int g = 0; g < ng; ++g) ps.add(s_g[g][jj]);
+    float4 r = ps.result();
+    r = make_float4(r.x * scale, r.y * scale, r.z * scale, r.w * scale);
+    float4* dst = is_w ? reinterpret_cast<float4*>(dW + e * HH) + j : reinterpret_cast<float4*>(db + static_cast<int64_t>(e) * H) + j;
+    if (is_w ? acc_dw : acc_db) {
+        const float4 o = *dst;
+        r = make_float4(o.x + r.x, o.y + r.y, o.z + r.z, o.w + r.w);
+    }
+    *dst = r;
 }
 
 }  // namespace
@@ -476,8 +474,10 @@ cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const i
                                 int E, int H, int P, float scale, float* dW, float* db, int acc_dw, int acc_db,
                                 cudaStream_t s) {
     const int64_t HH = static_cast<int64_t>(H) * H;
-    const int nb_w = static_cast<int>((HH / 4 + 255) / 256);
-    dim3 grid(nb_w + 1, E);
+    const int nb_w = static_cast<int>((HH / 4 + kRedElems - 1) / kRedElems);
+    const int nb_b = (H / 4 + kRedElems - 1) / kRedElems;
+    if (P < 1 || P > kWgradMaxSplits) return cudaErrorInvalidValue;  // the group sums of one expert fit s_g
+    dim3 grid(nb_w + nb_b, E);
     launch_pdl(wgrad_reduce_kernel, dim3(grid), dim3(256), 0, s,
                part, part_db, offsets, T, E, H, P, scale, dW, db, acc_dw, acc_db);
     return cudaGetLastError();
