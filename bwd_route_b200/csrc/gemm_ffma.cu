@@ -371,20 +371,27 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
 // Sum of the n slots of each element in a fixed tree: slots are taken in groups
 // of eight added as ((s0+s1)+(s2+s3))+((s4+s5)+(s6+s7)) (missing slots of the last
 // group count as 0), and the group sums are added pairwise in order
-// (PairwiseSum). The group sums are independent, so the 8 warps of a block
-// compute the groups g = warp, warp + 8, ... of the block's 32 elements at once
-// (eight loads in flight each), and one thread per element then combines them in
-// order. grid.x: blocks of 32 float4 elements of dW[e], then of db[e]; grid.y = E.
+// (PairwiseSum). The group sums are independent: a block covers S chunks of 32
+// float4 elements, and its 8 warps compute the S x ng (chunk, group) sums at once
+// (eight loads in flight each); one thread per element then combines its groups
+// in order. S adapts to the expert's group count ng so that a block holds about
+// eight such sums: S = 8 for one group, down to S = 1 from five groups on, so an
+// expert with few slots uses few blocks and one with many spreads over many.
+// grid.x: one block per 32-element chunk of dW[e], then of db[e] (the most S = 1
+// needs; with S > 1 the blocks past the last chunk return at once); grid.y = E.
 constexpr int kRedElems = 32;
+constexpr int kRedWarps = 8;
 constexpr int kRedMaxGroups = (kWgradMaxSplits + 7) / 8;  // slots of one expert <= ranges <= kWgradMaxSplits
-__global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ part,
-                                                          const float* __restrict__ part_db,
-                                                          const int32_t* __restrict__ offsets, int64_t T, int E,
-                                                          int H, int P, float scale, float* __restrict__ dW,
-                                                          float* __restrict__ db, int acc_dw, int acc_db) {
+constexpr int kRedMaxItems = kRedMaxGroups > kRedWarps ? kRedMaxGroups : kRedWarps;
+__global__ void __launch_bounds__(kRedWarps * 32) wgrad_reduce_kernel(const float* __restrict__ part,
+                                                                     const float* __restrict__ part_db,
+                                                                     const int32_t* __restrict__ offsets, int64_t T,
+                                                                     int E, int H, int P, float scale,
+                                                                     float* __restrict__ dW, float* __restrict__ db,
+                                                                     int acc_dw, int acc_db) {
     griddep_wait();  // every global access below comes after the previous grid
     __shared__ int s_c[2];
-    __shared__ float4 s_g[kRedMaxGroups][kRedElems];
+    __shared__ float4 s_g[kRedMaxItems][kRedElems];
     const int e = blockIdx.y;
     // the ranges c that overlap expert e's tokens [a, b) are contiguous: thread c
     // tests range c (P <= blockDim.x) and the first / last overlapping one record it
@@ -406,30 +413,37 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
     const int c_lo = s_c[0], c_hi = s_c[1];
     const int n = c_hi - c_lo + 1;  // slots of expert e (0 for an expert with no tokens)
     const int ng = (n + 7) / 8;
+    const int S = ng <= 1 ? 8 : ng == 2 ? 4 : ng <= 4 ? 2 : 1;  // chunks per block: S x ng <= 8 up to 8 groups
     const int64_t HH = static_cast<int64_t>(H) * H;
     const int nb_w = static_cast<int>((HH / 4 + kRedElems - 1) / kRedElems);
     const bool is_w = static_cast<int>(blockIdx.x) < nb_w;
     if (is_w ? !dW : !db) return;  // block-uniform
     const int64_t count = is_w ? HH / 4 : H / 4;  // float4 elements of dW[e] or db[e]
-    const int jj = threadIdx.x & (kRedElems - 1), gs = threadIdx.x >> 5;
-    const int64_t j = static_cast<int64_t>(is_w ? blockIdx.x : blockIdx.x - nb_w) * kRedElems + jj;
-    const bool valid = j < count;
+    const int64_t chunk0 = static_cast<int64_t>(is_w ? blockIdx.x : blockIdx.x - nb_w) * S;
+    if (chunk0 * kRedElems >= count) return;  // block-uniform: past the last chunk at this S
     const float4* src = is_w ? reinterpret_cast<const float4*>(part + (static_cast<int64_t>(c_lo) + e) * HH)
                              : reinterpret_cast<const float4*>(part_db + (static_cast<int64_t>(c_lo) + e) * H);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int g = gs; g < ng; g += 8) {
+    for (int i = warp; i < S * ng; i += kRedWarps) {  // (chunk i % S, group i / S)
+        const int g = i / S;
+        const int64_t j = (chunk0 + i % S) * kRedElems + lane;
+        const bool valid = j < count;
         float4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int k = g * 8 + u;
             v[u] = (valid && k < n) ? __ldg(src + static_cast<int64_t>(k) * count + j) : z;
         }
-        s_g[g][jj] = add4(add4(add4(v[0], v[1]), add4(v[2], v[3])), add4(add4(v[4], v[5]), add4(v[6], v[7])));
+        s_g[i][lane] = add4(add4(add4(v[0], v[1]), add4(v[2], v[3])), add4(add4(v[4], v[5]), add4(v[6], v[7])));
     }
     __syncthreads();
-    if (gs != 0 || !valid) return;
+    if (static_cast<int>(threadIdx.x) >= S * kRedElems) return;
+    const int ch = threadIdx.x / kRedElems;
+    const int64_t j = (chunk0 + ch) * kRedElems + lane;
+    if (j >= count) return;
     PairwiseSum ps;
-    for (int g = 0; g < ng; ++g) ps.add(s_g[g][jj]);
+    for (int g = 0; g < ng; ++g) ps.add(s_g[g * S + ch][lane]);
     float4 r = ps.result();
     r = make_float4(r.x * scale, r.y * scale, r.z * scale, r.w * scale);
     float4* dst = is_w ? reinterpret_cast<float4*>(dW + e * HH) + j : reinterpret_cast<float4*>(db + static_cast<int64_t>(e) * H) + j;
@@ -478,7 +492,7 @@ cudaError_t launch_wgrad_reduce(const float* part, const float* part_db, const i
     const int nb_b = (H / 4 + kRedElems - 1) / kRedElems;
     if (P < 1 || P > kWgradMaxSplits) return cudaErrorInvalidValue;  // the group sums of one expert fit s_g
     dim3 grid(nb_w + nb_b, E);
-    launch_pdl(wgrad_reduce_kernel, dim3(grid), dim3(256), 0, s,
+    launch_pdl(wgrad_reduce_kernel, dim3(grid), dim3(kRedWarps * 32), 0, s,
                part, part_db, offsets, T, E, H, P, scale, dW, db, acc_dw, acc_db);
     return cudaGetLastError();
 }
