@@ -411,8 +411,7 @@ def main():
             gate.backward(x, d_out)
         if ev:
             ev[3].record(stream)
-        gate.aux(logits)
-        gate.update_lambda()
+        gate.aux_and_update_lambda(logits)
         if ev:
             ev[4].record(stream)
 
@@ -491,8 +490,7 @@ def main():
             gate.route(logits)
             gate.forward_mean_collapse(x)
             gate.backward_mean_collapse(x, d_out)
-            gate.aux(logits)
-            gate.update_lambda()
+            gate.aux_and_update_lambda(logits)
         else:
             gate.step(logits, x, d_out)
         h_loss.copy_(gate.loss, non_blocking=True)

@@ -277,6 +277,69 @@ moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_
     return MOE_OK;
 }
 
+namespace {
+
+// Argument checks of the adaptive-lambda update (shared by the separate call and
+// the one folded into the aux launch).
+moe_status_t check_lambda_args(const float* ent_ema, float lambda_floor, float lambda_max_extra, float ent_target,
+                               const float* lambda_out) {
+    if (!ent_ema || !lambda_out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(ent_ema, 4) || !aligned(lambda_out, 4)) return MOE_ERR_MISALIGNED;
+    if (!std::isfinite(ent_target) || !(ent_target > 0.0f)) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(lambda_floor) || !(lambda_floor >= 0.0f)) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(lambda_max_extra) || !(lambda_max_extra >= 0.0f)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+moe_status_t aux_impl(const float* gate_logits, const int32_t* counts, int64_t B, int64_t N_H, int32_t E,
+                      const float* lambda_eff, float* d_logits, float* loss_out, float* mean_p, float* stats,
+                      const LambdaNext& next, void* workspace, size_t workspace_bytes, void* stream) {
+    int64_t T = 0;
+    moe_status_t st = tokens(B, N_H, &T);
+    if (st != MOE_OK) return st;
+    if (E < 1 || E > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!counts || !lambda_eff || !loss_out || !mean_p) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && !gate_logits) return MOE_ERR_INVALID_ARG;
+    if (!aligned(gate_logits, 16) || !aligned(d_logits, 16) || !aligned(counts, 4) || !aligned(lambda_eff, 4) ||
+        !aligned(loss_out, 4) || !aligned(mean_p, 4) || !aligned(stats, 4))
+        return MOE_ERR_MISALIGNED;
+    const size_t lbytes = sizeof(float) * T * E;
+    // the next lambda may replace lambda_eff (read by every block before the last
+    // one writes it) or ent_ema (read by the thread that writes it), nothing else
+    const Range outs[5] = {{d_logits, lbytes},
+                           {loss_out, 2 * sizeof(float)},
+                           {mean_p, sizeof(float) * E},
+                           {stats, sizeof(float) * (3 * E + 4)},
+                           {next.out, next.out ? sizeof(float) : 0}};
+    const bool next_is_lambda = next.out && next.out == lambda_eff;
+    const Range ins[4] = {{gate_logits, lbytes},
+                          {counts, sizeof(int32_t) * E},
+                          {next_is_lambda ? nullptr : lambda_eff, next_is_lambda ? 0 : sizeof(float)},
+                          {workspace, workspace ? workspace_bytes : 0}};
+    if (any_alias(outs, 5, ins, 4)) return MOE_ERR_ALIAS;
+    if (next_is_lambda) {  // lambda_eff is then an output too: disjoint from the other outputs
+        const Range lam[1] = {{lambda_eff, sizeof(float)}};
+        if (any_alias(outs, 4, lam, 1)) return MOE_ERR_ALIAS;
+    }
+    if (next.out) {
+        const Range ema[1] = {{next.ent_ema, sizeof(float)}};
+        if (any_alias(outs, 4, ema, 1)) return MOE_ERR_ALIAS;
+    }
+    const WsLayout L = ws_layout(T, E, 0);
+    if (!workspace) return MOE_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
+    if (workspace_bytes < L.route_end) return MOE_ERR_WORKSPACE;
+    DeviceInfo* dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    return cuda_status(launch_aux(gate_logits, counts, T, E, lambda_eff, d_logits, loss_out, mean_p, stats,
+                                  reinterpret_cast<float*>(ws + L.aux_psum),
+                                  reinterpret_cast<uint32_t*>(ws + kWsTicketOffset), next,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
 }  // namespace moe
 
 using namespace moe;
@@ -465,44 +528,32 @@ moe_status_t moe_aux_loss_fwd_bwd(const float* gate_logits, const int32_t* count
                                   int32_t E, const float* lambda_eff, float* d_logits, float* loss_out,
                                   float* mean_p, float* stats, void* workspace, size_t workspace_bytes,
                                   void* stream) {
-    int64_t T = 0;
-    moe_status_t st = tokens(B, N_H, &T);
+    return aux_impl(gate_logits, counts, B, N_H, E, lambda_eff, d_logits, loss_out, mean_p, stats, LambdaNext{},
+                    workspace, workspace_bytes, stream);
+}
+
+moe_status_t moe_aux_loss_fwd_bwd_lambda_update(const float* gate_logits, const int32_t* counts, int64_t B,
+                                                int64_t N_H, int32_t E, const float* lambda_eff, float* d_logits,
+                                                float* loss_out, float* mean_p, float* stats, const float* ent_ema,
+                                                float lambda_floor, float lambda_max_extra, float ent_target,
+                                                float* lambda_next, void* workspace, size_t workspace_bytes,
+                                                void* stream) {
+    moe_status_t st = check_lambda_args(ent_ema, lambda_floor, lambda_max_extra, ent_target, lambda_next);
     if (st != MOE_OK) return st;
-    if (E < 1 || E > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (!counts || !lambda_eff || !loss_out || !mean_p) return MOE_ERR_INVALID_ARG;
-    if (T > 0 && !gate_logits) return MOE_ERR_INVALID_ARG;
-    if (!aligned(gate_logits, 16) || !aligned(d_logits, 16) || !aligned(counts, 4) || !aligned(lambda_eff, 4) ||
-        !aligned(loss_out, 4) || !aligned(mean_p, 4) || !aligned(stats, 4))
-        return MOE_ERR_MISALIGNED;
-    const size_t lbytes = sizeof(float) * T * E;
-    const Range outs[4] = {{d_logits, lbytes},
-                           {loss_out, 2 * sizeof(float)},
-                           {mean_p, sizeof(float) * E},
-                           {stats, sizeof(float) * (3 * E + 4)}};
-    const Range ins[4] = {{gate_logits, lbytes},
-                          {counts, sizeof(int32_t) * E},
-                          {lambda_eff, sizeof(float)},
-                          {workspace, workspace ? workspace_bytes : 0}};
-    if (any_alias(outs, 4, ins, 4)) return MOE_ERR_ALIAS;
-    const WsLayout L = ws_layout(T, E, 0);
-    if (!workspace) return MOE_ERR_WORKSPACE;
-    if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
-    if (workspace_bytes < L.route_end) return MOE_ERR_WORKSPACE;
-    DeviceInfo* dev = nullptr;
-    if (device_info(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    return cuda_status(launch_aux(gate_logits, counts, T, E, lambda_eff, d_logits, loss_out, mean_p, stats,
-                                  reinterpret_cast<float*>(ws + L.aux_psum),
-                                  reinterpret_cast<uint32_t*>(ws + kWsTicketOffset), static_cast<cudaStream_t>(stream)));
+    LambdaNext next;
+    next.ent_ema = ent_ema;
+    next.floor = lambda_floor;
+    next.extra = lambda_max_extra;
+    next.target = ent_target;
+    next.out = lambda_next;
+    return aux_impl(gate_logits, counts, B, N_H, E, lambda_eff, d_logits, loss_out, mean_p, stats, next, workspace,
+                    workspace_bytes, stream);
 }
 
 moe_status_t moe_lambda_eff_update(const float* ent_ema, float lambda_floor, float lambda_max_extra,
                                    float ent_target, float* lambda_eff, void* stream) {
-    if (!ent_ema || !lambda_eff) return MOE_ERR_INVALID_ARG;
-    if (!aligned(ent_ema, 4) || !aligned(lambda_eff, 4)) return MOE_ERR_MISALIGNED;
-    if (!std::isfinite(ent_target) || !(ent_target > 0.0f)) return MOE_ERR_INVALID_ARG;
-    if (!std::isfinite(lambda_floor) || !(lambda_floor >= 0.0f)) return MOE_ERR_INVALID_ARG;
-    if (!std::isfinite(lambda_max_extra) || !(lambda_max_extra >= 0.0f)) return MOE_ERR_INVALID_ARG;
+    moe_status_t st = check_lambda_args(ent_ema, lambda_floor, lambda_max_extra, ent_target, lambda_eff);
+    if (st != MOE_OK) return st;
     return cuda_status(launch_lambda_eff(ent_ema, lambda_floor, lambda_max_extra, ent_target, lambda_eff,
                                          static_cast<cudaStream_t>(stream)));
 }

@@ -27,7 +27,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 32;                                   // tokens a warp handles at a time
-constexpr int kChunksPerWarp = kAuxTokPerBlk / (kWarps * kChunk);  // 4
+static_assert(kAuxTokPerBlkSmall == kWarps * kChunk && kAuxTokPerBlkLarge == 4 * kWarps * kChunk,
+              "aux blocks of 1 or 4 chunks per warp");
 
 // Shared-memory slot of float4 q (experts 4q..4q+3) of token row t when a row
 // holds Q = EMAX / 4 float4s: the XOR swizzle spreads the 8 rows read by one
@@ -42,22 +43,40 @@ __device__ __forceinline__ int row_slot(int t, int q) {
 
 __device__ void aux_finalize_block(const float* blk_psum, int64_t nblk,
                                    const int32_t* __restrict__ counts, int64_t T, int E,
-                                   const float* __restrict__ lambda_eff, float* __restrict__ loss_out,
+                                   const float* lambda_eff, float* __restrict__ loss_out,
                                    float* __restrict__ mean_p, float* __restrict__ stats);
 
-// One block per 1024 consecutive tokens; warp w handles chunks w, w + 8, w + 16,
-// w + 24 of 32 tokens. The warp stages all four chunks' logits in its own
+// The adaptive lambda of the next step from the gate-entropy EMA (a NaN EMA gives
+// the floor): floor + extra * max(0, target - ent_ema) / target.
+__device__ __forceinline__ float lambda_from_ema(float ent_ema, float floor, float extra, float target) {
+    float deficit = target - ent_ema;
+    if (!(deficit > 0.0f)) deficit = 0.0f;  // max(0, .); NaN gives 0
+    return floor + extra * deficit / target;
+}
+
+// Called by every thread of the block that finalized: after the barrier no
+// thread of it reads lambda_eff any more (the other blocks read it before they
+// took their tickets), so next.out may be lambda_eff.
+__device__ __forceinline__ void write_lambda_next(const LambdaNext& next) {
+    if (!next.out) return;
+    __syncthreads();
+    if (threadIdx.x == 0) *next.out = lambda_from_ema(__ldcg(next.ent_ema), next.floor, next.extra, next.target);
+}
+
+// One block per CPW x 256 consecutive tokens (CPW = 1 or 4); warp w handles
+// chunks w, w + 8, ... of 32 tokens. The warp stages all its chunks' logits in its own
 // shared buffer (128-bit loads, every load in flight before the first use, no
 // block barrier for the data), lane t computes token t of each chunk reading
 // its row as float4s, and the gradients go back out with 128-bit stores. When
 // E is not a multiple of 4 the rows are moved one float at a time.
-template <int EMAX>
+template <int EMAX, int kChunksPerWarp>
 __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__ logits,
                                                       const int32_t* __restrict__ counts, int64_t T, int E,
-                                                      const float* __restrict__ lambda_eff,
+                                                      const float* lambda_eff,
                                                       float* __restrict__ d_logits, float* __restrict__ blk_psum,
                                                       uint32_t* __restrict__ ticket, float* __restrict__ loss_out,
-                                                      float* __restrict__ mean_p, float* __restrict__ stats) {
+                                                      float* __restrict__ mean_p, float* __restrict__ stats,
+                                                      LambdaNext next) {
     griddep_wait();  // every global access below comes after the previous grid
     constexpr int Q = EMAX / 4;          // float4s per staged row
     constexpr int BUF4 = kChunk * Q;     // float4s per chunk buffer
@@ -67,7 +86,8 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x < EMAX)
         s_frac[threadIdx.x] = threadIdx.x < E ? static_cast<float>(counts[threadIdx.x]) / static_cast<float>(T) : 0.0f;
-    const float lam = *lambda_eff;
+    // through L2: the last block may overwrite lambda_eff (next.out) once every block has used it
+    const float lam = __ldcg(lambda_eff);
     const float scale = lam * static_cast<float>(E) / static_cast<float>(T);
     const bool vec = (E == EMAX);        // rows move as whole float4s
     float4* wbuf = s_dyn4 + warp * kChunksPerWarp * BUF4;
@@ -75,7 +95,7 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
     int n[kChunksPerWarp];
 #pragma unroll
     for (int j = 0; j < kChunksPerWarp; ++j) {
-        c0[j] = static_cast<int64_t>(blockIdx.x) * kAuxTokPerBlk + (j * kWarps + warp) * kChunk;
+        c0[j] = static_cast<int64_t>(blockIdx.x) * (kChunksPerWarp * kWarps * kChunk) + (j * kWarps + warp) * kChunk;
         n[j] = c0[j] >= T ? 0 : static_cast<int>((T - c0[j] < kChunk) ? (T - c0[j]) : kChunk);
     }
     if (vec) {
@@ -201,6 +221,7 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
         __threadfence();
         aux_finalize_block(blk_psum, gridDim.x, counts, T, E, lambda_eff, loss_out, mean_p, stats);
         if (threadIdx.x == 0) *ticket = 0u;
+        write_lambda_next(next);
     }
 }
 
@@ -210,7 +231,7 @@ __global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__
 // loads in flight), then an xor butterfly combines the lanes.
 __device__ void aux_finalize_block(const float* blk_psum, int64_t nblk,
                                    const int32_t* __restrict__ counts, int64_t T, int E,
-                                   const float* __restrict__ lambda_eff, float* __restrict__ loss_out,
+                                   const float* lambda_eff, float* __restrict__ loss_out,
                                    float* __restrict__ mean_p, float* __restrict__ stats) {
     __shared__ double s_sum[32];
     __shared__ float s_mean[32];
@@ -219,7 +240,7 @@ __device__ void aux_finalize_block(const float* blk_psum, int64_t nblk,
     __shared__ float s_lam;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
-    if (threadIdx.x == 0) s_lam = *lambda_eff;
+    if (threadIdx.x == 0) s_lam = __ldcg(lambda_eff);
     if (threadIdx.x < E) s_cnt[threadIdx.x] = counts[threadIdx.x];
     for (int e = warp; e < E; e += nwarps) {
         double acc = 0.0;
@@ -279,19 +300,18 @@ __device__ void aux_finalize_block(const float* blk_psum, int64_t nblk,
 
 // The empty batch: only the finalize (zeros, and lambda in the stats).
 __global__ void __launch_bounds__(kThreads) aux_finalize_kernel(const int32_t* __restrict__ counts, int E,
-                                                               const float* __restrict__ lambda_eff,
+                                                               const float* lambda_eff,
                                                                float* __restrict__ loss_out, float* __restrict__ mean_p,
-                                                               float* __restrict__ stats) {
+                                                               float* __restrict__ stats, LambdaNext next) {
     griddep_wait();  // every global access below comes after the previous grid
     aux_finalize_block(nullptr, 0, counts, 0, E, lambda_eff, loss_out, mean_p, stats);
+    write_lambda_next(next);
 }
 
 __global__ void lambda_eff_kernel(const float* __restrict__ ent_ema, float lambda_floor, float lambda_max_extra,
                                   float ent_target, float* __restrict__ lambda_eff) {
     griddep_wait();  // every global access below comes after the previous grid
-    float deficit = ent_target - *ent_ema;
-    if (!(deficit > 0.0f)) deficit = 0.0f;  // max(0, .); a NaN entropy gives the floor
-    *lambda_eff = lambda_floor + lambda_max_extra * deficit / ent_target;
+    *lambda_eff = lambda_from_ema(*ent_ema, lambda_floor, lambda_max_extra, ent_target);
 }
 
 // Producer of the gate-entropy signal the lambda controller reads (one warp;
@@ -331,26 +351,32 @@ cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, fl
 
 cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, int E, const float* lambda_eff,
                        float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,
-                       uint32_t* ticket, cudaStream_t s) {
+                       uint32_t* ticket, LambdaNext next, cudaStream_t s) {
     if (T == 0) {
         launch_pdl(aux_finalize_kernel, dim3(1), dim3(kThreads), 0, s,
-                   counts, E, lambda_eff, loss_out, mean_p, stats);
+                   counts, E, lambda_eff, loss_out, mean_p, stats, next);
         return cudaGetLastError();
     }
-    const int64_t nblk = (T + kAuxTokPerBlk - 1) / kAuxTokPerBlk;
-    const size_t smem = sizeof(float) * kWarps * kChunksPerWarp * kChunk * (E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32);
-    if (E <= 4)
-        launch_pdl(aux_kernel<4>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
-                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
-    else if (E <= 8)
-        launch_pdl(aux_kernel<8>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
-                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
-    else if (E <= 16)
-        launch_pdl(aux_kernel<16>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
-                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
-    else
-        launch_pdl(aux_kernel<32>, dim3((unsigned)nblk), dim3(kThreads), smem, s,
-                   logits, counts, T, E, lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats);
+    const int tpb = aux_tok_per_blk(T);
+    const int64_t nblk = (T + tpb - 1) / tpb;
+    const int cpw = tpb / (kWarps * kChunk);
+    const int emax = E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32;
+    const size_t smem = sizeof(float) * kWarps * cpw * kChunk * emax;
+#define MOE_AUX_LAUNCH(EM, CPW)                                                                              \
+    launch_pdl(aux_kernel<EM, CPW>, dim3((unsigned)nblk), dim3(kThreads), smem, s, logits, counts, T, E,     \
+               lambda_eff, d_logits, blk_psum, ticket, loss_out, mean_p, stats, next)
+    if (cpw == 1) {
+        if (emax == 4) MOE_AUX_LAUNCH(4, 1);
+        else if (emax == 8) MOE_AUX_LAUNCH(8, 1);
+        else if (emax == 16) MOE_AUX_LAUNCH(16, 1);
+        else MOE_AUX_LAUNCH(32, 1);
+    } else {
+        if (emax == 4) MOE_AUX_LAUNCH(4, 4);
+        else if (emax == 8) MOE_AUX_LAUNCH(8, 4);
+        else if (emax == 16) MOE_AUX_LAUNCH(16, 4);
+        else MOE_AUX_LAUNCH(32, 4);
+    }
+#undef MOE_AUX_LAUNCH
     return cudaGetLastError();
 }
 
@@ -363,11 +389,11 @@ cudaError_t launch_lambda_eff(const float* ent_ema, float lambda_floor, float la
 
 cudaError_t aux_set_smem_limits() {
     // 8 warps x 4 chunks x 32 tokens x 32 experts x 4 bytes = 128 KiB for the widest instance
-    cudaError_t e = cudaFuncSetAttribute(aux_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(float) * kWarps * kChunksPerWarp * kChunk * 16));
+    cudaError_t e = cudaFuncSetAttribute(aux_kernel<16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(float) * kWarps * 4 * kChunk * 16));
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(aux_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(float) * kWarps * kChunksPerWarp * kChunk * 32));
+    return cudaFuncSetAttribute(aux_kernel<32, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(float) * kWarps * 4 * kChunk * 32));
 }
 
 }  // namespace moe

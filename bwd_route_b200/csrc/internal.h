@@ -8,9 +8,14 @@
 
 namespace moe {
 
-// Tokens handled by one block of the routing and aux kernels.
+// Tokens handled by one block of the routing kernels, and by one block of the
+// aux kernel: 256 up to kAuxSmallT tokens (more blocks, a shorter chain per
+// block), 1024 above (fewer per-block partial sums for the last block to add).
 constexpr int kRouteTokPerBlk = 1024;
-constexpr int kAuxTokPerBlk = 1024;
+constexpr int kAuxTokPerBlkSmall = 256;
+constexpr int kAuxTokPerBlkLarge = 1024;
+constexpr int64_t kAuxSmallT = 262144;
+inline int aux_tok_per_blk(int64_t T) { return T <= kAuxSmallT ? kAuxTokPerBlkSmall : kAuxTokPerBlkLarge; }
 
 // Weight-gradient contraction: the expert-sorted token list is cut into
 // `wgrad_splits(T)` equal ranges (further cut at expert boundaries); range c
@@ -48,7 +53,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline WsLayout ws_layout(int64_t T, int E, int H) {
     WsLayout L;
     const int64_t nr = T > 0 ? (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk : 1;
-    const int64_t na = T > 0 ? (T + kAuxTokPerBlk - 1) / kAuxTokPerBlk : 1;
+    const int64_t na = T > 0 ? (T + aux_tok_per_blk(T) - 1) / aux_tok_per_blk(T) : 1;
     const int P = wgrad_splits(T);
     size_t off = 0;
     L.flags = off;
@@ -76,11 +81,21 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int32_t* expert_
                          int32_t* offsets, int32_t* perm, int32_t* blk_counts, int32_t* blk_base,
                          cudaStream_t s);
 
+// The adaptive-lambda update that can follow the aux loss in the same launch:
+// out = floor + extra * max(0, target - *ent_ema) / target. out == nullptr: none.
+struct LambdaNext {
+    const float* ent_ema = nullptr;
+    float floor = 0.0f, extra = 0.0f, target = 1.0f;
+    float* out = nullptr;
+};
+
 // ticket: a uint32 of the workspace's reserved head (zeroed by
 // moe_top1_workspace_init); the aux kernel's last block resets it after use.
+// With next.out set, the last block also writes the next lambda once every block
+// has read lambda_eff (next.out may be lambda_eff).
 cudaError_t launch_aux(const float* logits, const int32_t* counts, int64_t T, int E, const float* lambda_eff,
                        float* d_logits, float* loss_out, float* mean_p, float* stats, float* blk_psum,
-                       uint32_t* ticket, cudaStream_t s);
+                       uint32_t* ticket, LambdaNext next, cudaStream_t s);
 
 cudaError_t launch_usage_entropy_ema(const int32_t* counts, int64_t T, int E, float alpha, int reset,
                                      float* usage_ema, float* ent_ema, float* ent_step, cudaStream_t s);

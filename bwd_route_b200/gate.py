@@ -30,13 +30,13 @@ class MoETop1Gate:
     # scan folded in) while ceil(T / 1024) * E <= 32768, else 3 (a separate scan);
     # fwd 1; bwd 3 (d_x, the weight-gradient contraction and the slot reduction),
     # or 2 for the horizon-mean gradient with TF32 at H = 256 (one fused kernel for
-    # both contractions, then the reduction); aux 1 (its last block finalizes);
-    # lambda 1
+    # both contractions, then the reduction); aux with the lambda update 1 (its
+    # last block finalizes the loss, then writes the next lambda)
     @staticmethod
     def launches_per_step(math: int, H: int, T: int, E: int, mean_collapse: bool = False) -> int:
         route = 2 if -(-T // 1024) * E <= 32768 else 3
         bwd = 2 if (math == ops.MOE_MATH_TF32 and mean_collapse and H == 256) else 3
-        return route + 1 + bwd + 1 + 1
+        return route + 1 + bwd + 1  # aux and the lambda update share one launch
 
     def __init__(self, W: torch.Tensor, bias: torch.Tensor, B: int, N_H: int, math: int = ops.MOE_MATH_TF32,
                  lambda_floor: float = 0.01, lambda_max_extra: float = 0.09, ent_target: float = 1.0,
@@ -99,6 +99,13 @@ class MoETop1Gate:
         ops.moe_aux_loss_fwd_bwd(gate_logits, self.routing.counts, self.B, self.N_H, self.E, self.lambda_eff,
                                  self.d_logits, self.loss, self.mean_p, self.stats, self.ws, stream)
 
+    def aux_and_update_lambda(self, gate_logits, stream=None):
+        """aux() and then update_lambda() in one launch (the same bits)."""
+        ops.moe_aux_loss_fwd_bwd_lambda_update(gate_logits, self.routing.counts, self.B, self.N_H, self.E,
+                                               self.lambda_eff, self.d_logits, self.loss, self.mean_p, self.stats,
+                                               self.ent_ema, self.lambda_floor, self.lambda_max_extra,
+                                               self.ent_target, self.lambda_eff, self.ws, stream)
+
     def update_lambda(self, stream=None):
         ops.moe_lambda_eff_update(self.ent_ema, self.lambda_floor, self.lambda_max_extra, self.ent_target,
                                   self.lambda_eff, stream)
@@ -142,5 +149,4 @@ class MoETop1Gate:
         self.route(gate_logits, stream)
         self.forward(x, stream)
         self.backward(x, d_out, stream)
-        self.aux(gate_logits, stream)
-        self.update_lambda(stream)
+        self.aux_and_update_lambda(gate_logits, stream)

@@ -32,7 +32,7 @@ EXPORTED = [
     "moe_top1_bwd", "moe_aux_loss_fwd_bwd", "moe_lambda_eff_update", "moe_top1_device_flags",
     "moe_status_string", "moe_top1_abi_version", "moe_top1_route_noalloc", "moe_top1_selftest_wait_timeout",
     "moe_usage_entropy_ema_update", "moe_top1_bwd_mean_collapse", "moe_top1_fwd_mean_collapse",
-    "moe_top1_check_routing",
+    "moe_top1_check_routing", "moe_aux_loss_fwd_bwd_lambda_update",
 ]
 MOE_NOALLOC_MAX_TOKENS = 2097152
 
@@ -82,6 +82,9 @@ def lib() -> ctypes.CDLL:
         L.moe_top1_bwd_mean_collapse.argtypes = L.moe_top1_bwd.argtypes
         L.moe_aux_loss_fwd_bwd.restype = I32
         L.moe_aux_loss_fwd_bwd.argtypes = [P, P, I64, I64, I32, P, P, P, P, P, P, SZ, P]
+        L.moe_aux_loss_fwd_bwd_lambda_update.restype = I32
+        L.moe_aux_loss_fwd_bwd_lambda_update.argtypes = [P, P, I64, I64, I32, P, P, P, P, P, P, ctypes.c_float,
+                                                         ctypes.c_float, ctypes.c_float, P, P, SZ, P]
         L.moe_lambda_eff_update.restype = I32
         L.moe_lambda_eff_update.argtypes = [P, ctypes.c_float, ctypes.c_float, ctypes.c_float, P, P]
         L.moe_top1_device_flags.restype = I32
@@ -236,6 +239,18 @@ def moe_aux_loss_fwd_bwd(gate_logits, counts, B: int, N_H: int, E: int, lambda_e
            lib().moe_aux_loss_fwd_bwd(_ptr(gate_logits, f), _ptr(counts, torch.int32), B, N_H, E,
                                       _ptr(lambda_eff, f), _ptr(d_logits, f), _ptr(loss_out, f), _ptr(mean_p, f),
                                       _ptr(stats, f), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_aux_loss_fwd_bwd_lambda_update(gate_logits, counts, B: int, N_H: int, E: int, lambda_eff, d_logits,
+                                      loss_out, mean_p, stats, ent_ema, lambda_floor: float,
+                                      lambda_max_extra: float, ent_target: float, lambda_next, ws: torch.Tensor,
+                                      stream=None):
+    f = torch.float32
+    _check("moe_aux_loss_fwd_bwd_lambda_update",
+           lib().moe_aux_loss_fwd_bwd_lambda_update(
+               _ptr(gate_logits, f), _ptr(counts, torch.int32), B, N_H, E, _ptr(lambda_eff, f), _ptr(d_logits, f),
+               _ptr(loss_out, f), _ptr(mean_p, f), _ptr(stats, f), _ptr(ent_ema, f), lambda_floor,
+               lambda_max_extra, ent_target, _ptr(lambda_next, f), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def moe_lambda_eff_update(ent_ema, lambda_floor: float, lambda_max_extra: float, ent_target: float, lambda_eff,

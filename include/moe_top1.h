@@ -61,8 +61,11 @@ extern "C" {
  *    unchanged).
  * 5: adds the MOE_BWD_SINGLE_PASS flag of the backward calls; moe_top1_bwd with
  *    TF32 and every output requested takes two contraction passes by default
- *    (results within fp32 rounding of version 4's single pass). */
-#define MOE_TOP1_ABI_VERSION 5
+ *    (results within fp32 rounding of version 4's single pass).
+ * 6: adds moe_aux_loss_fwd_bwd_lambda_update (the aux loss and the lambda update
+ *    in one launch); the aux loss's per-block sums of p cover 256 tokens up to
+ *    262,144 tokens (mean_p within fp32 rounding of version 5 there). */
+#define MOE_TOP1_ABI_VERSION 6
 
 typedef enum {
     MOE_OK = 0,
@@ -289,6 +292,25 @@ moe_status_t moe_aux_loss_fwd_bwd(const float* gate_logits, const int32_t* count
                                   int64_t N_H, int32_t E, const float* lambda_eff,
                                   float* d_logits, float* loss_out, float* mean_p, float* stats,
                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_aux_loss_fwd_bwd and then moe_lambda_eff_update in one launch (the order of
+ * a training step: this step's loss uses the current weight, the controller then
+ * sets the next one). Every output of moe_aux_loss_fwd_bwd is computed with
+ * lambda = *lambda_eff as it was when the call began; then
+ *   *lambda_next = lambda_floor + lambda_max_extra * max(0, ent_target - *ent_ema) / ent_target
+ * is written by the block that finishes last, after every block has read
+ * lambda_eff. lambda_next may be lambda_eff (the weight for the next step replaces
+ * this step's) or ent_ema, and must not overlap any other output. Arguments,
+ * requirements and errors are those of the two calls; every bit of every output
+ * is the same as theirs.
+ */
+moe_status_t moe_aux_loss_fwd_bwd_lambda_update(const float* gate_logits, const int32_t* counts, int64_t B,
+                                                int64_t N_H, int32_t E, const float* lambda_eff,
+                                                float* d_logits, float* loss_out, float* mean_p, float* stats,
+                                                const float* ent_ema, float lambda_floor,
+                                                float lambda_max_extra, float ent_target, float* lambda_next,
+                                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Adaptive load-balance weight. [P2] opening paragraph:

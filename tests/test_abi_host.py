@@ -53,7 +53,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_top1_abi_version() == 5
+    assert L.moe_top1_abi_version() == 6
     for s, name in enumerate(ops._STATUS):
         assert L.moe_status_string(s).decode() == name
     assert L.moe_status_string(99).decode() == "MOE_ERR_UNKNOWN"
@@ -144,6 +144,41 @@ def test_aux_and_lambda_reject_bad_arguments(L):
     assert u(e, -0.01, 0.09, 1.0, out, None) == INVALID
     assert u(e, 0.01, float("inf"), 1.0, out, None) == INVALID
     assert u(_p(A + 2), 0.01, 0.09, 1.0, out, None) == MISALIGNED
+
+
+def test_aux_with_lambda_update_rejects_bad_arguments(L):
+    """The folded call checks the arguments of both calls; the next lambda may be
+    lambda_eff or ent_ema and nothing else the call touches (the aliasing checks
+    run before the workspace check, so a too-small workspace marks a call that
+    got past them)."""
+    lg, cnt, lam = _p(A), _p(A + 0x1000000), _p(A + 0x1000100)
+    d, loss, mp, st = _p(A + 0x2000000), _p(A + 0x3000000), _p(A + 0x3000100), _p(A + 0x3000200)
+    ema, nxt = _p(A + 0x1000200), _p(A + 0x1000300)
+    ws, wsb = _p(A + 0x40000000), 1 << 20
+    f = L.moe_aux_loss_fwd_bwd_lambda_update
+
+    def call(**k):
+        return f(k.get("lg", lg), cnt, 8, 5, k.get("E", 4), k.get("lam", lam), k.get("d", d), loss,
+                 k.get("mp", mp), st, k.get("ema", ema), k.get("floor", 0.01), k.get("extra", 0.09),
+                 k.get("target", 1.0), k.get("nxt", nxt), ws, k.get("wsb", wsb), None)
+
+    assert call(E=0) == SHAPE
+    assert call(ema=None) == INVALID
+    assert call(nxt=None) == INVALID
+    assert call(target=0.0) == INVALID
+    assert call(target=float("nan")) == INVALID
+    assert call(floor=-0.01) == INVALID
+    assert call(extra=float("inf")) == INVALID
+    assert call(nxt=_p(A + 0x1000302)) == MISALIGNED
+    assert call(nxt=loss) == ALIAS                      # next lambda on loss_out
+    assert call(nxt=_p(A + 0x2000000 + 32)) == ALIAS    # next lambda inside d_logits
+    assert call(nxt=_p(A + 16)) == ALIAS                # next lambda inside the logits
+    assert call(nxt=cnt) == ALIAS                       # next lambda on counts
+    assert call(lam=mp, nxt=mp) == ALIAS                # lambda_eff (written) on mean_p
+    assert call(ema=d) == ALIAS                         # ent_ema inside d_logits
+    assert call(wsb=16) == WORKSPACE                    # separate buffers
+    assert call(nxt=lam, wsb=16) == WORKSPACE           # next lambda replaces lambda_eff
+    assert call(nxt=ema, wsb=16) == WORKSPACE           # next lambda replaces ent_ema
 
 
 def test_bwd_mean_collapse_rejects_bad_arguments(L):

@@ -108,3 +108,63 @@ def test_closed_loop_follows_the_oracle_and_is_deterministic():
     assert runs[0] == runs[1]
     # the skew (+2 on expert 4, ~71 % of tokens) keeps the entropy below the target: lambda above the floor
     assert runs[0][-1][2] > 0.01
+
+
+AUX_CASES = [wl.WORKLOADS["tiny_b8_e4_h128"], wl.WORKLOADS["skewed_b4096_e8_h128"],
+             wl.make_spec("aux_b52429_h5_e5", 52429, 5, 5, 32, 405),  # 1024-token blocks, rows moved per float
+             wl.make_spec("aux_empty_b0_e3", 0, 5, 3, 32, 406)]
+
+
+@pytest.mark.parametrize("spec", AUX_CASES, ids=lambda s: s.name)
+@pytest.mark.parametrize("target", ["separate", "lambda_eff", "ent_ema"])
+def test_aux_with_lambda_update_is_the_two_calls(spec, target):
+    """moe_aux_loss_fwd_bwd_lambda_update gives every bit of moe_aux_loss_fwd_bwd
+    followed by moe_lambda_eff_update: the loss and d_logits with the weight the
+    call began with, then the next weight, written into a buffer of its own, over
+    lambda_eff, or over ent_ema. Twice in a row (the ticket is reset)."""
+    inp = wl.generate(spec, with_activations=False)
+    B, N_H, E, T = spec.B, spec.N_H, spec.E, spec.T
+    logits = torch.from_numpy(np.ascontiguousarray(inp.gate_logits)).cuda() if T else None
+    routing = ops.Routing.empty(T, E, "cuda")
+    ws = ops.new_workspace(T, E, 32, "cuda")
+    if T:
+        ops.moe_top1_route(logits, B, N_H, E, routing, ws)
+    else:
+        routing.counts.zero_()
+    lam0, ema0, floor, extra, tgt = 0.03, 0.2, 0.01, 0.09, 1.0
+
+    def outs():
+        return {"d": Guarded(T * E), "loss": Guarded(2), "mp": Guarded(E), "st": Guarded(3 * E + 4)}
+
+    # the two calls
+    ref = outs()
+    lam = torch.tensor([lam0], device="cuda")
+    ema = torch.tensor([ema0], device="cuda")
+    ops.moe_aux_loss_fwd_bwd(logits, routing.counts, B, N_H, E, lam, ref["d"].t if T else None, ref["loss"].t,
+                             ref["mp"].t, ref["st"].t, ws)
+    ops.moe_lambda_eff_update(ema, floor, extra, tgt, lam)
+    torch.cuda.synchronize()
+    lam_next = float(lam.item())
+    assert lam_next != np.float32(lam0)
+    for rep in range(2):
+        got = outs()
+        lam = Guarded(1)
+        lam.t.fill_(lam0)
+        ema = Guarded(1)
+        ema.t.fill_(ema0)
+        nxt = Guarded(1)
+        out_buf = {"separate": nxt, "lambda_eff": lam, "ent_ema": ema}[target]
+        ops.moe_aux_loss_fwd_bwd_lambda_update(logits, routing.counts, B, N_H, E, lam.t,
+                                               got["d"].t if T else None, got["loss"].t, got["mp"].t,
+                                               got["st"].t, ema.t, floor, extra, tgt, out_buf.t, ws)
+        torch.cuda.synchronize()
+        assert ops.moe_top1_device_flags(ws) == 0
+        for k in got:
+            assert got[k].guards_intact(), k
+            assert got[k].host().tobytes() == ref[k].host().tobytes(), k
+        assert lam.guards_intact() and ema.guards_intact() and nxt.guards_intact()
+        assert float(out_buf.t.item()) == lam_next
+        if target != "lambda_eff":
+            assert float(lam.t.item()) == np.float32(lam0)
+        if target != "ent_ema":
+            assert float(ema.t.item()) == np.float32(ema0)
