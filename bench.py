@@ -130,7 +130,8 @@ CALL_KERNELS = {
     ("fwd", False): ["grouped_ffma_kernel"],
     ("bwd", True): ["grouped_tf32_kernel (d_x)", "wgrad_tf32_kernel", "wgrad_reduce_kernel"],
     ("bwd", False): ["grouped_ffma_kernel (d_x)", "wgrad_ffma_kernel", "wgrad_reduce_kernel"],
-    ("bwd", "mean_collapse"): ["bwd_fused_pair_kernel", "wgrad_reduce_kernel"],
+    ("bwd", "single_pass_256"): ["bwd_fused_pair_kernel", "wgrad_reduce_kernel"],
+    ("bwd", "single_pass_128"): ["bwd_fused_single_kernel", "wgrad_reduce_kernel"],
 }
 
 
@@ -156,13 +157,17 @@ def scale_traffic(measured: int, fixed: int, scale: float) -> int:
     return int(round(fixed + (measured - fixed) * scale))
 
 
-def bwd_passes(math_name: str, grad: str, H: int) -> int:
+def bwd_passes(math_name: str, grad: str, H: int, T: int) -> int:
     """Contraction passes of the library's default TF32 backward: one fused pass for
-    the horizon-mean gradient at H = 256, two (d_x; dW and db) otherwise."""
-    return 1 if (math_name == "tf32" and grad == "mean_collapse" and H == 256) else 2
+    the horizon-mean gradient at H = 256 and at H = 128 above 65,536 tokens, two
+    (d_x; dW and db) otherwise."""
+    if math_name != "tf32":
+        return 2
+    return 1 if ((grad == "mean_collapse" and H == 256) or (H == 128 and T > 65536)) else 2
 
 
-def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "token", H: int = 256):
+def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "token", H: int = 256,
+                     T: int = 1048576):
     """DRAM bytes (read + write) of one launch of `call`, from the committed ncu
     record (counters taken on a smaller case of the same shape and scaled to the
     workload), or None when there is no record for this workload, gradient mode
@@ -176,7 +181,7 @@ def recorded_traffic(call: str, workload: str, math_name: str, grad: str = "toke
                 continue
             if code_sha1([os.path.join(HERE, f) for f in rec["source_files"]]) != rec["code_sha1"]:
                 return None
-            if call == "bwd" and rec.get("bwd_passes") != bwd_passes(math_name, grad, H):
+            if call == "bwd" and rec.get("bwd_passes") != bwd_passes(math_name, grad, H, T):
                 return None
             v = rec["traffic_bytes_per_call"].get(call)
             return int(v) if v is not None else None
@@ -517,11 +522,12 @@ def main():
                        "math": args.math, "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": l2_note(spec, collapse, flush is not None)},
             "roofline": {"bound": "hbm", "kernel": dominant, "launches_in_call": CALL_KERNELS[
-                             (dominant, "mean_collapse") if (fused and collapse and H == 256 and dominant == "bwd")
+                             (dominant, f"single_pass_{H}") if (fused and dominant == "bwd" and
+                                                                bwd_passes(args.math, args.grad, H, T) == 1)
                              else (dominant, fused)],
                          "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm,
-                         "traffic": recorded_traffic(dominant, spec.name, args.math, args.grad, H),
+                         "traffic": recorded_traffic(dominant, spec.name, args.math, args.grad, H, T),
                          "algorithmic_bytes": kbytes[dominant], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "flops": step_flops, "t_roofline_ms": t_roof * 1e3,
                               "frac": t_roof * 1e3 / ms_per_step,

@@ -232,13 +232,10 @@ moe_status_t bwd_impl(const float* x, const float* W, const float* d_out, int64_
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
     // One pass over d_out (d_x and the dW / db partial sums together), or two (d_x,
-    // then dW / db): the single pass reads d_out and x once, but on the B200 the two
-    // passes take less time for the per-token gradient (0.735 against 0.792 ms at
-    // 1,048,576 tokens, H 256), so the single pass is the default only for the
-    // [B, H] gradient of the horizon mean at H = 256 (0.733 against 0.757 ms), and
-    // on request (MOE_BWD_SINGLE_PASS).
+    // then dW / db): bwd_single_pass_default gives the measured rule, and
+    // MOE_BWD_SINGLE_PASS asks for the single pass at every size.
     const bool single_pass = math == MOE_MATH_TF32 && d_x && (dW || db) &&
-                             ((accumulate_flags & MOE_BWD_SINGLE_PASS) || (collapse && H == 256));
+                             ((accumulate_flags & MOE_BWD_SINGLE_PASS) || bwd_single_pass_default(H, T, collapse));
     if (single_pass) {
         // H = 256: pairs of CTAs (as many as run at once); H = 128: single CTAs, one
         // per wgrad_splits(T) range

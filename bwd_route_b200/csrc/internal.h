@@ -23,7 +23,19 @@ inline int aux_tok_per_blk(int64_t T) { return T <= kAuxSmallT ? kAuxTokPerBlkSm
 // only, so the reduction tree -- and hence every bit of dW and db -- is fixed
 // for a given routing.
 constexpr int kWgradMaxSplits = 148;
-constexpr int kWgradMinTokPerSplit = 256;
+constexpr int kWgradMinTokPerSplit = 128;  // one 128-token tile: more CTAs at small T
+// The TF32 backward strategy when the caller does not ask for one: a single pass
+// over d_out (d_x and the dW / db partial sums together) for the horizon-mean
+// gradient at H = 256, and at H = 128 above 65,536 tokens; two passes otherwise.
+// Measured on a B200 (backward call, CUDA graph), two passes against one: H 128,
+// 40,960 tokens 27.7 / 29.5 us, 65,535: 36.3 / 37.6, 81,920: 45.1 / 40.9,
+// 131,070: 64.1 / 53.6, 262,144: 110.5 / 88.8, 1,048,576: 396 / 327; H 256,
+// 1,048,576 tokens, per-token gradient 0.735 / 0.792 ms, horizon-mean gradient
+// 0.757 / 0.733 ms.
+constexpr int64_t kBwdSinglePassMinT128 = 65536;
+inline bool bwd_single_pass_default(int H, int64_t T, bool collapse) {
+    return (collapse && H == 256) || (H == 128 && T > kBwdSinglePassMinT128);
+}
 inline int wgrad_splits(int64_t T) {
     int64_t p = (T + kWgradMinTokPerSplit - 1) / kWgradMinTokPerSplit;
     if (p < 1) p = 1;

@@ -29,13 +29,15 @@ class MoETop1Gate:
     # kernels launched per step with T > 0: route 2 (count; scatter with the
     # scan folded in) while ceil(T / 1024) * E <= 32768, else 3 (a separate scan);
     # fwd 1; bwd 3 (d_x, the weight-gradient contraction and the slot reduction),
-    # or 2 for the horizon-mean gradient with TF32 at H = 256 (one fused kernel for
-    # both contractions, then the reduction); aux with the lambda update 1 (its
+    # or 2 where the TF32 backward takes one fused pass for both contractions
+    # (the horizon-mean gradient at H = 256; H = 128 above 65,536 tokens), then the
+    # reduction; aux with the lambda update 1 (its
     # last block finalizes the loss, then writes the next lambda)
     @staticmethod
     def launches_per_step(math: int, H: int, T: int, E: int, mean_collapse: bool = False) -> int:
         route = 2 if -(-T // 1024) * E <= 32768 else 3
-        bwd = 2 if (math == ops.MOE_MATH_TF32 and mean_collapse and H == 256) else 3
+        single = math == ops.MOE_MATH_TF32 and ((mean_collapse and H == 256) or (H == 128 and T > 65536))
+        bwd = 2 if single else 3
         return route + 1 + bwd + 1  # aux and the lambda update share one launch
 
     def __init__(self, W: torch.Tensor, bias: torch.Tensor, B: int, N_H: int, math: int = ops.MOE_MATH_TF32,

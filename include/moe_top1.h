@@ -62,7 +62,9 @@ extern "C" {
  * 5: adds the MOE_BWD_SINGLE_PASS flag of the backward calls; moe_top1_bwd with
  *    TF32 and every output requested takes two contraction passes by default
  *    (results within fp32 rounding of version 4's single pass).
- * 6: adds moe_aux_loss_fwd_bwd_lambda_update (the aux loss and the lambda update
+ * 6: the TF32 backward takes the single pass by default at H = 128 above 65,536
+ *    tokens; the weight-gradient ranges hold 128 tokens or more (256 before), so
+ *    dW / db below 18,944 tokens sum in another fixed order; adds moe_aux_loss_fwd_bwd_lambda_update (the aux loss and the lambda update
  *    in one launch); the aux loss's per-block sums of p cover 256 tokens up to
  *    262,144 tokens (mean_p within fp32 rounding of version 5 there). */
 #define MOE_TOP1_ABI_VERSION 6
@@ -222,10 +224,11 @@ moe_status_t moe_top1_fwd_mean_collapse(const float* x, const float* W, const fl
  * requested, the backward runs either two contraction passes (d_x; then dW and
  * db) or a single pass that computes all three from one read of d_out (or
  * grad_ctx_mean) and x ([P1] kernel list: one backward produces d_fused_ctx and
- * dW / db). The single pass moves about a third less DRAM traffic, but on a B200
- * the two passes take less time for the per-token gradient, so moe_top1_bwd uses
- * them by default; moe_top1_bwd_mean_collapse uses the single pass at H = 256,
- * where it is the faster. This bit requests the single pass in both calls. The
+ * dW / db). The single pass moves about a third less DRAM traffic. On a B200 it is
+ * the faster at H = 128 above 65,536 tokens, and for the horizon-mean gradient at
+ * H = 256, so both calls take it there by default and the two passes elsewhere
+ * (at H = 256 the two passes are the faster for the per-token gradient). This bit
+ * requests the single pass in both calls at every size. The
  * two strategies add the dW / db partial sums in different fixed orders: each is
  * bitwise reproducible, and they agree to fp32 rounding. Ignored for FFMA. */
 #define MOE_BWD_SINGLE_PASS 0x100u

@@ -72,7 +72,7 @@ def test_traffic_record_is_well_formed_and_keyed_to_the_sources():
             # once per pass (about 1.24 at this shape), the single pass once
             hi = 1.35 if (call == "bwd" and rec["bwd_passes"] == 2) else 1.1
             assert 0.85 < v / per[call] < hi, (grad, call, v / per[call])
-        assert rec["bwd_passes"] == bench.bwd_passes("tf32", grad, LARGE.H)
+        assert rec["bwd_passes"] == bench.bwd_passes("tf32", grad, LARGE.H, LARGE.T)
     # the lookup refuses other workloads, the FFMA path and a gradient mode with no record
     assert bench.recorded_traffic("fwd", "mid_b16384_e8_h256", "tf32") is None
     assert bench.recorded_traffic("fwd", LARGE.name, "ffma") is None
