@@ -8,14 +8,11 @@
 
 namespace moe {
 
-// Tokens handled by one block of the routing kernels, and by one block of the
-// aux kernel: 256 up to kAuxSmallT tokens (more blocks, a shorter chain per
-// block), 1024 above (fewer per-block partial sums for the last block to add).
+// Tokens handled by one block of the routing kernels; the fewest tokens one
+// block of the aux kernel handles (the workspace has a partial-sum row for
+// every such block).
 constexpr int kRouteTokPerBlk = 1024;
-constexpr int kAuxTokPerBlkSmall = 256;
-constexpr int kAuxTokPerBlkLarge = 1024;
-constexpr int64_t kAuxSmallT = 262144;
-inline int aux_tok_per_blk(int64_t T) { return T <= kAuxSmallT ? kAuxTokPerBlkSmall : kAuxTokPerBlkLarge; }
+constexpr int kAuxMinTokPerBlk = 256;
 
 // Weight-gradient contraction: the expert-sorted token list is cut into
 // `wgrad_splits(T)` equal ranges (further cut at expert boundaries); range c
@@ -65,7 +62,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline WsLayout ws_layout(int64_t T, int E, int H) {
     WsLayout L;
     const int64_t nr = T > 0 ? (T + kRouteTokPerBlk - 1) / kRouteTokPerBlk : 1;
-    const int64_t na = T > 0 ? (T + aux_tok_per_blk(T) - 1) / aux_tok_per_blk(T) : 1;
+    const int64_t na = T > 0 ? (T + kAuxMinTokPerBlk - 1) / kAuxMinTokPerBlk : 1;
     const int P = wgrad_splits(T);
     size_t off = 0;
     L.flags = off;

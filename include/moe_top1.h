@@ -66,7 +66,7 @@ extern "C" {
  *    tokens; the weight-gradient ranges hold 128 tokens or more (256 before), so
  *    dW / db below 18,944 tokens sum in another fixed order; adds moe_aux_loss_fwd_bwd_lambda_update (the aux loss and the lambda update
  *    in one launch); the aux loss's per-block sums of p cover 256 tokens up to
- *    262,144 tokens (mean_p within fp32 rounding of version 5 there). */
+ *    131,072 tokens (mean_p within fp32 rounding of version 5 there). */
 #define MOE_TOP1_ABI_VERSION 6
 
 typedef enum {

@@ -111,7 +111,7 @@ def test_closed_loop_follows_the_oracle_and_is_deterministic():
 
 
 AUX_CASES = [wl.WORKLOADS["tiny_b8_e4_h128"], wl.WORKLOADS["skewed_b4096_e8_h128"],
-             wl.make_spec("aux_b52429_h5_e5", 52429, 5, 5, 32, 405),  # 1024-token blocks, rows moved per float
+             wl.make_spec("aux_b26215_h5_e5", 26215, 5, 5, 32, 405),  # 1024-token blocks, rows moved per float
              wl.make_spec("aux_empty_b0_e3", 0, 5, 3, 32, 406)]
 
 

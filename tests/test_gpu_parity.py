@@ -296,13 +296,13 @@ def test_deterministic_bitwise(math_mode, name):
         assert a[k].tobytes() == b[k].tobytes(), k
 
 
-@pytest.mark.parametrize("B,N_H,E", [(65536, 4, 8), (52429, 5, 5), (52429, 5, 16), (52429, 5, 32)])
+@pytest.mark.parametrize("B,N_H,E", [(32768, 4, 8), (26215, 5, 5), (26215, 5, 16), (26215, 5, 32)])
 def test_aux_around_the_block_size_switch(B, N_H, E):
-    """The aux kernel takes 256-token blocks up to 262,144 tokens and 1024-token
-    blocks above. 262,144 tokens is the last count with the small blocks (1024 of
-    them); 262,145 is the first with the large ones, and its last block holds one
-    token. Routing and aux against the oracle, at every expert-row width (E = 5
-    moves rows one float at a time)."""
+    """The aux kernel takes 256-token blocks up to 131,072 tokens and 1024-token
+    blocks above. 131,072 tokens is the last count with the small blocks (512 of
+    them); 131,075 is past the switch, and its last block holds three tokens.
+    Routing and aux against the oracle, at every expert-row width (E = 5 moves
+    rows one float at a time)."""
     inp = wl.generate(wl.make_spec(f"aux_b{B}_h{N_H}_e{E}", B, N_H, E, 32, 400 + E))
     lam = lam_of(inp)
     g = run_gpu(inp, ops.MOE_MATH_FFMA, lam, parts=("route", "aux"))
