@@ -322,6 +322,12 @@ moe_status_t aux_impl(const float* gate_logits, const int32_t* counts, int64_t B
         const Range ema[1] = {{next.ent_ema, sizeof(float)}};
         if (any_alias(outs, 4, ema, 1)) return MOE_ERR_ALIAS;
     }
+    // the kernel writes the workspace (per-block sums, ticket) while other blocks
+    // still read the inputs: none of them may lie inside it
+    const Range wsr{workspace, workspace ? workspace_bytes : 0};
+    if (overlap(wsr, ins[0]) || overlap(wsr, ins[1]) || overlap(wsr, {lambda_eff, sizeof(float)}) ||
+        (next.out && overlap(wsr, {next.ent_ema, sizeof(float)})))
+        return MOE_ERR_ALIAS;
     const WsLayout L = ws_layout(T, E, 0);
     if (!workspace) return MOE_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;

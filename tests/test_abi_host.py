@@ -176,6 +176,8 @@ def test_aux_with_lambda_update_rejects_bad_arguments(L):
     assert call(nxt=cnt) == ALIAS                       # next lambda on counts
     assert call(lam=mp, nxt=mp) == ALIAS                # lambda_eff (written) on mean_p
     assert call(ema=d) == ALIAS                         # ent_ema inside d_logits
+    assert call(ema=_p(A + 0x40000100)) == ALIAS        # ent_ema inside the workspace
+    assert call(lam=_p(A + 0x40000100)) == ALIAS        # lambda_eff inside the workspace
     assert call(wsb=16) == WORKSPACE                    # separate buffers
     assert call(nxt=lam, wsb=16) == WORKSPACE           # next lambda replaces lambda_eff
     assert call(nxt=ema, wsb=16) == WORKSPACE           # next lambda replaces ent_ema
