@@ -289,7 +289,9 @@ moe_status_t moe_top1_bwd_mean_collapse(const float* x, const float* W, const fl
  * may be NULL) and, if stats is not NULL, stats [3E + 4] = frac[E], mean_p[E],
  * counts[E] (as float), aux_raw, lambda, H(frac), H(mean_p) where
  * H(q) = -sum q ln q (0 ln 0 = 0). T = 0 gives zeros everywhere. counts must be
- * the routing of the same tokens. Needs the workspace.
+ * the routing of the same tokens. Needs the workspace; gate_logits, counts and
+ * lambda_eff must not lie inside it (the kernel writes it while they are read:
+ * MOE_ERR_ALIAS).
  */
 moe_status_t moe_aux_loss_fwd_bwd(const float* gate_logits, const int32_t* counts, int64_t B,
                                   int64_t N_H, int32_t E, const float* lambda_eff,
@@ -304,7 +306,8 @@ moe_status_t moe_aux_loss_fwd_bwd(const float* gate_logits, const int32_t* count
  *   *lambda_next = lambda_floor + lambda_max_extra * max(0, ent_target - *ent_ema) / ent_target
  * is written by the block that finishes last, after every block has read
  * lambda_eff. lambda_next may be lambda_eff (the weight for the next step replaces
- * this step's) or ent_ema, and must not overlap any other output. Arguments,
+ * this step's) or ent_ema, and must not overlap any other output; ent_ema must not
+ * lie inside the workspace. Arguments,
  * requirements and errors are those of the two calls; every bit of every output
  * is the same as theirs.
  */
