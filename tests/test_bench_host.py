@@ -83,3 +83,27 @@ def test_traffic_scaling_rule():
     # fixed part kept, token part times the ratio
     assert bench.scale_traffic(1000, 100, 4) == 100 + 900 * 4
     assert bench.scale_traffic(100, 100, 4) == 100
+
+
+def test_backward_strategy_rule_agrees_across_the_library_and_the_python_side():
+    """The default TF32 backward strategy is decided in the library
+    (bwd_single_pass_default in csrc/internal.h); the benchmark's pass count and
+    the gate's launch count restate it. All three must agree: one pass for the
+    horizon-mean gradient at H = 256 and at H = 128 above the library's threshold."""
+    import re
+    from bwd_route_b200 import ops
+    from bwd_route_b200.gate import MoETop1Gate
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = open(os.path.join(root, "bwd_route_b200", "csrc", "internal.h")).read()
+    limit = int(re.search(r"constexpr int64_t kBwdSinglePassMinT128 = (\d+);", src).group(1))
+    assert "return (collapse && H == 256) || (H == 128 && T > kBwdSinglePassMinT128);" in src
+    for H in (128, 256):
+        for T in (1, limit - 1, limit, limit + 1, 4 * limit):
+            for grad in ("token", "mean_collapse"):
+                collapse = grad == "mean_collapse"
+                lib = (collapse and H == 256) or (H == 128 and T > limit)
+                assert bench.bwd_passes("tf32", grad, H, T) == (1 if lib else 2), (H, T, grad)
+                assert bench.bwd_passes("ffma", grad, H, T) == 2
+                n_tf32 = MoETop1Gate.launches_per_step(ops.MOE_MATH_TF32, H, T, 8, collapse)
+                n_ffma = MoETop1Gate.launches_per_step(ops.MOE_MATH_FFMA, H, T, 8, collapse)
+                assert n_ffma - n_tf32 == (1 if lib else 0), (H, T, grad)
