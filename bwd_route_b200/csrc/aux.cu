@@ -76,8 +76,11 @@ __device__ __forceinline__ void write_lambda_next(const LambdaNext& next) {
 // block barrier for the data), lane t computes token t of each chunk reading
 // its row as float4s, and the gradients go back out with 128-bit stores. When
 // E is not a multiple of 4 the rows are moved one float at a time.
+// With four chunks per warp and rows of at most 8 experts a block holds 32 KB of
+// shared memory, so 7 blocks fit an SM if each thread keeps to 32 registers: the
+// 1024 blocks of 1,048,576 tokens then run in one wave instead of two.
 template <int EMAX, int kChunksPerWarp>
-__global__ void __launch_bounds__(kThreads) aux_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(kThreads, (kChunksPerWarp == 4 && EMAX <= 8) ? 7 : 1) aux_kernel(const float* __restrict__ logits,
                                                       const int32_t* __restrict__ counts, int64_t T, int E,
                                                       const float* lambda_eff,
                                                       float* __restrict__ d_logits, float* __restrict__ blk_psum,
